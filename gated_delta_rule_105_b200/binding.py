@@ -1,0 +1,171 @@
+"""Thin Python binding over libgdn's C ABI (argument marshalling only).
+
+Every step of the forward pass runs in libgdn's CUDA kernels; this module only checks torch tensors,
+allocates outputs with torch and passes raw pointers and the current CUDA stream.  There is no CPU
+fallback: without the built library or a CUDA device every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, GDN_ERR_DEVICE_ARG = range(6)
+GDN_F32, GDN_BF16 = 0, 1
+KERNELS = {"auto": 0, "simt": 1, "tc": 2}
+KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
+
+_lib = None
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"libgdn status {status}: {msg}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libgdn.so and declare its signatures.  Raises if the library has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libgdn.so not found at {path}: build it with "
+                           "`python -m gated_delta_rule_105_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    vp, fp, i, f, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.gdn_workspace_bytes.argtypes = [i] * 7
+    lib.gdn_workspace_bytes.restype = sz
+    lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [i] * 7 + [vp, i, vp, sz, vp]
+    lib.gdn_chunk_fwd.restype = i
+    lib.gdn2_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, f, fp, vp, fp] + [i] * 7 + [vp, i, vp, sz, vp]
+    lib.gdn2_chunk_fwd.restype = i
+    lib.gdn_set_kernel.argtypes = [i]
+    lib.gdn_set_kernel.restype = i
+    lib.gdn_last_kernel.argtypes = []
+    lib.gdn_last_kernel.restype = i
+    lib.gdn_check_error.argtypes = [vp]
+    lib.gdn_check_error.restype = i
+    lib.gdn_status_string.argtypes = [i]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_last_error.argtypes = []
+    lib.gdn_last_error.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _raise_on(status: int):
+    if status != GDN_OK:
+        lib = load_library()
+        raise GdnError(status, f"{lib.gdn_status_string(status).decode()}: {lib.gdn_last_error().decode()}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_dev(name, t, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libgdn has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return GDN_F32
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    raise ValueError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def set_kernel(name: str) -> None:
+    """Select the kernel family ("auto", "simt" or "tc") for later calls (process-wide)."""
+    _raise_on(load_library().gdn_set_kernel(KERNELS[name]))
+
+
+def last_kernel() -> str:
+    return KERNEL_NAMES[load_library().gdn_last_kernel()]
+
+
+def check_error(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel reported a device-side error."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    _raise_on(load_library().gdn_check_error(ctypes.c_void_p(s.cuda_stream)))
+
+
+def _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state):
+    _check_dev("q", q)
+    dt = q.dtype
+    _check_dev("k", k, dt)
+    _check_dev("v", v, dt)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k must be [B,T,H,dk] and v [B,T,H,dv] with matching B, T, H")
+    n_seq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None:
+        _check_dev("cu_seqlens", cu_seqlens, torch.int32)
+    _check_dev("h0", h0, torch.float32)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
+    if hT is None and output_final_state:
+        hT = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=q.device)
+    return B, T, H, dk, dv, n_seq, o, hT
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, output_final_state=True, cu_seqlens=None, BT=64,
+                  o=None, hT=None):
+    """Chunked gated delta rule forward through ``gdn_chunk_fwd`` of the C ABI.
+
+    q, k [B,T,H,dk] and v [B,T,H,dv] (fp32 or bf16), g, beta [B,T,H] fp32, h0 [N,H,dk,dv] fp32 or None,
+    cu_seqlens int32 [N+1] (B == 1) or None.  Returns (o [B,T,H,dv] in q's dtype, hT [N,H,dk,dv] fp32).
+    """
+    B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state)
+    _check_dev("g", g, torch.float32)
+    _check_dev("beta", beta, torch.float32)
+    if g.shape != (B, T, H) or beta.shape != (B, T, H):
+        raise ValueError("g and beta must be [B,T,H]")
+    scale = dk ** -0.5 if scale is None else float(scale)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    st = load_library().gdn_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(o), _ptr(hT),
+        B, T, H, dk, dv, BT, _dtype_code(q), _ptr(cu_seqlens), 0 if cu_seqlens is None else n_seq,
+        None, 0, ctypes.c_void_p(stream))
+    _raise_on(st)
+    return o, hT
+
+
+def gdn2_chunk_fwd(q, k, v, g, b, w, scale=None, h0=None, output_final_state=True, cu_seqlens=None, BT=64,
+                   o=None, hT=None):
+    """Gated Delta Rule-2 forward through ``gdn2_chunk_fwd`` of the C ABI.
+
+    g (per-channel log-decay) and b (erase gate) are [B,T,H,dk] fp32, w (write gate) is [B,T,H,dv] fp32.
+    """
+    B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state)
+    for name, t, shape in (("g", g, (B, T, H, dk)), ("b", b, (B, T, H, dk)), ("w", w, (B, T, H, dv))):
+        _check_dev(name, t, torch.float32)
+        if t.shape != shape:
+            raise ValueError(f"{name} must be {list(shape)}")
+    scale = dk ** -0.5 if scale is None else float(scale)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    st = load_library().gdn2_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), scale, _ptr(h0), _ptr(o), _ptr(hT),
+        B, T, H, dk, dv, BT, _dtype_code(q), _ptr(cu_seqlens), 0 if cu_seqlens is None else n_seq,
+        None, 0, ctypes.c_void_p(stream))
+    _raise_on(st)
+    return o, hT
+
+
+def chunk_gated_delta_rule(q, k, v, g, beta, scale=None, initial_state=None, output_final_state=True,
+                           cu_seqlens=None):
+    """The token mixer call by the name the pages use; same as :func:`gdn_chunk_fwd`."""
+    return gdn_chunk_fwd(q, k, v, g, beta, scale, initial_state, output_final_state, cu_seqlens)

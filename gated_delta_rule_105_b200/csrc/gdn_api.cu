@@ -1,0 +1,188 @@
+// libgdn C ABI: host-side argument checks, kernel selection and launches.  Every kernel of the library
+// is included here so that they share one device error word without relocatable device code.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+
+#include "gdn.h"
+#include "gdn_common.cuh"
+#include "gdn_simt.cuh"
+#include "gdn_tc.cuh"
+
+namespace gdn {
+
+__device__ unsigned int g_err_word;
+
+static thread_local char t_msg[512];
+static thread_local gdn_kernel t_last_kernel = GDN_KERNEL_AUTO;
+static std::atomic<int> g_kernel_choice{GDN_KERNEL_AUTO};
+
+static gdn_status fail(gdn_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_msg, sizeof(t_msg), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static unsigned* err_word_ptr(gdn_status* st) {
+    unsigned* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_err_word);
+    if (e != cudaSuccess) {
+        *st = fail(GDN_ERR_CUDA, "cudaGetSymbolAddress(error word): %s", cudaGetErrorString(e));
+        return nullptr;
+    }
+    *st = GDN_OK;
+    return ptr;
+}
+
+// Host checks shared by both operations.  Nothing touches the device before these pass.
+static gdn_status check_common(const void* q, const void* k, const void* v, const float* g, const float* gate,
+                               const float* w, bool gdn2, float scale, const float* h0, const void* o,
+                               const float* hT, int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt,
+                               const int32_t* cu, int n_seqs, void* ws, size_t ws_bytes, int* n_seq_out) {
+    t_msg[0] = 0;
+    if (T > 0 && (!q || !k || !v || !g || !gate || !o || (gdn2 && !w)))
+        return fail(GDN_ERR_INVALID_ARG, "a required pointer (q, k, v, g, %s, o%s) is NULL",
+                    gdn2 ? "b" : "beta", gdn2 ? ", w" : "");
+    const void* ptrs[] = {q, k, v, g, gate, w, h0, o, hT, cu, ws};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return fail(GDN_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", ptr);
+    if (B < 1 || H < 1 || T < 0) return fail(GDN_ERR_INVALID_ARG, "need B >= 1, H >= 1, T >= 0 (got %d, %d, %d)", B, H, T);
+    if (BT != kChunk) return fail(GDN_ERR_UNSUPPORTED, "BT must be %d (got %d)", kChunk, BT);
+    if (dk != 64 && dk != 128) return fail(GDN_ERR_UNSUPPORTED, "dk must be 64 or 128 (got %d)", dk);
+    if (dv < 64 || dv > 256 || dv % 64 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "dv must be a multiple of 64 in [64, 256] (got %d)", dv);
+    if (dt != GDN_F32 && dt != GDN_BF16) return fail(GDN_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
+    if (!std::isfinite(scale)) return fail(GDN_ERR_INVALID_ARG, "scale is not finite");
+    if (ws_bytes > 0 && !ws) return fail(GDN_ERR_INVALID_ARG, "ws_bytes > 0 with a NULL workspace");
+    if (cu) {
+        if (B != 1) return fail(GDN_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (got %d)", B);
+        if (n_seqs < 1 || n_seqs > 65535) return fail(GDN_ERR_INVALID_ARG, "n_seqs must be in [1, 65535] (got %d)", n_seqs);
+        *n_seq_out = n_seqs;
+    } else {
+        if (n_seqs != 0 && n_seqs != B)
+            return fail(GDN_ERR_INVALID_ARG, "without cu_seqlens n_seqs must be 0 or B (got %d)", n_seqs);
+        if (B > 65535) return fail(GDN_ERR_INVALID_ARG, "B must be <= 65535 (got %d)", B);
+        *n_seq_out = B;
+    }
+    if (H > 65535) return fail(GDN_ERR_INVALID_ARG, "H must be <= 65535 (got %d)", H);
+    const double elems = (double)B * T * H * (dk > dv ? dk : dv);
+    if (elems > 9.0e15) return fail(GDN_ERR_INVALID_ARG, "tensor too large");
+    return GDN_OK;
+}
+
+template <typename TIn, int DK, bool GDN2>
+static gdn_status launch_simt_dk(const FwdParams& p, unsigned* err, cudaStream_t stream) {
+    using L = SimtSmem<DK, kSimtDVT, GDN2>;
+    auto kern = gdn_simt_fwd_kernel<TIn, DK, kSimtDVT, GDN2>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    dim3 grid(p.dv / kSimtDVT, p.H, p.n_seq);
+    kern<<<grid, kSimtThreads, L::bytes, stream>>>(p, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "SIMT kernel launch: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+template <bool GDN2>
+static gdn_status launch_simt(const FwdParams& p, gdn_dtype dt, unsigned* err, cudaStream_t stream) {
+    if (dt == GDN_F32)
+        return p.dk == 64 ? launch_simt_dk<float, 64, GDN2>(p, err, stream)
+                          : launch_simt_dk<float, 128, GDN2>(p, err, stream);
+    return p.dk == 64 ? launch_simt_dk<__nv_bfloat16, 64, GDN2>(p, err, stream)
+                      : launch_simt_dk<__nv_bfloat16, 128, GDN2>(p, err, stream);
+}
+
+static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, cudaStream_t stream) {
+    const int choice = g_kernel_choice.load();
+    const bool tc_ok = dt == GDN_BF16 && tc_supported(p, gdn2);
+    if (choice == GDN_KERNEL_TC && !tc_ok)
+        return fail(GDN_ERR_UNSUPPORTED, "the tcgen05 kernel needs bf16 inputs and a supported shape");
+    gdn_status st;
+    unsigned* err = err_word_ptr(&st);
+    if (!err) return st;
+    if (p.n_seq == 0 || p.H == 0) return GDN_OK;
+    const bool use_tc = tc_ok && choice != GDN_KERNEL_SIMT;
+    if (use_tc) {
+        st = launch_tc(p, gdn2, err, stream);
+        if (st == GDN_OK) t_last_kernel = GDN_KERNEL_TC;
+        else if (st == GDN_ERR_CUDA) fail(st, "tcgen05 kernel launch: %s", tc_last_error());
+        return st;
+    }
+    st = gdn2 ? launch_simt<true>(p, dt, err, stream) : launch_simt<false>(p, dt, err, stream);
+    if (st == GDN_OK) t_last_kernel = GDN_KERNEL_SIMT;
+    return st;
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+size_t gdn_workspace_bytes(int, int, int, int, int, int, int) { return 0; }
+
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         float scale, const float* h0, void* o, float* hT, int B, int T, int H, int dk, int dv,
+                         int BT, gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs, void* workspace,
+                         size_t ws_bytes, cudaStream_t stream) {
+    int n_seq = 0;
+    gdn_status st = check_common(q, k, v, g, beta, nullptr, false, scale, h0, o, hT, B, T, H, dk, dv, BT, dt,
+                                 cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
+    if (st != GDN_OK) return st;
+    FwdParams p{q, k, v, g, beta, nullptr, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
+    return run(p, false, dt, stream);
+}
+
+gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* b,
+                          const float* w, float scale, const float* h0, void* o, float* hT, int B, int T, int H,
+                          int dk, int dv, int BT, gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs,
+                          void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    int n_seq = 0;
+    gdn_status st = check_common(q, k, v, g, b, w, true, scale, h0, o, hT, B, T, H, dk, dv, BT, dt, cu_seqlens,
+                                 n_seqs, workspace, ws_bytes, &n_seq);
+    if (st != GDN_OK) return st;
+    FwdParams p{q, k, v, g, b, w, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
+    return run(p, true, dt, stream);
+}
+
+gdn_status gdn_set_kernel(gdn_kernel kernel) {
+    if (kernel != GDN_KERNEL_AUTO && kernel != GDN_KERNEL_SIMT && kernel != GDN_KERNEL_TC)
+        return fail(GDN_ERR_INVALID_ARG, "unknown kernel family %d", (int)kernel);
+    g_kernel_choice.store(kernel);
+    return GDN_OK;
+}
+
+gdn_kernel gdn_last_kernel(void) { return t_last_kernel; }
+
+gdn_status gdn_check_error(cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+    unsigned word = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&word, g_err_word, sizeof(word));
+    if (e == cudaSuccess && word) e = cudaMemcpyToSymbol(g_err_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "error word: %s", cudaGetErrorString(e));
+    if (word & kErrTimeout) return fail(GDN_ERR_TIMEOUT, "a bounded device wait ran out (word 0x%x)", word);
+    if (word & kErrSeqlens) return fail(GDN_ERR_DEVICE_ARG, "cu_seqlens out of order or out of range (word 0x%x)", word);
+    return GDN_OK;
+}
+
+const char* gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case GDN_ERR_CUDA: return "CUDA error";
+        case GDN_ERR_TIMEOUT: return "device wait timed out";
+        case GDN_ERR_DEVICE_ARG: return "invalid cu_seqlens seen on the device";
+    }
+    return "unknown status";
+}
+
+const char* gdn_last_error(void) { return t_msg; }
+
+}  // extern "C"

@@ -1,0 +1,291 @@
+// SIMT (fp32 FMA) chunked forward kernel for GDN and GDN-2.
+//
+// One CTA owns one (sequence n, head h, block of DVT value columns) and walks that sequence's chunks of
+// 64 tokens in order, keeping its DK x DVT slice of the state in shared memory (fp32).  The value columns
+// of the state never interact (every update is a left-multiplication on the key axis plus a rank-one
+// write), so slicing dv across CTAs is exact.  All arithmetic is fp32 on CUDA cores: this is the path
+// for fp32 inputs (tensor-core operand rounding would exceed a 1e-4 error budget) and the simple
+// reference path for bf16 inputs.
+//
+// Per chunk (rows r, s < 64; zero rows pad a partial chunk, which makes them inert: k = v = 0,
+// beta = b = w = 0 and g = 0 so the padded cumulative gate stays at the last real token's value):
+//   G_r   = log2(e) * sum_{s<=r} g_s                           (GDN-2: per key channel)
+//   A_rs  = beta_r (k_r . k_s) 2^(G_r - G_s)        s < r      (GDN-2: sum_i b_ri k_ri k_si 2^(G_ri - G_si))
+//   P_rs  = (q_r . k_s) 2^(G_r - G_s)               s <= r     (GDN-2: per-channel factor inside the sum)
+//   Tm    = (I + A)^-1                               forward substitution, one column per thread
+//   X     = beta V - diag(beta 2^G) K h              (GDN-2: w.V - (b.2^G.K) h)
+//   U     = Tm X
+//   O     = scale [ (Q . 2^G) h + P U ]
+//   h    <- 2^(G_last) h + (K . 2^(G_last - G))^T U  (GDN-2: Diag(2^G_last) h + (K . 2^(G_last - G))^T U)
+// This is the WY form of the intra-chunk dependency and the chunk-to-chunk state pass described in the
+// GatedDeltaNet data-flow walkthrough (yfxerp.com/news/367755), section "Chunked parallelism", and for
+// GDN-2 in the Gated DeltaNet-2 article (7minutos.es), section "Entrenamiento fragmentado".
+#pragma once
+
+#include "gdn_common.cuh"
+
+namespace gdn {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSimtDVT = 32;  // value columns per CTA
+
+template <int DK, int DVT, bool GDN2>
+struct SimtSmem {
+    static constexpr int LDK = DK + 1;  // padded row stride: conflict-free column walks
+    static constexpr int LDT = kChunk + 1;
+    static constexpr int nK = kChunk * LDK;
+    static constexpr int oK = 0;                       // K [64][LDK]
+    static constexpr int oQ = oK + nK;                 // Q, then Q.2^G (GDN-2)
+    static constexpr int oBK = oQ + nK;                // GDN-2: b.K, then b.K.2^G, then K.2^(G_last-G)
+    static constexpr int oG = oBK + (GDN2 ? nK : 0);   // GDN-2: cumulative gate per channel
+    static constexpr int oV = oG + (GDN2 ? nK : 0);    // scaled V, then X
+    static constexpr int oU = oV + kChunk * DVT;       // U
+    static constexpr int oH = oU + kChunk * DVT;       // state slice [DK][DVT]
+    static constexpr int oA = oH + DK * DVT;           // A [64][LDT]
+    static constexpr int oT = oA + kChunk * LDT;       // (I+A)^-1
+    static constexpr int oP = oT + kChunk * LDT;       // P
+    static constexpr int oG1 = oP + kChunk * LDT;      // GDN: cumulative gate [64]
+    static constexpr int oB1 = oG1 + kChunk;           // GDN: beta [64]
+    static constexpr int oF = oB1 + kChunk;            // GDN: 2^(G_last - G_s) [64]
+    static constexpr int total = oF + kChunk;
+    static constexpr size_t bytes = sizeof(float) * (size_t)total;
+};
+
+template <typename TIn, int DK, int DVT, bool GDN2>
+__global__ void __launch_bounds__(kSimtThreads)
+gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
+    using L = SimtSmem<DK, DVT, GDN2>;
+    constexpr int LDK = L::LDK, LDT = L::LDT, NT = kSimtThreads;
+    constexpr int PER = kChunk * DVT / NT;  // (row, column) outputs per thread
+    static_assert(kChunk * DVT % NT == 0, "tile must divide evenly");
+    extern __shared__ float sm[];
+    float* sK = sm + L::oK;
+    float* sQ = sm + L::oQ;
+    float* sBK = sm + L::oBK;
+    float* sG = sm + L::oG;
+    float* sV = sm + L::oV;
+    float* sU = sm + L::oU;
+    float* sH = sm + L::oH;
+    float* sA = sm + L::oA;
+    float* sT = sm + L::oT;
+    float* sP = sm + L::oP;
+    float* sG1 = sm + L::oG1;
+    float* sB1 = sm + L::oB1;
+    float* sF = sm + L::oF;
+
+    const int tid = threadIdx.x;
+    const int j0 = blockIdx.x * DVT;
+    const int h = blockIdx.y;
+    const int n = blockIdx.z;
+    const int H = p.H, dv = p.dv, T = p.T;
+    const TIn* __restrict__ q = static_cast<const TIn*>(p.q);
+    const TIn* __restrict__ k = static_cast<const TIn*>(p.k);
+    const TIn* __restrict__ v = static_cast<const TIn*>(p.v);
+    TIn* __restrict__ o = static_cast<TIn*>(p.o);
+
+    int row, bos, eos;
+    if (p.cu_seqlens) {
+        row = 0;
+        bos = p.cu_seqlens[n];
+        eos = p.cu_seqlens[n + 1];
+        if (bos < 0 || eos < bos || eos > T) {
+            if (tid == 0) atomicOr(err, kErrSeqlens);
+            return;
+        }
+    } else {
+        row = n;
+        bos = 0;
+        eos = T;
+    }
+
+    const size_t state_base = ((size_t)n * H + h) * DK * (size_t)dv + j0;
+    for (int e = tid; e < DK * DVT; e += NT) {
+        const int i = e / DVT, j = e % DVT;
+        sH[e] = p.h0 ? p.h0[state_base + (size_t)i * dv + j] : 0.f;
+    }
+
+    for (int c0 = bos; c0 < eos; c0 += kChunk) {
+        const int Lc = min(kChunk, eos - c0);
+        __syncthreads();  // the previous chunk is done with every buffer
+        // ---- load the chunk (zero-padded past Lc)
+        for (int e = tid; e < kChunk * DK; e += NT) {
+            const int r = e / DK, i = e % DK;
+            float kv = 0.f, qv = 0.f, gv = 0.f, bv = 0.f;
+            if (r < Lc) {
+                const size_t tok = ((size_t)row * T + c0 + r) * H + h;
+                kv = to_f32(k[tok * DK + i]);
+                qv = to_f32(q[tok * DK + i]);
+                if (GDN2) {
+                    gv = p.g[tok * DK + i];
+                    bv = p.beta[tok * DK + i];
+                }
+            }
+            sK[r * LDK + i] = kv;
+            sQ[r * LDK + i] = qv;
+            if (GDN2) {
+                sG[r * LDK + i] = gv;
+                sBK[r * LDK + i] = bv * kv;
+            }
+        }
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int r = e / DVT, j = e % DVT;
+            float x = 0.f;
+            if (r < Lc) {
+                const size_t tok = ((size_t)row * T + c0 + r) * H + h;
+                const float vv = to_f32(v[tok * dv + j0 + j]);
+                x = GDN2 ? p.w[tok * dv + j0 + j] * vv : p.beta[tok] * vv;
+            }
+            sV[e] = x;
+        }
+        if (!GDN2 && tid < kChunk) {
+            const int r = tid;
+            const size_t tok = ((size_t)row * T + c0 + r) * H + h;
+            sG1[r] = r < Lc ? p.g[tok] : 0.f;
+            sB1[r] = r < Lc ? p.beta[tok] : 0.f;
+        }
+        __syncthreads();
+        // ---- chunk-local cumulative gate, base 2
+        if (GDN2) {
+            for (int i = tid; i < DK; i += NT) {
+                float acc = 0.f;
+                for (int r = 0; r < kChunk; ++r) {
+                    acc += sG[r * LDK + i];
+                    sG[r * LDK + i] = acc * kLog2e;
+                }
+            }
+        } else if (tid == 0) {
+            float acc = 0.f;
+            for (int r = 0; r < kChunk; ++r) {
+                acc += sG1[r];
+                sG1[r] = acc * kLog2e;
+            }
+        }
+        __syncthreads();
+        // ---- A (strictly lower) and P (lower incl. diagonal)
+        for (int e = tid; e < kChunk * kChunk; e += NT) {
+            const int r = e / kChunk, s = e % kChunk;
+            float a = 0.f, pp = 0.f;
+            if (s <= r) {
+                if (GDN2) {
+                    for (int i = 0; i < DK; ++i) {
+                        const float f = exp2f(sG[r * LDK + i] - sG[s * LDK + i]);
+                        const float ks = sK[s * LDK + i] * f;
+                        a = fmaf(sBK[r * LDK + i], ks, a);
+                        pp = fmaf(sQ[r * LDK + i], ks, pp);
+                    }
+                } else {
+                    float dkk = 0.f, dqk = 0.f;
+                    for (int i = 0; i < DK; ++i) {
+                        const float ks = sK[s * LDK + i];
+                        dkk = fmaf(sK[r * LDK + i], ks, dkk);
+                        dqk = fmaf(sQ[r * LDK + i], ks, dqk);
+                    }
+                    const float f = exp2f(sG1[r] - sG1[s]);
+                    a = sB1[r] * f * dkk;
+                    pp = f * dqk;
+                }
+                if (s == r) a = 0.f;
+            }
+            sA[r * LDT + s] = a;
+            sP[r * LDT + s] = pp;
+        }
+        __syncthreads();
+        // ---- GDN-2: fold 2^G into Q and b.K (in place); (I + A)^-1 by forward substitution
+        if (GDN2) {
+            for (int e = tid; e < kChunk * DK; e += NT) {
+                const int r = e / DK, i = e % DK;
+                const float f = exp2f(sG[r * LDK + i]);
+                sQ[r * LDK + i] *= f;
+                sBK[r * LDK + i] *= f;
+            }
+        }
+        if (tid < kChunk) {
+            const int c = tid;
+            for (int r = 0; r < c; ++r) sT[r * LDT + c] = 0.f;
+            for (int r = c; r < kChunk; ++r) {
+                float t = (r == c) ? 1.f : 0.f;
+                for (int s = c; s < r; ++s) t = fmaf(-sA[r * LDT + s], sT[s * LDT + c], t);
+                sT[r * LDT + c] = t;
+            }
+        }
+        __syncthreads();
+        // ---- X = (scaled V) - (erase-side keys . 2^G) h ;  Oi = (Q . 2^G) h  (kept in registers)
+        float oi[PER];
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+            const int e = tid + m * NT;
+            const int r = e / DVT, j = e % DVT;
+            float kh = 0.f, qh = 0.f;
+            if (GDN2) {
+                for (int i = 0; i < DK; ++i) {
+                    const float hv = sH[i * DVT + j];
+                    kh = fmaf(sBK[r * LDK + i], hv, kh);
+                    qh = fmaf(sQ[r * LDK + i], hv, qh);
+                }
+                sV[e] -= kh;
+                oi[m] = qh;
+            } else {
+                for (int i = 0; i < DK; ++i) {
+                    const float hv = sH[i * DVT + j];
+                    kh = fmaf(sK[r * LDK + i], hv, kh);
+                    qh = fmaf(sQ[r * LDK + i], hv, qh);
+                }
+                const float f = exp2f(sG1[r]);
+                sV[e] -= sB1[r] * f * kh;
+                oi[m] = f * qh;
+            }
+        }
+        __syncthreads();
+        // ---- U = (I+A)^-1 X ; decay factors for the state update
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+            const int e = tid + m * NT;
+            const int r = e / DVT, j = e % DVT;
+            float u = 0.f;
+            for (int s = 0; s <= r; ++s) u = fmaf(sT[r * LDT + s], sV[s * DVT + j], u);
+            sU[e] = u;
+        }
+        if (GDN2) {
+            for (int e = tid; e < kChunk * DK; e += NT) {
+                const int s = e / DK, i = e % DK;
+                sBK[s * LDK + i] = sK[s * LDK + i] * exp2f(sG[(kChunk - 1) * LDK + i] - sG[s * LDK + i]);
+            }
+        } else if (tid < kChunk) {
+            sF[tid] = exp2f(sG1[kChunk - 1] - sG1[tid]);
+        }
+        __syncthreads();
+        // ---- O = scale (Oi + P U) ; h <- 2^G_last h + Ktilde^T U
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+            const int e = tid + m * NT;
+            const int r = e / DVT, j = e % DVT;
+            float acc = oi[m];
+            for (int s = 0; s <= r; ++s) acc = fmaf(sP[r * LDT + s], sU[s * DVT + j], acc);
+            if (r < Lc) {
+                const size_t tok = ((size_t)row * T + c0 + r) * H + h;
+                o[tok * dv + j0 + j] = from_f32<TIn>(p.scale * acc);
+            }
+        }
+        for (int e = tid; e < DK * DVT; e += NT) {
+            const int i = e / DVT, j = e % DVT;
+            float acc;
+            if (GDN2) {
+                acc = exp2f(sG[(kChunk - 1) * LDK + i]) * sH[e];
+                for (int s = 0; s < kChunk; ++s) acc = fmaf(sBK[s * LDK + i], sU[s * DVT + j], acc);
+            } else {
+                acc = exp2f(sG1[kChunk - 1]) * sH[e];
+                for (int s = 0; s < kChunk; ++s) acc = fmaf(sK[s * LDK + i] * sF[s], sU[s * DVT + j], acc);
+            }
+            sH[e] = acc;
+        }
+    }
+    __syncthreads();
+    if (p.hT) {
+        for (int e = tid; e < DK * DVT; e += NT) {
+            const int i = e / DVT, j = e % DVT;
+            p.hT[state_base + (size_t)i * dv + j] = sH[e];
+        }
+    }
+}
+
+}  // namespace gdn

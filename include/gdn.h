@@ -1,0 +1,110 @@
+/*
+ * libgdn -- chunked gated delta rule forward pass on NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * Operations
+ *   gdn_chunk_fwd   Gated delta rule (GDN): per (sequence, head), with state S (dk x dv, fp32),
+ *                     S_t = exp(g_t) S_{t-1} + k_t u_t^T,   u_t = beta_t v_t - beta_t exp(g_t) S_{t-1}^T k_t,
+ *                     o_t = scale * S_t^T q_t   (read after the write at t).
+ *                   Definition: GatedDeltaNet data-flow walkthrough (yfxerp.com/news/367755), section
+ *                   "Delta Rule: predict first, then correct" (the token-by-token reference loop); the
+ *                   chunked evaluation (BT = 64 tokens per chunk, one state handed between chunks, WY form
+ *                   of the intra-chunk dependency, gate cumsum times log2(e) so exp2 can be used) follows
+ *                   section "Chunked parallelism: how the Triton kernels turn serial into parallel".
+ *   gdn2_chunk_fwd  Gated Delta Rule-2 (GDN-2): per-channel decay alpha_t = exp(g_t) on the key axis,
+ *                   erase gate b_t on the key axis, write gate w_t on the value axis,
+ *                     S_t = (I - k_t (b_t . k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T,  o_t = scale S_t^T q_t.
+ *                   Definition: NVIDIA Gated DeltaNet-2 article (7minutos.es), section "Regla-2 del Delta
+ *                   cerrado: dos puertas en lugar de una"; chunk size C = 64 from section "Entrenamiento
+ *                   fragmentado".
+ *   The read-out o_t and scale = dk^-1/2 are not printed on the pages; o_t = scale S_t^T q_t is the adopted
+ *   reading (the same for both operations).
+ *
+ * Layouts (row-major, contiguous, all device pointers):
+ *   q, k        [B, T, H, dk]   dtype `dt` (GDN_F32 or GDN_BF16)
+ *   v, o        [B, T, H, dv]   dtype `dt`
+ *   GDN:   g, beta  [B, T, H]        fp32; g is the natural-log decay (g <= 0 expected), beta the write strength
+ *   GDN-2: g, b     [B, T, H, dk]    fp32 per-channel log-decay and erase gate;  w [B, T, H, dv] fp32 write gate
+ *   h0, hT      [N, H, dk, dv]  fp32, N = B, or n_seqs with cu_seqlens.  h0 == NULL means zeros;
+ *                               hT == NULL means the final state is not written.
+ *   cu_seqlens  int32 [n_seqs + 1] or NULL.  With cu_seqlens, B must be 1 and the T tokens of the single
+ *               row are n_seqs packed sequences [cu[n], cu[n+1]); the state starts from h0[n] at each
+ *               sequence start and chunks are aligned to the sequence start (the last may be partial).
+ *               cu[0] = 0, non-decreasing, cu[n_seqs] = T; a zero-length sequence gives hT[n] = h0[n].
+ *
+ * Supported shapes: BT == 64; dk in {64, 128}; dv a multiple of 64 in [64, 256]; B >= 1, H >= 1, T >= 0.
+ * Every pointer must be 16-byte aligned.  The library never allocates, frees or synchronises inside a
+ * *_fwd call: the caller owns every buffer, and work is enqueued on `stream` (asynchronous).
+ *
+ * Errors
+ *   Arguments are checked on the host before anything is enqueued; a failed check returns
+ *   GDN_ERR_INVALID_ARG (bad pointer, size, alignment) or GDN_ERR_UNSUPPORTED (a shape or option outside
+ *   the supported set) and has no side effects.  A failed launch returns GDN_ERR_CUDA.  Conditions only the
+ *   device can see (a cu_seqlens entry out of order or out of range; a bounded wait that ran out) set a
+ *   device error word instead of faulting; gdn_check_error() synchronises the stream and reports it.
+ *   gdn_last_error() returns a short description of the most recent failure on the calling thread.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,
+    GDN_ERR_UNSUPPORTED = 2,
+    GDN_ERR_CUDA = 3,
+    GDN_ERR_TIMEOUT = 4,
+    GDN_ERR_DEVICE_ARG = 5 /* reported by gdn_check_error: cu_seqlens out of order or out of range */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype; /* dtype of q, k, v, o */
+
+/* Kernel family used for a call.  AUTO picks the tensor-core (tcgen05) kernel for bf16 inputs when the
+ * shape allows it and the SIMT fp32 kernel otherwise.  SIMT forces the fp32-FMA kernel (any dtype); TC
+ * forces the tcgen05 kernel (bf16 only; GDN_ERR_UNSUPPORTED otherwise). */
+typedef enum { GDN_KERNEL_AUTO = 0, GDN_KERNEL_SIMT = 1, GDN_KERNEL_TC = 2 } gdn_kernel;
+
+/* Bytes of caller-provided device workspace a call with these sizes needs (0: pass NULL, 0). */
+size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs);
+
+/* Gated delta rule forward; see the header comment for the definition, layouts and errors. */
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         float scale, const float* h0, void* o, float* hT,
+                         int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt,
+                         const int32_t* cu_seqlens, int n_seqs,
+                         void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Gated Delta Rule-2 forward; g, b are [B,T,H,dk] and w is [B,T,H,dv], all fp32. */
+gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* b,
+                          const float* w, float scale, const float* h0, void* o, float* hT,
+                          int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt,
+                          const int32_t* cu_seqlens, int n_seqs,
+                          void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Selects the kernel family for later calls from any thread (process-wide; default AUTO). */
+gdn_status gdn_set_kernel(gdn_kernel kernel);
+
+/* Kernel family that the most recent successful *_fwd call on this thread launched. */
+gdn_kernel gdn_last_kernel(void);
+
+/* Synchronises `stream`, then reads and clears the device error word of the current device:
+ * GDN_OK, GDN_ERR_TIMEOUT, GDN_ERR_DEVICE_ARG, or GDN_ERR_CUDA if the stream reports a CUDA error. */
+gdn_status gdn_check_error(cudaStream_t stream);
+
+/* Static description of a status code. */
+const char* gdn_status_string(gdn_status status);
+
+/* Description of the most recent failure on the calling thread ("" if none). */
+const char* gdn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

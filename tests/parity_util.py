@@ -1,0 +1,96 @@
+"""Helpers shared by the parity tests: run the CUDA path and the fp64 oracle on the same inputs.
+
+Tolerance (stated for this method): max |x - x_ref| / rms(x_ref), separately for o and hT, at most
+1e-4 for fp32 inputs and 2e-2 for bf16 inputs with fp32 gates and state.
+"""
+import numpy as np
+import torch
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def relerr(x, ref):
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref ** 2))
+    return float(np.max(np.abs(x - ref)) / max(rms, 1e-30)) if ref.size else 0.0
+
+
+def f64(t):
+    return None if t is None else t.detach().to("cpu", torch.float64).numpy()
+
+
+def to_dev(inp, device="cuda"):
+    out = {}
+    for key, val in inp.items():
+        out[key] = val.to(device) if isinstance(val, torch.Tensor) else val
+    return out
+
+
+def run_cuda(inp, variant, output_final_state=True):
+    """Run the C ABI through the binding on device copies of ``inp``; returns (o, hT) on the device."""
+    from gated_delta_rule_105_b200 import gdn2_chunk_fwd, gdn_chunk_fwd
+    d = to_dev(inp)
+    if variant == "gdn":
+        return gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"],
+                             output_final_state, d["cu_seqlens"])
+    return gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["scale"], d["h0"],
+                          output_final_state, d["cu_seqlens"])
+
+
+def seq_spans(inp):
+    B, T = inp["q"].shape[:2]
+    cu = inp["cu_seqlens"]
+    if cu is None:
+        return [(b, 0, T) for b in range(B)]
+    cu = [int(x) for x in cu]
+    return [(0, cu[n], cu[n + 1]) for n in range(len(cu) - 1)]
+
+
+def run_oracle(inp, variant, threads=8):
+    """Whole-input fp64 oracle run (small inputs)."""
+    import oracle
+    cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].numpy()
+    if variant == "gdn":
+        return oracle.gdn_fwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]), f64(inp["beta"]),
+                              inp["scale"], f64(inp["h0"]), cu_seqlens=cu, threads=threads)
+    return oracle.gdn2_fwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]), f64(inp["b"]),
+                           f64(inp["w"]), inp["scale"], f64(inp["h0"]), cu_seqlens=cu, threads=threads)
+
+
+def oracle_units(inp, variant, units, threads=8):
+    """fp64 oracle on a few (sequence n, head h) units of a large input, each sliced out on its own.
+
+    Returns {(n, h): (o [L, dv], hT [dk, dv])}.
+    """
+    import oracle
+    spans = seq_spans(inp)
+    results = {}
+
+    def one(unit):
+        n, h = unit
+        row, t0, t1 = spans[n]
+
+        def sl(t):
+            return None if t is None else f64(t[row:row + 1, t0:t1, h:h + 1])
+
+        h0 = None if inp["h0"] is None else f64(inp["h0"][n:n + 1, h:h + 1])
+        if variant == "gdn":
+            o, hT = oracle.gdn_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]), sl(inp["beta"]),
+                                   inp["scale"], h0)
+        else:
+            o, hT = oracle.gdn2_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]), sl(inp["b"]),
+                                    sl(inp["w"]), inp["scale"], h0)
+        results[unit] = (o[0, :, 0], hT[0, 0])
+
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(1, min(threads, len(units)))) as ex:
+        list(ex.map(one, units))
+    return results
+
+
+def unit_slices(inp, o, hT, unit):
+    """The CUDA outputs of one (n, h) unit as fp64 numpy: (o [L, dv], hT [dk, dv])."""
+    n, h = unit
+    row, t0, t1 = seq_spans(inp)[n]
+    return f64(o[row, t0:t1, h]), f64(hT[n, h])

@@ -1,0 +1,100 @@
+"""CPU tests of the C ABI: the library loads, exports what include/gdn.h declares, and rejects bad
+arguments on the host before touching a device (no compute call runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_105_b200 import build
+    build.build()
+    from gated_delta_rule_105_b200.binding import load_library
+    return load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn\w*)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["gdn_chunk_fwd", "gdn2_chunk_fwd", "gdn_workspace_bytes", "gdn_check_error", "gdn_status_string",
+              "gdn_last_error", "gdn_set_kernel", "gdn_last_kernel"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libgdn.so does not export {name}"
+
+
+def test_exported_symbols_are_unmangled_c():
+    out = os.popen(f"nm -D --defined-only {os.path.join(ROOT, 'gated_delta_rule_105_b200', 'libgdn.so')}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}$", out, flags=re.M), name
+
+
+A = 0x10000  # a 16-byte aligned fake device address; never dereferenced by the host checks
+
+
+def call(lib, **kw):
+    args = dict(q=A, k=A, v=A, g=A, beta=A, scale=0.125, h0=None, o=A, hT=None, B=1, T=64, H=1, dk=64, dv=64,
+                BT=64, dt=1, cu=None, n_seqs=0, ws=None, ws_bytes=0, stream=None)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    return lib.gdn_chunk_fwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]), vp(args["beta"]),
+                             args["scale"], vp(args["h0"]), vp(args["o"]), vp(args["hT"]), args["B"], args["T"],
+                             args["H"], args["dk"], args["dv"], args["BT"], args["dt"], vp(args["cu"]),
+                             args["n_seqs"], vp(args["ws"]), args["ws_bytes"], vp(args["stream"]))
+
+
+def call2(lib, **kw):
+    args = dict(q=A, k=A, v=A, g=A, b=A, w=A, B=1, T=64, H=1, dk=64, dv=64, BT=64, dt=1)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    return lib.gdn2_chunk_fwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]), vp(args["b"]),
+                              vp(args["w"]), 0.125, None, vp(A), None, args["B"], args["T"], args["H"], args["dk"],
+                              args["dv"], args["BT"], args["dt"], None, 0, None, 0, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(o=None), 1), (dict(beta=None), 1),
+    (dict(q=A + 8), 1), (dict(hT=A + 4), 1), (dict(h0=A + 2), 1),
+    (dict(B=0), 1), (dict(H=0), 1), (dict(T=-1), 1),
+    (dict(BT=32), 2), (dict(dk=96), 2), (dict(dk=256), 2), (dict(dv=32), 2), (dict(dv=320), 2), (dict(dv=96), 2),
+    (dict(dt=7), 2), (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1),
+    (dict(cu=A, B=2, n_seqs=2), 1), (dict(cu=A, n_seqs=0), 1), (dict(n_seqs=3), 1),
+    (dict(ws=None, ws_bytes=64), 1),
+])
+def test_host_checks_reject_bad_arguments(lib, kw, status):
+    assert call(lib, **kw) == status
+    assert lib.gdn_last_error().decode() != ""
+
+
+@pytest.mark.parametrize("kw,status", [(dict(w=None), 1), (dict(b=None), 1), (dict(w=A + 8), 1), (dict(dk=32), 2)])
+def test_host_checks_gdn2(lib, kw, status):
+    assert call2(lib, **kw) == status
+
+
+def test_status_strings_and_kernel_choice(lib):
+    for s in range(6):
+        assert lib.gdn_status_string(s).decode() not in ("", "unknown status")
+    assert lib.gdn_set_kernel(9) == 1
+    assert lib.gdn_set_kernel(0) == 0
+    assert lib.gdn_workspace_bytes(4, 4096, 16, 128, 256, 64, 0) == 0
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    from gated_delta_rule_105_b200 import gdn_chunk_fwd
+    q = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        gdn_chunk_fwd(q, q, q, torch.zeros(1, 4, 1), torch.zeros(1, 4, 1))

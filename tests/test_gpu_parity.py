@@ -1,0 +1,141 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, element by element.
+
+Small inputs span several 64-token chunks and a ragged tail and are compared in full; the five
+measured workloads run at full size in the bench's launch configuration and are compared on sampled
+(sequence, head) units, which the oracle computes one at a time.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_105_b200.inputs import WORKLOADS, generate, generate_workload
+from parity_util import TOL, f64, oracle_units, relerr, run_cuda, run_oracle, unit_slices
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = {"f32": ["simt"], "bf16": ["simt", "tc"]}
+
+
+@pytest.fixture(autouse=True)
+def _reset_kernel():
+    yield
+    from gated_delta_rule_105_b200 import set_kernel
+    set_kernel("auto")
+
+
+def use_kernel(name):
+    from gated_delta_rule_105_b200 import set_kernel
+    set_kernel(name)
+
+
+def check(o, hT, ref_o, ref_hT, dtype, what=""):
+    eo, eh = relerr(f64(o), ref_o), relerr(f64(hT), ref_hT)
+    assert np.isfinite(f64(o)).all() and np.isfinite(f64(hT)).all(), what
+    assert eo <= TOL[dtype] and eh <= TOL[dtype], f"{what}: o err {eo:.3g}, hT err {eh:.3g} (tol {TOL[dtype]})"
+    return eo, eh
+
+
+SHAPES = [(T, 128, 128) for T in (1, 63, 64, 65, 130, 257)] + [(130, 64, 64), (130, 128, 256), (97, 64, 192)]
+
+
+@pytest.mark.parametrize("variant", ["gdn", "gdn2"])
+@pytest.mark.parametrize("dtype,kernel", [("f32", "simt"), ("bf16", "simt"), ("bf16", "tc")])
+@pytest.mark.parametrize("T,dk,dv", SHAPES)
+def test_small_shapes(variant, dtype, kernel, T, dk, dv):
+    inp = generate(2, T, 2, dk, dv, dtype, seed=T * 7 + dk + dv, variant=variant, h0_std=0.05)
+    use_kernel(kernel)
+    o, hT = run_cuda(inp, variant)
+    torch.cuda.synchronize()
+    ro, rh = run_oracle(inp, variant)
+    check(o, hT, ro, rh, dtype, f"{variant} {dtype} {kernel} T={T} dk={dk} dv={dv}")
+
+
+@pytest.mark.parametrize("variant", ["gdn", "gdn2"])
+@pytest.mark.parametrize("dtype,kernel", [("f32", "simt"), ("bf16", "simt"), ("bf16", "tc")])
+def test_varlen_with_empty_and_ragged_sequences(variant, dtype, kernel):
+    cu = np.array([0, 1, 1, 64, 129, 200, 330], dtype=np.int32)
+    inp = generate(1, int(cu[-1]), 3, 64, 128, dtype, seed=11, variant=variant, h0_std=0.1, cu_seqlens=cu)
+    use_kernel(kernel)
+    o, hT = run_cuda(inp, variant)
+    ro, rh = run_oracle(inp, variant)
+    check(o, hT, ro, rh, dtype, f"varlen {variant} {dtype} {kernel}")
+    assert np.array_equal(f64(hT)[1], f64(inp["h0"])[1])  # zero-length sequence: hT = h0
+
+
+@pytest.mark.parametrize("dtype,kernel", [("f32", "simt"), ("bf16", "simt"), ("bf16", "tc")])
+def test_no_final_state_and_zero_h0(dtype, kernel):
+    inp = generate(1, 100, 2, 64, 64, dtype, seed=5)
+    use_kernel(kernel)
+    o, hT = run_cuda(inp, "gdn", output_final_state=False)
+    assert hT is None
+    ro, _ = run_oracle(inp, "gdn")
+    assert relerr(f64(o), ro) <= TOL[dtype]
+
+
+def test_empty_sequence_length_zero_copies_state():
+    inp = generate(2, 0, 2, 64, 64, "f32", seed=3, h0_std=0.3)
+    o, hT = run_cuda(inp, "gdn")
+    assert o.numel() == 0 and torch.equal(hT.cpu(), inp["h0"])
+
+
+@pytest.mark.parametrize("kernel", ["simt", "tc"])
+def test_split_continuation_through_state(kernel):
+    """Running [0, t0) then [t0, T) with hT fed back as h0 equals one run (state is the resume point)."""
+    inp = generate(2, 300, 2, 128, 128, "bf16", seed=21, h0_std=0.02)
+    use_kernel(kernel)
+    o, hT = run_cuda(inp, "gdn")
+    t0 = 128
+    per_token = ("q", "k", "v", "g", "beta")
+    a = {k: (v[:, :t0].contiguous() if k in per_token else v) for k, v in inp.items()}
+    b = {k: (v[:, t0:].contiguous() if k in per_token else v) for k, v in inp.items()}
+    oa, ha = run_cuda(a, "gdn")
+    b["h0"] = ha.cpu()
+    ob, hb = run_cuda(b, "gdn")
+    assert relerr(f64(torch.cat([oa, ob], 1)), f64(o)) < 1e-2 and relerr(f64(hb), f64(hT)) < 1e-2
+
+
+@pytest.mark.parametrize("kernel", ["simt", "tc"])
+def test_deterministic_bits(kernel):
+    inp = generate(2, 200, 4, 128, 256, "bf16", seed=8)
+    use_kernel(kernel)
+    o1, h1 = run_cuda(inp, "gdn")
+    o2, h2 = run_cuda(inp, "gdn")
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+def test_bad_cu_seqlens_reported_by_device_word():
+    from gated_delta_rule_105_b200 import GdnError, check_error
+    inp = generate(1, 128, 2, 64, 64, "bf16", seed=4, cu_seqlens=np.array([0, 100, 50, 128], dtype=np.int32))
+    run_cuda(inp, "gdn")
+    with pytest.raises(GdnError) as ei:
+        check_error()
+    assert ei.value.status == 5
+    check_error()  # the word was cleared
+
+
+# ------------------------------------------------------------------ the measured workloads at full size
+def sample_units(inp, H, n=3):
+    n_seq = inp["h0"].shape[0] if inp["h0"] is not None else (
+        inp["q"].shape[0] if inp["cu_seqlens"] is None else inp["cu_seqlens"].numel() - 1)
+    cand = [(0, 0), (n_seq - 1, H - 1), (n_seq // 2, H // 2)]
+    return cand[:n]
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+def test_workload_full_size_sampled(name, kernel):
+    w = WORKLOADS[name]
+    if kernel == "simt" and w.dtype == "f32":
+        pytest.skip("auto is simt for fp32")
+    inp = generate_workload(w)
+    use_kernel(kernel)
+    o, hT = run_cuda(inp, w.variant)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(hT).all()
+    units = sample_units(inp, w.H)
+    ref = oracle_units(inp, w.variant, units)
+    for u in units:
+        ou, hu = unit_slices(inp, o, hT, u)
+        ro, rh = ref[u]
+        eo, eh = relerr(ou, ro), relerr(hu, rh)
+        assert eo <= TOL[w.dtype] and eh <= TOL[w.dtype], f"{name} {kernel} unit {u}: o {eo:.3g} hT {eh:.3g}"
