@@ -40,9 +40,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, fp, i, f, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.gdn_workspace_bytes.argtypes = [i] * 7
     lib.gdn_workspace_bytes.restype = sz
-    lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [i] * 7 + [vp, i, vp, sz, vp]
+    lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [i] * 8 + [vp, i, vp, sz, vp]
     lib.gdn_chunk_fwd.restype = i
-    lib.gdn2_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, f, fp, vp, fp] + [i] * 7 + [vp, i, vp, sz, vp]
+    lib.gdn2_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, f, fp, vp, fp] + [i] * 8 + [vp, i, vp, sz, vp]
     lib.gdn2_chunk_fwd.restype = i
     lib.gdn_set_kernel.argtypes = [i]
     lib.gdn_set_kernel.restype = i
@@ -102,9 +102,12 @@ def check_error(stream=None) -> None:
     _raise_on(load_library().gdn_check_error(ctypes.c_void_p(s.cuda_stream)))
 
 
-def _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state):
+def _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype):
     _check_dev("q", q)
     dt = q.dtype
+    o_dtype = dt if o_dtype is None else o_dtype
+    if o_dtype not in (torch.float32, dt):
+        raise ValueError(f"o_dtype must be float32 or q's dtype, got {o_dtype}")
     _check_dev("k", k, dt)
     _check_dev("v", v, dt)
     B, T, H, dk = q.shape
@@ -116,20 +119,23 @@ def _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state):
         _check_dev("cu_seqlens", cu_seqlens, torch.int32)
     _check_dev("h0", h0, torch.float32)
     if o is None:
-        o = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
+        o = torch.empty((B, T, H, dv), dtype=o_dtype, device=q.device)
+    elif o.dtype != o_dtype:
+        raise ValueError(f"o must be {o_dtype}")
     if hT is None and output_final_state:
         hT = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=q.device)
     return B, T, H, dk, dv, n_seq, o, hT
 
 
 def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, output_final_state=True, cu_seqlens=None, BT=64,
-                  o=None, hT=None):
+                  o=None, hT=None, o_dtype=None):
     """Chunked gated delta rule forward through ``gdn_chunk_fwd`` of the C ABI.
 
     q, k [B,T,H,dk] and v [B,T,H,dv] (fp32 or bf16), g, beta [B,T,H] fp32, h0 [N,H,dk,dv] fp32 or None,
-    cu_seqlens int32 [N+1] (B == 1) or None.  Returns (o [B,T,H,dv] in q's dtype, hT [N,H,dk,dv] fp32).
+    cu_seqlens int32 [N+1] (B == 1) or None.  Returns (o [B,T,H,dv], hT [N,H,dk,dv] fp32); o is in
+    ``o_dtype`` (float32, or q's dtype -- the default).
     """
-    B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state)
+    B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype)
     _check_dev("g", g, torch.float32)
     _check_dev("beta", beta, torch.float32)
     if g.shape != (B, T, H) or beta.shape != (B, T, H):
@@ -138,19 +144,19 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, output_final_state=True
     stream = torch.cuda.current_stream(q.device).cuda_stream
     st = load_library().gdn_chunk_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(o), _ptr(hT),
-        B, T, H, dk, dv, BT, _dtype_code(q), _ptr(cu_seqlens), 0 if cu_seqlens is None else n_seq,
-        None, 0, ctypes.c_void_p(stream))
+        B, T, H, dk, dv, BT, _dtype_code(q), _dtype_code(o), _ptr(cu_seqlens),
+        0 if cu_seqlens is None else n_seq, None, 0, ctypes.c_void_p(stream))
     _raise_on(st)
     return o, hT
 
 
 def gdn2_chunk_fwd(q, k, v, g, b, w, scale=None, h0=None, output_final_state=True, cu_seqlens=None, BT=64,
-                   o=None, hT=None):
+                   o=None, hT=None, o_dtype=None):
     """Gated Delta Rule-2 forward through ``gdn2_chunk_fwd`` of the C ABI.
 
     g (per-channel log-decay) and b (erase gate) are [B,T,H,dk] fp32, w (write gate) is [B,T,H,dv] fp32.
     """
-    B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state)
+    B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype)
     for name, t, shape in (("g", g, (B, T, H, dk)), ("b", b, (B, T, H, dk)), ("w", w, (B, T, H, dv))):
         _check_dev(name, t, torch.float32)
         if t.shape != shape:
@@ -159,8 +165,8 @@ def gdn2_chunk_fwd(q, k, v, g, b, w, scale=None, h0=None, output_final_state=Tru
     stream = torch.cuda.current_stream(q.device).cuda_stream
     st = load_library().gdn2_chunk_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), scale, _ptr(h0), _ptr(o), _ptr(hT),
-        B, T, H, dk, dv, BT, _dtype_code(q), _ptr(cu_seqlens), 0 if cu_seqlens is None else n_seq,
-        None, 0, ctypes.c_void_p(stream))
+        B, T, H, dk, dv, BT, _dtype_code(q), _dtype_code(o), _ptr(cu_seqlens),
+        0 if cu_seqlens is None else n_seq, None, 0, ctypes.c_void_p(stream))
     _raise_on(st)
     return o, hT
 

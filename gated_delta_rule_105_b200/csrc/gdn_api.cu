@@ -43,7 +43,7 @@ static unsigned* err_word_ptr(gdn_status* st) {
 static gdn_status check_common(const void* q, const void* k, const void* v, const float* g, const float* gate,
                                const float* w, bool gdn2, float scale, const float* h0, const void* o,
                                const float* hT, int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt,
-                               const int32_t* cu, int n_seqs, void* ws, size_t ws_bytes, int* n_seq_out) {
+                               gdn_dtype o_dt, const int32_t* cu, int n_seqs, void* ws, size_t ws_bytes, int* n_seq_out) {
     t_msg[0] = 0;
     if (T > 0 && (!q || !k || !v || !g || !gate || !o || (gdn2 && !w)))
         return fail(GDN_ERR_INVALID_ARG, "a required pointer (q, k, v, g, %s, o%s) is NULL",
@@ -57,6 +57,8 @@ static gdn_status check_common(const void* q, const void* k, const void* v, cons
     if (dv < 64 || dv > 256 || dv % 64 != 0)
         return fail(GDN_ERR_UNSUPPORTED, "dv must be a multiple of 64 in [64, 256] (got %d)", dv);
     if (dt != GDN_F32 && dt != GDN_BF16) return fail(GDN_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
+    if (o_dt != GDN_F32 && o_dt != dt)
+        return fail(GDN_ERR_UNSUPPORTED, "o_dt must be GDN_F32 or the input dtype (got %d)", (int)o_dt);
     if (!std::isfinite(scale)) return fail(GDN_ERR_INVALID_ARG, "scale is not finite");
     if (ws_bytes > 0 && !ws) return fail(GDN_ERR_INVALID_ARG, "ws_bytes > 0 with a NULL workspace");
     if (cu) {
@@ -75,31 +77,36 @@ static gdn_status check_common(const void* q, const void* k, const void* v, cons
     return GDN_OK;
 }
 
-template <typename TIn, int DK, bool GDN2>
+template <typename TIn, typename TOut, int DK, bool GDN2>
 static gdn_status launch_simt_dk(const FwdParams& p, unsigned* err, cudaStream_t stream) {
-    using L = SimtSmem<DK, kSimtDVT, GDN2>;
-    auto kern = gdn_simt_fwd_kernel<TIn, DK, kSimtDVT, GDN2>;
+    constexpr int DVT = SimtDVT<GDN2>::value;
+    using L = SimtSmem<DK, DVT, GDN2>;
+    auto kern = gdn_simt_fwd_kernel<TIn, TOut, DK, DVT, GDN2>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    dim3 grid(p.dv / kSimtDVT, p.H, p.n_seq);
+    dim3 grid(p.dv / DVT, p.H, p.n_seq);
     kern<<<grid, kSimtThreads, L::bytes, stream>>>(p, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "SIMT kernel launch: %s", cudaGetErrorString(e));
     return GDN_OK;
 }
 
-template <bool GDN2>
-static gdn_status launch_simt(const FwdParams& p, gdn_dtype dt, unsigned* err, cudaStream_t stream) {
-    if (dt == GDN_F32)
-        return p.dk == 64 ? launch_simt_dk<float, 64, GDN2>(p, err, stream)
-                          : launch_simt_dk<float, 128, GDN2>(p, err, stream);
-    return p.dk == 64 ? launch_simt_dk<__nv_bfloat16, 64, GDN2>(p, err, stream)
-                      : launch_simt_dk<__nv_bfloat16, 128, GDN2>(p, err, stream);
+template <typename TIn, typename TOut, bool GDN2>
+static gdn_status launch_simt_io(const FwdParams& p, unsigned* err, cudaStream_t stream) {
+    return p.dk == 64 ? launch_simt_dk<TIn, TOut, 64, GDN2>(p, err, stream)
+                      : launch_simt_dk<TIn, TOut, 128, GDN2>(p, err, stream);
 }
 
-static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, cudaStream_t stream) {
+template <bool GDN2>
+static gdn_status launch_simt(const FwdParams& p, gdn_dtype dt, gdn_dtype o_dt, unsigned* err, cudaStream_t stream) {
+    if (dt == GDN_F32) return launch_simt_io<float, float, GDN2>(p, err, stream);
+    if (o_dt == GDN_F32) return launch_simt_io<__nv_bfloat16, float, GDN2>(p, err, stream);
+    return launch_simt_io<__nv_bfloat16, __nv_bfloat16, GDN2>(p, err, stream);
+}
+
+static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, gdn_dtype o_dt, cudaStream_t stream) {
     const int choice = g_kernel_choice.load();
-    const bool tc_ok = dt == GDN_BF16 && tc_supported(p, gdn2);
+    const bool tc_ok = dt == GDN_BF16 && tc_supported(p, gdn2, o_dt == GDN_F32);
     if (choice == GDN_KERNEL_TC && !tc_ok)
         return fail(GDN_ERR_UNSUPPORTED, "the tcgen05 kernel needs bf16 inputs and a supported shape");
     gdn_status st;
@@ -108,12 +115,12 @@ static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, cudaStream_t 
     if (p.n_seq == 0 || p.H == 0) return GDN_OK;
     const bool use_tc = tc_ok && choice != GDN_KERNEL_SIMT;
     if (use_tc) {
-        st = launch_tc(p, gdn2, err, stream);
+        st = launch_tc(p, gdn2, o_dt == GDN_F32, err, stream);
         if (st == GDN_OK) t_last_kernel = GDN_KERNEL_TC;
         else if (st == GDN_ERR_CUDA) fail(st, "tcgen05 kernel launch: %s", tc_last_error());
         return st;
     }
-    st = gdn2 ? launch_simt<true>(p, dt, err, stream) : launch_simt<false>(p, dt, err, stream);
+    st = gdn2 ? launch_simt<true>(p, dt, o_dt, err, stream) : launch_simt<false>(p, dt, o_dt, err, stream);
     if (st == GDN_OK) t_last_kernel = GDN_KERNEL_SIMT;
     return st;
 }
@@ -128,26 +135,26 @@ size_t gdn_workspace_bytes(int, int, int, int, int, int, int) { return 0; }
 
 gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float scale, const float* h0, void* o, float* hT, int B, int T, int H, int dk, int dv,
-                         int BT, gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs, void* workspace,
-                         size_t ws_bytes, cudaStream_t stream) {
+                         int BT, gdn_dtype dt, gdn_dtype o_dt, const int32_t* cu_seqlens, int n_seqs,
+                         void* workspace, size_t ws_bytes, cudaStream_t stream) {
     int n_seq = 0;
     gdn_status st = check_common(q, k, v, g, beta, nullptr, false, scale, h0, o, hT, B, T, H, dk, dv, BT, dt,
-                                 cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
+                                 o_dt, cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
     if (st != GDN_OK) return st;
     FwdParams p{q, k, v, g, beta, nullptr, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
-    return run(p, false, dt, stream);
+    return run(p, false, dt, o_dt, stream);
 }
 
 gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* b,
                           const float* w, float scale, const float* h0, void* o, float* hT, int B, int T, int H,
-                          int dk, int dv, int BT, gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs,
-                          void* workspace, size_t ws_bytes, cudaStream_t stream) {
+                          int dk, int dv, int BT, gdn_dtype dt, gdn_dtype o_dt, const int32_t* cu_seqlens,
+                          int n_seqs, void* workspace, size_t ws_bytes, cudaStream_t stream) {
     int n_seq = 0;
-    gdn_status st = check_common(q, k, v, g, b, w, true, scale, h0, o, hT, B, T, H, dk, dv, BT, dt, cu_seqlens,
-                                 n_seqs, workspace, ws_bytes, &n_seq);
+    gdn_status st = check_common(q, k, v, g, b, w, true, scale, h0, o, hT, B, T, H, dk, dv, BT, dt, o_dt,
+                                 cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
     if (st != GDN_OK) return st;
     FwdParams p{q, k, v, g, b, w, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
-    return run(p, true, dt, stream);
+    return run(p, true, dt, o_dt, stream);
 }
 
 gdn_status gdn_set_kernel(gdn_kernel kernel) {

@@ -10,6 +10,7 @@ namespace gdn {
 // log2(e): the chunk-local cumulative gate is kept in base 2 so the kernels can use exp2
 // (GatedDeltaNet data-flow walkthrough, section "Chunked parallelism": cumsum of g times 1.44269504).
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr double kLog2eD = 1.4426950408889634;
 constexpr int kChunk = 64;  // BT = C = 64 tokens per chunk
 
 // Bits of the device error word (read and cleared by gdn_check_error).

@@ -10,6 +10,9 @@
 // Per chunk (rows r, s < 64; zero rows pad a partial chunk, which makes them inert: k = v = 0,
 // beta = b = w = 0 and g = 0 so the padded cumulative gate stays at the last real token's value):
 //   G_r   = log2(e) * sum_{s<=r} g_s                           (GDN-2: per key channel)
+// G is accumulated and differenced in fp64: with strong decay |G| reaches ~10^3 inside a chunk, where an
+// fp32 cumsum loses ~1e-4 absolute in G_r - G_s for nearby r, s -- as much as the whole fp32 error
+// budget.  Only the (small) differences are rounded to fp32 before exp2.
 //   A_rs  = beta_r (k_r . k_s) 2^(G_r - G_s)        s < r      (GDN-2: sum_i b_ri k_ri k_si 2^(G_ri - G_si))
 //   P_rs  = (q_r . k_s) 2^(G_r - G_s)               s <= r     (GDN-2: per-channel factor inside the sum)
 //   Tm    = (I + A)^-1                               forward substitution, one column per thread
@@ -27,49 +30,50 @@
 namespace gdn {
 
 constexpr int kSimtThreads = 256;
-constexpr int kSimtDVT = 32;  // value columns per CTA
+// value columns per CTA: GDN-2 keeps a per-channel fp64 gate in shared memory, so it takes a narrower slice
+template <bool GDN2> struct SimtDVT { static constexpr int value = GDN2 ? 16 : 32; };
 
+// Shared-memory map in 4-byte words.  The fp64 gate block comes first so it is 8-byte aligned.
 template <int DK, int DVT, bool GDN2>
 struct SimtSmem {
     static constexpr int LDK = DK + 1;  // padded row stride: conflict-free column walks
     static constexpr int LDT = kChunk + 1;
     static constexpr int nK = kChunk * LDK;
-    static constexpr int oK = 0;                       // K [64][LDK]
-    static constexpr int oQ = oK + nK;                 // Q, then Q.2^G (GDN-2)
-    static constexpr int oBK = oQ + nK;                // GDN-2: b.K, then b.K.2^G, then K.2^(G_last-G)
-    static constexpr int oG = oBK + (GDN2 ? nK : 0);   // GDN-2: cumulative gate per channel
-    static constexpr int oV = oG + (GDN2 ? nK : 0);    // scaled V, then X
-    static constexpr int oU = oV + kChunk * DVT;       // U
-    static constexpr int oH = oU + kChunk * DVT;       // state slice [DK][DVT]
-    static constexpr int oA = oH + DK * DVT;           // A [64][LDT]
-    static constexpr int oT = oA + kChunk * LDT;       // (I+A)^-1
-    static constexpr int oP = oT + kChunk * LDT;       // P
-    static constexpr int oG1 = oP + kChunk * LDT;      // GDN: cumulative gate [64]
-    static constexpr int oB1 = oG1 + kChunk;           // GDN: beta [64]
-    static constexpr int oF = oB1 + kChunk;            // GDN: 2^(G_last - G_s) [64]
+    static constexpr int oGd = 0;                              // fp64 cumulative gate: GDN-2 [64][LDK], GDN [64]
+    static constexpr int oK = oGd + 2 * (GDN2 ? nK : kChunk);  // K [64][LDK]
+    static constexpr int oQ = oK + nK;                         // Q, then Q.2^G (GDN-2)
+    static constexpr int oBK = oQ + nK;                        // GDN-2: b.K, then b.K.2^G, then K.2^(G_last-G)
+    static constexpr int oV = oBK + (GDN2 ? nK : 0);           // scaled V, then X
+    static constexpr int oH = oV + kChunk * DVT;               // state slice [DK][DVT]
+    static constexpr int oA = oH + DK * DVT;                   // A [64][LDT]; its space then holds U [64][DVT]
+    static constexpr int oT = oA + kChunk * LDT;               // (I+A)^-1
+    static constexpr int oP = oT + kChunk * LDT;               // P
+    static constexpr int oB1 = oP + kChunk * LDT;              // GDN: beta [64]
+    static constexpr int oF = oB1 + kChunk;                    // GDN: 2^(G_last - G_s) [64]
     static constexpr int total = oF + kChunk;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
+    static_assert(kChunk * DVT <= kChunk * LDT, "U must fit in the space of A");
 };
 
-template <typename TIn, int DK, int DVT, bool GDN2>
+template <typename TIn, typename TOut, int DK, int DVT, bool GDN2>
 __global__ void __launch_bounds__(kSimtThreads)
 gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
     using L = SimtSmem<DK, DVT, GDN2>;
     constexpr int LDK = L::LDK, LDT = L::LDT, NT = kSimtThreads;
     constexpr int PER = kChunk * DVT / NT;  // (row, column) outputs per thread
     static_assert(kChunk * DVT % NT == 0, "tile must divide evenly");
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
+    double* sG = reinterpret_cast<double*>(sm + L::oGd);  // GDN-2 [64][LDK]
+    double* sG1 = sG;                                     // GDN [64]
     float* sK = sm + L::oK;
     float* sQ = sm + L::oQ;
     float* sBK = sm + L::oBK;
-    float* sG = sm + L::oG;
     float* sV = sm + L::oV;
-    float* sU = sm + L::oU;
     float* sH = sm + L::oH;
     float* sA = sm + L::oA;
+    float* sU = sm + L::oA;  // U is formed after (I+A)^-1, when A is no longer needed
     float* sT = sm + L::oT;
     float* sP = sm + L::oP;
-    float* sG1 = sm + L::oG1;
     float* sB1 = sm + L::oB1;
     float* sF = sm + L::oF;
 
@@ -81,7 +85,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
     const TIn* __restrict__ q = static_cast<const TIn*>(p.q);
     const TIn* __restrict__ k = static_cast<const TIn*>(p.k);
     const TIn* __restrict__ v = static_cast<const TIn*>(p.v);
-    TIn* __restrict__ o = static_cast<TIn*>(p.o);
+    TOut* __restrict__ o = static_cast<TOut*>(p.o);
 
     int row, bos, eos;
     if (p.cu_seqlens) {
@@ -123,7 +127,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
             sK[r * LDK + i] = kv;
             sQ[r * LDK + i] = qv;
             if (GDN2) {
-                sG[r * LDK + i] = gv;
+                sG[r * LDK + i] = (double)gv;
                 sBK[r * LDK + i] = bv * kv;
             }
         }
@@ -140,24 +144,24 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
         if (!GDN2 && tid < kChunk) {
             const int r = tid;
             const size_t tok = ((size_t)row * T + c0 + r) * H + h;
-            sG1[r] = r < Lc ? p.g[tok] : 0.f;
+            sG1[r] = r < Lc ? (double)p.g[tok] : 0.0;
             sB1[r] = r < Lc ? p.beta[tok] : 0.f;
         }
         __syncthreads();
         // ---- chunk-local cumulative gate, base 2
         if (GDN2) {
             for (int i = tid; i < DK; i += NT) {
-                float acc = 0.f;
+                double acc = 0.0;
                 for (int r = 0; r < kChunk; ++r) {
                     acc += sG[r * LDK + i];
-                    sG[r * LDK + i] = acc * kLog2e;
+                    sG[r * LDK + i] = acc * kLog2eD;
                 }
             }
         } else if (tid == 0) {
-            float acc = 0.f;
+            double acc = 0.0;
             for (int r = 0; r < kChunk; ++r) {
                 acc += sG1[r];
-                sG1[r] = acc * kLog2e;
+                sG1[r] = acc * kLog2eD;
             }
         }
         __syncthreads();
@@ -168,7 +172,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
             if (s <= r) {
                 if (GDN2) {
                     for (int i = 0; i < DK; ++i) {
-                        const float f = exp2f(sG[r * LDK + i] - sG[s * LDK + i]);
+                        const float f = exp2f((float)(sG[r * LDK + i] - sG[s * LDK + i]));
                         const float ks = sK[s * LDK + i] * f;
                         a = fmaf(sBK[r * LDK + i], ks, a);
                         pp = fmaf(sQ[r * LDK + i], ks, pp);
@@ -180,7 +184,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
                         dkk = fmaf(sK[r * LDK + i], ks, dkk);
                         dqk = fmaf(sQ[r * LDK + i], ks, dqk);
                     }
-                    const float f = exp2f(sG1[r] - sG1[s]);
+                    const float f = exp2f((float)(sG1[r] - sG1[s]));
                     a = sB1[r] * f * dkk;
                     pp = f * dqk;
                 }
@@ -194,7 +198,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
         if (GDN2) {
             for (int e = tid; e < kChunk * DK; e += NT) {
                 const int r = e / DK, i = e % DK;
-                const float f = exp2f(sG[r * LDK + i]);
+                const float f = exp2f((float)sG[r * LDK + i]);
                 sQ[r * LDK + i] *= f;
                 sBK[r * LDK + i] *= f;
             }
@@ -230,7 +234,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
                     kh = fmaf(sK[r * LDK + i], hv, kh);
                     qh = fmaf(sQ[r * LDK + i], hv, qh);
                 }
-                const float f = exp2f(sG1[r]);
+                const float f = exp2f((float)sG1[r]);
                 sV[e] -= sB1[r] * f * kh;
                 oi[m] = f * qh;
             }
@@ -248,10 +252,10 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
         if (GDN2) {
             for (int e = tid; e < kChunk * DK; e += NT) {
                 const int s = e / DK, i = e % DK;
-                sBK[s * LDK + i] = sK[s * LDK + i] * exp2f(sG[(kChunk - 1) * LDK + i] - sG[s * LDK + i]);
+                sBK[s * LDK + i] = sK[s * LDK + i] * exp2f((float)(sG[(kChunk - 1) * LDK + i] - sG[s * LDK + i]));
             }
         } else if (tid < kChunk) {
-            sF[tid] = exp2f(sG1[kChunk - 1] - sG1[tid]);
+            sF[tid] = exp2f((float)(sG1[kChunk - 1] - sG1[tid]));
         }
         __syncthreads();
         // ---- O = scale (Oi + P U) ; h <- 2^G_last h + Ktilde^T U
@@ -263,17 +267,17 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
             for (int s = 0; s <= r; ++s) acc = fmaf(sP[r * LDT + s], sU[s * DVT + j], acc);
             if (r < Lc) {
                 const size_t tok = ((size_t)row * T + c0 + r) * H + h;
-                o[tok * dv + j0 + j] = from_f32<TIn>(p.scale * acc);
+                o[tok * dv + j0 + j] = from_f32<TOut>(p.scale * acc);
             }
         }
         for (int e = tid; e < DK * DVT; e += NT) {
             const int i = e / DVT, j = e % DVT;
             float acc;
             if (GDN2) {
-                acc = exp2f(sG[(kChunk - 1) * LDK + i]) * sH[e];
+                acc = exp2f((float)sG[(kChunk - 1) * LDK + i]) * sH[e];
                 for (int s = 0; s < kChunk; ++s) acc = fmaf(sBK[s * LDK + i], sU[s * DVT + j], acc);
             } else {
-                acc = exp2f(sG1[kChunk - 1]) * sH[e];
+                acc = exp2f((float)sG1[kChunk - 1]) * sH[e];
                 for (int s = 0; s < kChunk; ++s) acc = fmaf(sK[s * LDK + i] * sF[s], sU[s * DVT + j], acc);
             }
             sH[e] = acc;

@@ -21,7 +21,9 @@
  *
  * Layouts (row-major, contiguous, all device pointers):
  *   q, k        [B, T, H, dk]   dtype `dt` (GDN_F32 or GDN_BF16)
- *   v, o        [B, T, H, dv]   dtype `dt`
+ *   v           [B, T, H, dv]   dtype `dt`
+ *   o           [B, T, H, dv]   dtype `o_dt`: GDN_F32, or `dt` itself.  A bf16 o carries the format's own
+ *                               rounding (half an ulp, 2^-9 relative, per element) on top of the kernel's error.
  *   GDN:   g, beta  [B, T, H]        fp32; g is the natural-log decay (g <= 0 expected), beta the write strength
  *   GDN-2: g, b     [B, T, H, dk]    fp32 per-channel log-decay and erase gate;  w [B, T, H, dv] fp32 write gate
  *   h0, hT      [N, H, dk, dv]  fp32, N = B, or n_seqs with cu_seqlens.  h0 == NULL means zeros;
@@ -63,7 +65,7 @@ typedef enum {
     GDN_ERR_DEVICE_ARG = 5 /* reported by gdn_check_error: cu_seqlens out of order or out of range */
 } gdn_status;
 
-typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype; /* dtype of q, k, v, o */
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype; /* dtype of q, k, v (dt) and of o (o_dt) */
 
 /* Kernel family used for a call.  AUTO picks the tensor-core (tcgen05) kernel for bf16 inputs when the
  * shape allows it and the SIMT fp32 kernel otherwise.  SIMT forces the fp32-FMA kernel (any dtype); TC
@@ -76,14 +78,14 @@ size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_se
 /* Gated delta rule forward; see the header comment for the definition, layouts and errors. */
 gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float scale, const float* h0, void* o, float* hT,
-                         int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt,
+                         int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt, gdn_dtype o_dt,
                          const int32_t* cu_seqlens, int n_seqs,
                          void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* Gated Delta Rule-2 forward; g, b are [B,T,H,dk] and w is [B,T,H,dv], all fp32. */
 gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* b,
                           const float* w, float scale, const float* h0, void* o, float* hT,
-                          int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt,
+                          int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt, gdn_dtype o_dt,
                           const int32_t* cu_seqlens, int n_seqs,
                           void* workspace, size_t ws_bytes, cudaStream_t stream);
 

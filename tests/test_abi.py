@@ -47,12 +47,12 @@ A = 0x10000  # a 16-byte aligned fake device address; never dereferenced by the 
 
 def call(lib, **kw):
     args = dict(q=A, k=A, v=A, g=A, beta=A, scale=0.125, h0=None, o=A, hT=None, B=1, T=64, H=1, dk=64, dv=64,
-                BT=64, dt=1, cu=None, n_seqs=0, ws=None, ws_bytes=0, stream=None)
+                BT=64, dt=1, odt=0, cu=None, n_seqs=0, ws=None, ws_bytes=0, stream=None)
     args.update(kw)
     vp = ctypes.c_void_p
     return lib.gdn_chunk_fwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]), vp(args["beta"]),
                              args["scale"], vp(args["h0"]), vp(args["o"]), vp(args["hT"]), args["B"], args["T"],
-                             args["H"], args["dk"], args["dv"], args["BT"], args["dt"], vp(args["cu"]),
+                             args["H"], args["dk"], args["dv"], args["BT"], args["dt"], args["odt"], vp(args["cu"]),
                              args["n_seqs"], vp(args["ws"]), args["ws_bytes"], vp(args["stream"]))
 
 
@@ -62,7 +62,7 @@ def call2(lib, **kw):
     vp = ctypes.c_void_p
     return lib.gdn2_chunk_fwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]), vp(args["b"]),
                               vp(args["w"]), 0.125, None, vp(A), None, args["B"], args["T"], args["H"], args["dk"],
-                              args["dv"], args["BT"], args["dt"], None, 0, None, 0, None)
+                              args["dv"], args["BT"], args["dt"], 0, None, 0, None, 0, None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -70,7 +70,7 @@ def call2(lib, **kw):
     (dict(q=A + 8), 1), (dict(hT=A + 4), 1), (dict(h0=A + 2), 1),
     (dict(B=0), 1), (dict(H=0), 1), (dict(T=-1), 1),
     (dict(BT=32), 2), (dict(dk=96), 2), (dict(dk=256), 2), (dict(dv=32), 2), (dict(dv=320), 2), (dict(dv=96), 2),
-    (dict(dt=7), 2), (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1),
+    (dict(dt=7), 2), (dict(dt=0, odt=1), 2), (dict(odt=5), 2), (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1),
     (dict(cu=A, B=2, n_seqs=2), 1), (dict(cu=A, n_seqs=0), 1), (dict(n_seqs=3), 1),
     (dict(ws=None, ws_bytes=64), 1),
 ])
