@@ -54,6 +54,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_error.argtypes = []
     lib.gdn_last_error.restype = ctypes.c_char_p
+    lib.gdn_debug_umma_selftest.argtypes = [vp, vp, vp, i, vp]
+    lib.gdn_debug_umma_selftest.restype = i
     _lib = lib
     return lib
 
@@ -100,6 +102,17 @@ def check_error(stream=None) -> None:
     """Synchronise the stream and raise if a kernel reported a device-side error."""
     s = torch.cuda.current_stream() if stream is None else stream
     _raise_on(load_library().gdn_check_error(ctypes.c_void_p(s.cuda_stream)))
+
+
+def umma_selftest(A, B, mode):
+    """Runs the tensor-core layout self-test (see ``gdn_debug_umma_selftest``); returns D = A B (fp32)."""
+    _check_dev("A", A, torch.float32)
+    _check_dev("B", B, torch.float32)
+    D = torch.empty((A.shape[0], B.shape[1]), dtype=torch.float32, device=A.device)
+    st = load_library().gdn_debug_umma_selftest(_ptr(A), _ptr(B), _ptr(D), int(mode),
+                                                 ctypes.c_void_p(torch.cuda.current_stream(A.device).cuda_stream))
+    _raise_on(st)
+    return D
 
 
 def _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype):

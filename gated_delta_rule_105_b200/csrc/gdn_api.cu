@@ -9,6 +9,7 @@
 #include "gdn_common.cuh"
 #include "gdn_simt.cuh"
 #include "gdn_tc.cuh"
+#include "gdn_tc_selftest.cuh"
 
 namespace gdn {
 
@@ -191,5 +192,21 @@ const char* gdn_status_string(gdn_status s) {
 }
 
 const char* gdn_last_error(void) { return t_msg; }
+
+gdn_status gdn_debug_umma_selftest(const float* A, const float* B, float* D, int mode, cudaStream_t stream) {
+    t_msg[0] = 0;
+    if (!A || !B || !D) return fail(GDN_ERR_INVALID_ARG, "NULL pointer");
+    if (mode < 0 || mode > 4) return fail(GDN_ERR_INVALID_ARG, "mode must be 0..4 (got %d)", mode);
+    gdn_status st;
+    unsigned* err = err_word_ptr(&st);
+    if (!err) return st;
+    const int smem = 65536 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(gdn_umma_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    gdn_umma_selftest_kernel<<<1, 128, smem, stream>>>(A, B, D, mode, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "selftest launch: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
 
 }  // extern "C"

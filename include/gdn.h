@@ -105,6 +105,14 @@ const char* gdn_status_string(gdn_status status);
 /* Description of the most recent failure on the calling thread ("" if none). */
 const char* gdn_last_error(void);
 
+/* Diagnostic (no counterpart on the pages): checks the tensor-core operand layouts the tcgen05 kernel uses.
+ * One CTA stages A (row-major [M][K] fp32, device) and B (row-major [K][N] fp32, device) as bf16 in shared
+ * memory in the layout selected by `mode` (0: A K-major 128x128, B K-major, N=64; 1: A MN-major 128x64,
+ * B K-major, N=64; 2: A K-major 128x64, B MN-major, N=128; 3: A K-major 128x128, B MN-major, N=64; 4: A
+ * 128x64 in tensor memory, B K-major, N=64), runs
+ * the MMA k-step loop, and writes D = A B (fp32, row-major [M][N], device).  Asynchronous on `stream`. */
+gdn_status gdn_debug_umma_selftest(const float* A, const float* B, float* D, int mode, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -27,7 +27,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["gdn_chunk_fwd", "gdn2_chunk_fwd", "gdn_workspace_bytes", "gdn_check_error", "gdn_status_string",
-              "gdn_last_error", "gdn_set_kernel", "gdn_last_kernel"]:
+              "gdn_last_error", "gdn_set_kernel", "gdn_last_kernel", "gdn_debug_umma_selftest"]:
         assert n in names
 
 
