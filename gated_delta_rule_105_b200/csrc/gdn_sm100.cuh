@@ -29,12 +29,16 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                  "r"(bytes)
                  : "memory");
 }
+// The suspend-time hint lets a waiting thread sleep (issuing nothing) until the phase completes or the
+// hint runs out, so warps that wait do not take issue slots from the warps that work.
+constexpr uint32_t kSuspendHintNs = 10000000u;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -208,6 +212,13 @@ __device__ __forceinline__ void tmem_st32u(uint32_t ta, const uint32_t (&r)[32])
         "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st16u(uint32_t ta, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(ta),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_st32(uint32_t ta, const float (&v)[32]) {
     const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
     asm volatile(
@@ -225,10 +236,30 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
+// 2^x by the hardware approximation (ex2.approx.ftz: relative error ~2^-22, results below 2^-126 flush
+// to zero), for the bf16 tensor-core path.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 // Splits x into hi = bf16(x) and lo = bf16(x - hi): hi + lo carries ~16 mantissa bits.
 __device__ __forceinline__ void split_bf16(float x, float& hi, float& lo) {
     hi = __bfloat162float(__float2bfloat16_rn(x));
     lo = x - hi;
+}
+// Writes 32 values as bf16 into 16-byte chunks c0 .. c0+3 of line `line` of a 128B-swizzled region.
+__device__ __forceinline__ void st_half_line_bf16(uint8_t* region, uint32_t line, int c0, const float (&x)[32],
+                                                  float scale = 1.f) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint4 u;
+        u.x = pack_bf16(x[8 * c + 0] * scale, x[8 * c + 1] * scale);
+        u.y = pack_bf16(x[8 * c + 2] * scale, x[8 * c + 3] * scale);
+        u.z = pack_bf16(x[8 * c + 4] * scale, x[8 * c + 5] * scale);
+        u.w = pack_bf16(x[8 * c + 6] * scale, x[8 * c + 7] * scale);
+        *reinterpret_cast<uint4*>(region + sw128(line, c0 + c)) = u;
+    }
 }
 // Writes 64 values (one 128-byte line of bf16) into line `line` of a 128B-swizzled region.
 __device__ __forceinline__ void st_line_bf16(uint8_t* region, uint32_t line, const float* x, float scale = 1.f) {

@@ -14,17 +14,17 @@
 //   O^T = diag(2^G) applied to h^T Q^T, + U^T P^T   (read-out, scaled by `scale` on the way out)
 //   h^T <- 2^(G_last) h^T + (U diag f)^T K
 // Precision: every bf16 operand whose rounding would reach the output at the bf16-ulp level is avoided or
-// split.  U and U diag f are kept as bf16 hi + lo pairs (in TMEM, as the A operand), P likewise (in
-// shared memory); the dominant diagonal beta_r v_r of T'' V is added in fp32 by the epilogue instead of
-// going through a bf16 T''; 2^G_r is applied to the fp32 accumulator of h^T Q^T instead of to Q.  The
-// remaining bf16 operands are h^T, W^T, T', the off-diagonal part of T'' and the inputs themselves.
+// split.  U and U diag f are kept as bf16 hi + lo pairs (in TMEM, as the A operand), P and T'' likewise
+// (in shared memory); 2^G_r is applied to the fp32 accumulator of h^T Q^T instead of to Q.  The remaining
+// bf16 operands are h^T, W^T, T' and the inputs themselves.
 // This is the WY form of the intra-chunk dependency with one state handed from chunk to chunk
 // (GatedDeltaNet data-flow walkthrough, yfxerp.com/news/367755, section "Chunked parallelism").
 //
 // Warp roles (16 warps): 0 TMA producer and gate prep; 1 issues the h-independent MMAs (S1, W^T) one chunk
-// ahead; 2 issues the serial MMAs (U^T, O^T, h^T); 3 idle; 4-7 (prep warpgroup) build A, P, (I+A)^-1,
-// T', T'' and -W^T; 8-11 and 12-15 (epilogue warpgroups) finish U and split it into bf16 operands, refresh
-// the bf16 copy of h^T and re-scale the fp32 state by the next chunk's decay, and write o and hT.
+// ahead; 2 issues the serial MMAs (U^T, O^T, h^T); 3 idle; 4-7 and 8-11 (two prep warpgroups, one per half
+// of the 64 chunk columns) build A, P, T', T'' and -W^T, the first of them also (I+A)^-1; 12-15 (epilogue
+// warpgroup) split U into bf16 operands, refresh the bf16 copy of h^T and re-scale the fp32 state by the
+// next chunk's decay, and write o and hT.
 // All mbarrier waits are bounded: on time-out the CTA sets the error word and drains to the exit.
 #pragma once
 
@@ -43,6 +43,7 @@ struct TcGate {  // one chunk's gate data, written by the producer warp
     float beta[64];  // beta (0 past the end of the sequence)
     float f[64];     // 2^(G_last - G_s)
     float eG[64];    // 2^(G_r)
+    float a[64];     // 2^(log2(e) g_r) = exp(g_r), the token's own decay (1 past the end of the sequence)
     float gamma;     // 2^(G_last)
     int L;           // valid rows in this chunk
     int pad[2];
@@ -54,8 +55,9 @@ struct TcSmem {
     static constexpr uint32_t KQ = 0;  // 2 stages x [K ch0-63 | Q ch0-63 | K ch64-127 | Q ch64-127], 8 KB each
     static constexpr uint32_t KQ_STAGE = 32768;
     static constexpr uint32_t V = KQ + 2 * KQ_STAGE;  // V tile: j 0-63 | j 64-127, 8 KB each (MN-major A)
-    static constexpr uint32_t TPP = V + 16384;        // T''[2] without its diagonal: [r][s] K-major, 8 KB each
-    static constexpr uint32_t TP = TPP + 16384;       // T': [r][s] K-major, 8 KB
+    static constexpr uint32_t TPP = V + 16384;        // T'' hi [2]: [r][s] K-major, 8 KB each
+    static constexpr uint32_t TPPL = TPP + 16384;     // T'' lo [2]
+    static constexpr uint32_t TP = TPPL + 16384;      // T': [r][s] K-major, 8 KB
     static constexpr uint32_t PH = TP + 8192;         // P hi [2]: [r][s] K-major, 8 KB each
     static constexpr uint32_t PL = PH + 16384;        // P lo [2]
     static constexpr uint32_t WT = PL + 16384;        // -W^T: lines i (128) x 64 r, MN-major B, 16 KB
@@ -76,21 +78,22 @@ enum TcBar : int {
     B_KQ_FULL = 0,    // [2] TMA K/Q landed (tx)
     B_KQ_EMPTY = 2,   // [2] serial MMAs of the stage's chunk done
     B_V_FULL = 4,     // V landed (tx)
-    B_V_EMPTY = 5,    // V read by the U^T MMA and by the epilogue's diagonal term (128)
+    B_V_EMPTY = 5,    // U^T MMA reading V done
     B_GATE = 6,       // [4] gate stage written
     B_S1_FULL = 10,   // S1 in TMEM
-    B_S1_FREE = 11,   // prep read S1 (128 arrivals)
-    B_TP_READY = 12,  // T' written (128)
+    B_S1_FREE = 11,   // prep read S1 (256 arrivals)
+    B_TP_READY = 12,  // T' written (256)
     B_W_FULL = 13,    // W^T in TMEM
-    B_PREP = 14,      // [2] T'', -W^T, P ready for the serial step (128)
+    B_PREP = 14,      // [2] T'', -W^T, P ready for the serial step (256)
     B_P_FREE = 16,    // [2] O^T MMA reading P done
     B_U_FULL = 18,    // U^T in TMEM (and -W^T, T'' no longer read)
     B_U_CONV = 19,    // U, U.f split into bf16 hi/lo in TMEM (128)
     B_H_FULL = 20,    // h^T MMA done
-    B_H_READY = 21,   // bf16 h^T staged and fp32 state re-scaled (256)
+    B_H_READY = 21,   // bf16 h^T staged in shared memory (128)
     B_O_FULL = 22,    // O^T MMAs done
     B_O_FREE = 23,    // O^T TMEM read (128)
     B_DRAIN = 24,     // [2] final commit of each MMA issuer
+    B_HM_READY = 26,  // fp32 state in TMEM re-scaled by the next chunk's decay (128)
 };
 
 // TMEM columns.  U^T is accumulated in fp32 at TM_U, then replaced in place by its bf16 hi (TM_U .. +31)
@@ -193,30 +196,54 @@ __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane,
         }
     }
     named_bar_sync(bar_id, 128);  // every diagonal inverse (and every A-block read) done
-    // off-diagonal blocks, within one warp each
-    auto block = [&](int i, int j, const Frag16* As, const int* ks, int nk) {
-        float x[2][4] = {};
-        for (int q = 0; q < nk; ++q) mma16(x, As[q], S, 16 * ks[q], 16 * j, lane);  // X = sum A_ik T_kj
+    // off-diagonal blocks, within one warp each: X = sum_k A_ik T_kj, parked in slot (i, j); T_ij = -T_ii X
+    auto finish = [&](int i, int j, const float (&x)[2][4]) {
         __syncwarp();
-        store16(S, 16 * i, 16 * j, lane, x, 1.f);  // park X in the (i, j) slot
+        store16(S, 16 * i, 16 * j, lane, x, 1.f);
         __syncwarp();
         Frag16 tii;
         load_a16(S, 16 * i, 16 * i, lane, tii);
         float y[2][4] = {};
-        mma16(y, tii, S, 16 * i, 16 * j, lane);  // T_ii X
+        mma16(y, tii, S, 16 * i, 16 * j, lane);
         __syncwarp();
         store16(S, 16 * i, 16 * j, lane, y, -1.f);
         __syncwarp();
     };
     if (wid == 0) {
-        { const Frag16 As[1] = {a10}; const int ks[1] = {0}; block(1, 0, As, ks, 1); }
-        { const Frag16 As[2] = {a20, a21}; const int ks[2] = {0, 1}; block(2, 0, As, ks, 2); }
-        { const Frag16 As[3] = {a30, a31, a32}; const int ks[3] = {0, 1, 2}; block(3, 0, As, ks, 3); }
+        {
+            float x[2][4] = {};
+            mma16(x, a10, S, 0, 0, lane);
+            finish(1, 0, x);
+        }
+        {
+            float x[2][4] = {};
+            mma16(x, a20, S, 0, 0, lane);
+            mma16(x, a21, S, 16, 0, lane);
+            finish(2, 0, x);
+        }
+        {
+            float x[2][4] = {};
+            mma16(x, a30, S, 0, 0, lane);
+            mma16(x, a31, S, 16, 0, lane);
+            mma16(x, a32, S, 32, 0, lane);
+            finish(3, 0, x);
+        }
     } else if (wid == 1) {
-        { const Frag16 As[1] = {a21}; const int ks[1] = {1}; block(2, 1, As, ks, 1); }
-        { const Frag16 As[2] = {a31, a32}; const int ks[2] = {1, 2}; block(3, 1, As, ks, 2); }
+        {
+            float x[2][4] = {};
+            mma16(x, a21, S, 16, 16, lane);
+            finish(2, 1, x);
+        }
+        {
+            float x[2][4] = {};
+            mma16(x, a31, S, 16, 16, lane);
+            mma16(x, a32, S, 32, 16, lane);
+            finish(3, 1, x);
+        }
     } else if (wid == 2) {
-        { const Frag16 As[1] = {a32}; const int ks[1] = {2}; block(3, 2, As, ks, 1); }
+        float x[2][4] = {};
+        mma16(x, a32, S, 32, 32, lane);
+        finish(3, 2, x);
     }
     named_bar_sync(bar_id, 128);
 }
@@ -281,10 +308,10 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     if (tid == 0) {
         for (int b = 0; b < (int)L::N_BARS; ++b) {
-            const uint32_t cnt = (b == B_S1_FREE || b == B_TP_READY || b == B_PREP || b == B_PREP + 1 ||
-                                  b == B_U_CONV || b == B_O_FREE || b == B_V_EMPTY)
-                                     ? 128u
-                                     : (b == B_H_READY ? 256u : 1u);
+            const uint32_t cnt =
+                (b == B_S1_FREE || b == B_TP_READY || b == B_PREP || b == B_PREP + 1)
+                    ? 256u
+                    : ((b == B_U_CONV || b == B_O_FREE || b == B_H_READY || b == B_HM_READY) ? 128u : 1u);
             mbar_init(&bars[b], cnt);
         }
         *abort_flag = 0;
@@ -354,12 +381,14 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             gs.G[2 * lane + 1] = G1;
             gs.beta[2 * lane] = bv[0];
             gs.beta[2 * lane + 1] = bv[1];
-            gs.f[2 * lane] = exp2f(Glast - G0);
-            gs.f[2 * lane + 1] = exp2f(Glast - G1);
-            gs.eG[2 * lane] = exp2f(G0);
-            gs.eG[2 * lane + 1] = exp2f(G1);
+            gs.f[2 * lane] = ex2_approx(Glast - G0);
+            gs.f[2 * lane + 1] = ex2_approx(Glast - G1);
+            gs.eG[2 * lane] = ex2_approx(G0);
+            gs.eG[2 * lane + 1] = ex2_approx(G1);
+            gs.a[2 * lane] = ex2_approx(gv[0] * kLog2e);
+            gs.a[2 * lane + 1] = ex2_approx(gv[1] * kLog2e);
             if (lane == 0) {
-                gs.gamma = exp2f(Glast);
+                gs.gamma = ex2_approx(Glast);
                 gs.L = Lc;
             }
             __syncwarp();
@@ -428,20 +457,23 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const uint32_t kq = sbase + L::KQ + st * L::KQ_STAGE;
                 if (!mbar_wait(&bars[B_PREP + st], (c >> 1) & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[B_V_FULL], c & 1, abort_flag, err)) break;
-                if (!mbar_wait(&bars[B_H_READY], c & 1, abort_flag, err)) break;
                 // the previous chunk's O^T MMAs read U from TM_U, which U^T below overwrites
                 if (c >= 1 && !mbar_wait(&bars[B_O_FULL], (c - 1) & 1, abort_flag, err)) break;
                 tc_fence_after();
-                // U^T = V^T T''^T - h^T W^T   (the diagonal beta_r v_r of T'' V is added by the epilogue)
+                // U^T = V^T (T''_hi + T''_lo)^T - h^T W^T ; the first half does not need the state
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem + TM_U, desc_mn_sw128(sbase + L::V + kk * 2048, 8192),
-                              desc_k_sw128(sbase + L::TPP + st * 8192 + kk * 32), id_u1, kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_bf16(tmem + TM_U, desc_mn_sw128(sbase + L::V + (kk & 3) * 2048, 8192),
+                              desc_k_sw128(sbase + (kk < 4 ? L::TPP : L::TPPL) + st * 8192 + (kk & 3) * 32), id_u1,
+                              kk > 0);
+                if (!mbar_wait(&bars[B_H_READY], c & 1, abort_flag, err)) break;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma_bf16(tmem + TM_U, desc_k_sw128(sbase + L::HT + (kk >> 2) * 16384 + (kk & 3) * 32),
                               desc_mn_sw128(sbase + L::WT + kk * 2048, 8192), id_u2, 1);
                 umma_commit(&bars[B_U_FULL]);
+                umma_commit(&bars[B_V_EMPTY]);
                 // O1^T = h^T Q^T (scaled by 2^G_r in the epilogue)
                 if (c >= 1 && !mbar_wait(&bars[B_O_FREE], (c - 1) & 1, abort_flag, err)) break;
                 tc_fence_after();
@@ -451,6 +483,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                               desc_k_sw128(kq + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32), id_o, kk > 0);
                 // h^T += (U diag f)^T K  (hi and lo halves) ;  O2^T = U^T P^T  (hi*hi + hi*lo + lo*hi)
                 if (!mbar_wait(&bars[B_U_CONV], c & 1, abort_flag, err)) break;
+                if (!mbar_wait(&bars[B_HM_READY], c & 1, abort_flag, err)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -472,76 +505,93 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             drain_wait(&bars[B_DRAIN + 1], 0);
         }
         __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
-        // ================================================================ prep warpgroup
-        // A timed-out wait does not break out here: the warpgroup finishes the iteration (with whatever data)
-        // and leaves together at the top of the next one, so no thread is left waiting at a named barrier.
-        const int t = tid - 128, wid = warp - 4;
+    } else if (warp >= 4 && warp < 12) {
+        // ================================================================ prep warpgroups
+        // A timed-out wait does not break out here: the warpgroups finish the iteration (with whatever data)
+        // and leave together at the top of the next one, so no thread is left waiting at a named barrier.
+        const int wsel = (warp - 4) >> 2;      // 0: chunk columns 0-31, 1: columns 32-63
+        const int t = (tid - 128) & 127;       // row of S1 / line of W^T (TMEM lane)
+        const int wid = warp & 3;
+        const int tp = tid - 128;              // 0..255 across both warpgroups
         for (int c = 0; c < nc; ++c) {
-            if (named_bar_or(2, 128, *abort_flag != 0)) break;
+            if (named_bar_or(2, 256, *abort_flag != 0)) break;
             const int st = c & 1;
             warp_wait(&bars[B_S1_FULL], c & 1, abort_flag, err);
             tc_fence_after();
-            float s1[64];
-            {
-                float v[32];
-                tmem_ld32(taddr(tmem, 32 * wid, TM_S1), v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 32; ++q) s1[q] = v[q];
-                tmem_ld32(taddr(tmem, 32 * wid, TM_S1 + 32), v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 32; ++q) s1[32 + q] = v[q];
-            }
+            float s1[32];
+            tmem_ld32(taddr(tmem, 32 * wid, TM_S1 + 32 * wsel), s1);
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bars[B_S1_FREE]);
             warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err);
             const TcGate& gs = gates[c & 3];
-            if (t < 64) {  // A row r
-                const int r = t;
-                const float Gr = gs.G[r], br = gs.beta[r];
+            // Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1): a running product from the highest column of
+            // this half at or below r, started there with one exp2
+            {
+                const int r = t & 63;
+                const int s_hi = 32 * wsel + 31;
+                const int top = r < s_hi ? r : s_hi;
+                float run = (top == r) ? 1.f : ex2_approx(gs.G[r] - gs.G[top]);
+                if (t < 64) {  // A row r: beta_r Gamma_rs (k_r . k_s), s < r
+                    const float br = gs.beta[r];
+                    float arow[32];
 #pragma unroll
-                for (int s = 0; s < 64; ++s)
-                    sA[r * L::AS_LD + s] = (s < r) ? br * exp2f(Gr - gs.G[s]) * s1[s] : 0.f;
-            } else {  // P row r, split into bf16 hi + lo
-                const int r = t - 64;
-                if (c >= 2) warp_wait(&bars[B_P_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err);
-                const float Gr = gs.G[r];
-                float lo[64];
+                    for (int q = 31; q >= 0; --q) {
+                        const int s = 32 * wsel + q;
+                        arow[q] = (s < r) ? br * run * s1[q] : 0.f;
+                        if (s <= top && s > 0) run *= gs.a[s];
+                    }
 #pragma unroll
-                for (int s = 0; s < 64; ++s) {
-                    const float x = (s <= r) ? exp2f(Gr - gs.G[s]) * s1[s] : 0.f;
-                    split_bf16(x, s1[s], lo[s]);
+                    for (int q = 0; q < 32; q += 4)
+                        *reinterpret_cast<float4*>(&sA[r * L::AS_LD + 32 * wsel + q]) =
+                            make_float4(arow[q], arow[q + 1], arow[q + 2], arow[q + 3]);
+                } else {  // P row r: Gamma_rs (q_r . k_s), s <= r, split into bf16 hi + lo
+                    if (c >= 2) warp_wait(&bars[B_P_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err);
+#pragma unroll
+                    for (int ch = 3; ch >= 0; --ch) {
+                        float xh[8], xl[8];
+#pragma unroll
+                        for (int q = 7; q >= 0; --q) {
+                            const int qq = 8 * ch + q, s = 32 * wsel + qq;
+                            const float x = (s <= r) ? run * s1[qq] : 0.f;
+                            if (s <= top && s > 0) run *= gs.a[s];
+                            split_bf16(x, xh[q], xl[q]);
+                        }
+                        const uint32_t off = sw128(r, 4 * wsel + ch);
+                        *reinterpret_cast<uint4*>(sm + L::PH + st * 8192 + off) =
+                            make_uint4(pack_bf16(xh[0], xh[1]), pack_bf16(xh[2], xh[3]), pack_bf16(xh[4], xh[5]),
+                                       pack_bf16(xh[6], xh[7]));
+                        *reinterpret_cast<uint4*>(sm + L::PL + st * 8192 + off) =
+                            make_uint4(pack_bf16(xl[0], xl[1]), pack_bf16(xl[2], xl[3]), pack_bf16(xl[4], xl[5]),
+                                       pack_bf16(xl[6], xl[7]));
+                    }
                 }
-                st_line_bf16(sm + L::PH + st * 8192, r, s1);
-                st_line_bf16(sm + L::PL + st * 8192, r, lo);
             }
-            named_bar_sync(1, 128);
-            invert_unit_lower64(sA, wid, lane, 1);
-            {  // T' = T diag(beta 2^G) and T'' = T diag(beta) without its diagonal, bf16, [r][s] K-major
-                const int r = t >> 1, half = t & 1;
-                float x1[32], x2[32];
+            named_bar_sync(1, 256);
+            if (wsel == 0) invert_unit_lower64(sA, wid, lane, 3);
+            named_bar_sync(1, 256);
+            {  // T' = T diag(beta 2^G) (bf16) and T'' = T diag(beta) (bf16 hi + lo), [r][s] K-major
+                const int r = tp >> 2, qd = tp & 3;  // 16 columns [16 qd, 16 qd + 16) of row r
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int s = 32 * half + q;
-                    const float tv = sA[r * L::AS_LD + s];
-                    x1[q] = tv * gs.beta[s] * gs.eG[s];
-                    x2[q] = (s == r) ? 0.f : tv * gs.beta[s];
-                }
+                for (int ch = 0; ch < 2; ++ch) {
+                    float x1[8], xh[8], xl[8];
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint4 u1, u2;
-                    u1.x = pack_bf16(x1[8 * ch + 0], x1[8 * ch + 1]);
-                    u1.y = pack_bf16(x1[8 * ch + 2], x1[8 * ch + 3]);
-                    u1.z = pack_bf16(x1[8 * ch + 4], x1[8 * ch + 5]);
-                    u1.w = pack_bf16(x1[8 * ch + 6], x1[8 * ch + 7]);
-                    u2.x = pack_bf16(x2[8 * ch + 0], x2[8 * ch + 1]);
-                    u2.y = pack_bf16(x2[8 * ch + 2], x2[8 * ch + 3]);
-                    u2.z = pack_bf16(x2[8 * ch + 4], x2[8 * ch + 5]);
-                    u2.w = pack_bf16(x2[8 * ch + 6], x2[8 * ch + 7]);
-                    *reinterpret_cast<uint4*>(sm + L::TP + sw128(r, 4 * half + ch)) = u1;
-                    *reinterpret_cast<uint4*>(sm + L::TPP + st * 8192 + sw128(r, 4 * half + ch)) = u2;
+                    for (int q = 0; q < 8; ++q) {
+                        const int s = 16 * qd + 8 * ch + q;
+                        const float tb = sA[r * L::AS_LD + s] * gs.beta[s];
+                        x1[q] = tb * gs.eG[s];
+                        split_bf16(tb, xh[q], xl[q]);
+                    }
+                    const uint32_t off = sw128(r, 2 * qd + ch);
+                    *reinterpret_cast<uint4*>(sm + L::TP + off) =
+                        make_uint4(pack_bf16(x1[0], x1[1]), pack_bf16(x1[2], x1[3]), pack_bf16(x1[4], x1[5]),
+                                   pack_bf16(x1[6], x1[7]));
+                    *reinterpret_cast<uint4*>(sm + L::TPP + st * 8192 + off) =
+                        make_uint4(pack_bf16(xh[0], xh[1]), pack_bf16(xh[2], xh[3]), pack_bf16(xh[4], xh[5]),
+                                   pack_bf16(xh[6], xh[7]));
+                    *reinterpret_cast<uint4*>(sm + L::TPPL + st * 8192 + off) =
+                        make_uint4(pack_bf16(xl[0], xl[1]), pack_bf16(xl[2], xl[3]), pack_bf16(xl[4], xl[5]),
+                                   pack_bf16(xl[6], xl[7]));
                 }
             }
             fence_proxy_async();
@@ -549,57 +599,50 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             warp_wait(&bars[B_W_FULL], c & 1, abort_flag, err);
             if (c >= 1) warp_wait(&bars[B_U_FULL], (c - 1) & 1, abort_flag, err);
             tc_fence_after();
-            {  // -W^T line i = t: 64 values over r
-                float v[32], w[64];
-                tmem_ld32(taddr(tmem, 32 * wid, TM_W), v);
+            {  // -W^T line i = t, columns r of this half
+                float v[32];
+                tmem_ld32(taddr(tmem, 32 * wid, TM_W + 32 * wsel), v);
                 tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 32; ++q) w[q] = v[q];
-                tmem_ld32(taddr(tmem, 32 * wid, TM_W + 32), v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 32; ++q) w[32 + q] = v[q];
-                st_line_bf16(sm + L::WT, t, w, -1.f);
+                st_half_line_bf16(sm + L::WT, t, 4 * wsel, v, -1.f);
             }
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bars[B_PREP + st]);
         }
-    } else if (warp >= 8) {
-        // ================================================================ epilogue warpgroups
-        const bool wg2 = warp < 12;
-        const int j = tid & 127;          // value column (TMEM lane)
-        const int ib = wg2 ? 0 : 64;      // key channels of the state this thread refreshes
+    } else if (warp >= 12) {
+        // ================================================================ epilogue warpgroup
+        const int j = tid & 127;  // value column (TMEM lane)
         const uint32_t lane_base = 32 * (warp & 3);
         // initial state: bf16 copy and fp32 master pre-scaled by the first chunk's decay
         if (warp_wait(&bars[B_GATE + 0], 0, abort_flag, err)) {
             const float g0 = gates[0].gamma;
-            float hv[64];
-#pragma unroll
-            for (int q = 0; q < 64; ++q)
-                hv[q] = p.h0 ? p.h0[state_base + (size_t)(ib + q) * dv + j] : 0.f;
-            st_line_bf16(sm + L::HT + (wg2 ? 0 : 16384), j, hv);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+#pragma unroll 1
+            for (int piece = 0; piece < 4; ++piece) {
                 float v[32];
+                const float* hp = p.h0 ? p.h0 + state_base + (size_t)(32 * piece) * dv + j : nullptr;
 #pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] = g0 * hv[32 * half + q];
-                tmem_st32(taddr(tmem, lane_base, TM_H + ib + 32 * half), v);
+                for (int q = 0; q < 32; ++q) {
+                    v[q] = hp ? *hp : 0.f;
+                    hp += hp ? dv : 0;
+                }
+                st_half_line_bf16(sm + L::HT + (piece >> 1) * 16384, j, 4 * (piece & 1), v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) v[q] *= g0;
+                tmem_st32(taddr(tmem, lane_base, TM_H + 32 * piece), v);
             }
             tmem_wait_st();
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bars[B_H_READY]);
+            mbar_arrive(&bars[B_HM_READY]);
         }
-        // V tile column j: 16-bit element of line r in the MN-major block (j / 64)
-        const uint8_t* vcol = sm + L::V + (j >> 6) * 8192 + ((j & 63) & 7) * 2;
-        const uint32_t vchunk = (j & 63) >> 3;
         for (int c = 0; c < nc; ++c) {
             const TcGate& gs = gates[c & 3];
-            if (wg2) {
-                if (!warp_wait(&bars[B_U_FULL], c & 1, abort_flag, err)) break;
-                if (!warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err)) break;
-                tc_fence_after();
+            // ---- U: fp32 accumulator -> bf16 hi/lo pairs for U and U diag f
+            if (!warp_wait(&bars[B_U_FULL], c & 1, abort_flag, err)) break;
+            if (!warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err)) break;
+            tc_fence_after();
+            {
                 float u[64];
                 {
                     float v[32];
@@ -612,97 +655,97 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                     for (int q = 0; q < 32; ++q) u[32 + q] = v[q];
                 }
-                // diagonal of T'' V in fp32: u_r += beta_r v_r
+                // all of U is in registers before the first store overwrites its fp32 columns
 #pragma unroll
-                for (int r = 0; r < 64; ++r) {
-                    const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vcol + sw128(r, vchunk)));
-                    u[r] = fmaf(gs.beta[r], vv, u[r]);
-                }
-                mbar_arrive(&bars[B_V_EMPTY]);
-                // U and U diag f as bf16 hi/lo pairs, two per 32-bit TMEM column
-                uint32_t hi[32], lo[32];
+                for (int part = 0; part < 4; ++part) {
+                    const int half = part & 1;      // which 32 values of u
+                    const bool scaled = part >= 2;  // U diag f
+                    uint32_t hi[16], lo[16];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    float h0f, l0f, h1f, l1f;
-                    split_bf16(u[2 * q], h0f, l0f);
-                    split_bf16(u[2 * q + 1], h1f, l1f);
-                    hi[q] = pack_bf16(h0f, h1f);
-                    lo[q] = pack_bf16(l0f, l1f);
+                    for (int q = 0; q < 16; ++q) {
+                        const int s0 = 32 * half + 2 * q;
+                        const float x0 = scaled ? u[s0] * gs.f[s0] : u[s0];
+                        const float x1 = scaled ? u[s0 + 1] * gs.f[s0 + 1] : u[s0 + 1];
+                        float h0f, l0f, h1f, l1f;
+                        split_bf16(x0, h0f, l0f);
+                        split_bf16(x1, h1f, l1f);
+                        hi[q] = pack_bf16(h0f, h1f);
+                        lo[q] = pack_bf16(l0f, l1f);
+                    }
+                    const uint32_t base = scaled ? TM_UF : TM_U;
+                    tmem_st16u(taddr(tmem, lane_base, base + 16 * half), hi);
+                    tmem_st16u(taddr(tmem, lane_base, base + 32 + 16 * half), lo);
                 }
-                tmem_st32u(taddr(tmem, lane_base, TM_U), hi);
-                tmem_st32u(taddr(tmem, lane_base, TM_U + 32), lo);
-#pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    float h0f, l0f, h1f, l1f;
-                    split_bf16(u[2 * q] * gs.f[2 * q], h0f, l0f);
-                    split_bf16(u[2 * q + 1] * gs.f[2 * q + 1], h1f, l1f);
-                    hi[q] = pack_bf16(h0f, h1f);
-                    lo[q] = pack_bf16(l0f, l1f);
-                }
-                tmem_st32u(taddr(tmem, lane_base, TM_UF), hi);
-                tmem_st32u(taddr(tmem, lane_base, TM_UF + 32), lo);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&bars[B_U_CONV]);
             }
-            // state refresh
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[B_U_CONV]);
+            // ---- state refresh: bf16 copy for the next chunk's MMAs, fp32 master times the next decay
             if (!warp_wait(&bars[B_H_FULL], c & 1, abort_flag, err)) break;
+            const bool last = c + 1 == nc;
+            if (!last && !warp_wait(&bars[B_GATE + ((c + 1) & 3)], ((c + 1) >> 2) & 1, abort_flag, err)) break;
             tc_fence_after();
-            float hv[64];
-            {
+            const float gn = last ? 1.f : gates[(c + 1) & 3].gamma;
+            // pass 1: the bf16 copy (what the next chunk's first MMAs wait for), or hT after the last chunk
+#pragma unroll 1
+            for (int piece = 0; piece < 4; ++piece) {
                 float v[32];
-                tmem_ld32(taddr(tmem, lane_base, TM_H + ib), v);
+                tmem_ld32(taddr(tmem, lane_base, TM_H + 32 * piece), v);
                 tmem_wait_ld();
+                if (!last) {
+                    st_half_line_bf16(sm + L::HT + (piece >> 1) * 16384, j, 4 * (piece & 1), v);
+                } else if (p.hT) {
+                    float* hp = p.hT + state_base + (size_t)(32 * piece) * dv + j;
 #pragma unroll
-                for (int q = 0; q < 32; ++q) hv[q] = v[q];
-                tmem_ld32(taddr(tmem, lane_base, TM_H + ib + 32), v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 32; ++q) hv[32 + q] = v[q];
-            }
-            if (c + 1 < nc) {
-                if (!warp_wait(&bars[B_GATE + ((c + 1) & 3)], ((c + 1) >> 2) & 1, abort_flag, err)) break;
-                const float gn = gates[(c + 1) & 3].gamma;
-                st_line_bf16(sm + L::HT + (wg2 ? 0 : 16384), j, hv);
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float v[32];
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) v[q] = gn * hv[32 * half + q];
-                    tmem_st32(taddr(tmem, lane_base, TM_H + ib + 32 * half), v);
+                    for (int q = 0; q < 32; ++q) {
+                        *hp = v[q];
+                        hp += dv;
+                    }
                 }
-                tmem_wait_st();
-                fence_proxy_async();
-                tc_fence_before();
-                mbar_arrive(&bars[B_H_READY]);
-            } else if (p.hT) {
-#pragma unroll 8
-                for (int q = 0; q < 64; ++q) p.hT[state_base + (size_t)(ib + q) * dv + j] = hv[q];
             }
-            if (!wg2) {  // output o_r = scale (2^G_r O1_r + O2_r)
-                if (!warp_wait(&bars[B_O_FULL], c & 1, abort_flag, err)) break;
-                tc_fence_after();
-                float ov[64];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float v1[32], v2[32];
-                    tmem_ld32(taddr(tmem, lane_base, TM_O1 + 32 * half), v1);
-                    tmem_ld32(taddr(tmem, lane_base, TM_O2 + 32 * half), v2);
+            if (!last) {
+                fence_proxy_async();
+                mbar_arrive(&bars[B_H_READY]);
+                // pass 2: the fp32 master times the next chunk's decay (needed only by the next h^T MMA)
+#pragma unroll 1
+                for (int piece = 0; piece < 4; ++piece) {
+                    float v[32];
+                    tmem_ld32(taddr(tmem, lane_base, TM_H + 32 * piece), v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) ov[32 * half + q] = fmaf(gs.eG[32 * half + q], v1[q], v2[q]);
+                    for (int q = 0; q < 32; ++q) v[q] *= gn;
+                    tmem_st32(taddr(tmem, lane_base, TM_H + 32 * piece), v);
                 }
+                tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars[B_O_FREE]);
-                const int Lc = gs.L;
-                const size_t tok0 = (size_t)row * T + bos + (size_t)c * kChunk;
-#pragma unroll 8
-                for (int r = 0; r < 64; ++r) {
+                mbar_arrive(&bars[B_HM_READY]);
+            }
+            // ---- output o_r = scale (2^G_r O1_r + O2_r)
+            if (!warp_wait(&bars[B_O_FULL], c & 1, abort_flag, err)) break;
+            tc_fence_after();
+            const int Lc = gs.L;
+            const size_t tok0 = (size_t)row * T + bos + (size_t)c * kChunk;
+            const size_t ostride = (size_t)H * dv;
+            size_t off = (tok0 * H + h) * (size_t)dv + j0 + j;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float v1[32], v2[32];
+                tmem_ld32(taddr(tmem, lane_base, TM_O1 + 32 * half), v1);
+                tmem_ld32(taddr(tmem, lane_base, TM_O2 + 32 * half), v2);
+                tmem_wait_ld();
+                if (half == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&bars[B_O_FREE]);
+                }
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int r = 32 * half + q;
                     if (r < Lc) {
-                        const size_t off = ((tok0 + r) * H + h) * (size_t)dv + j0 + j;
-                        if (O_F32) static_cast<float*>(p.o)[off] = p.scale * ov[r];
-                        else static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(p.scale * ov[r]);
+                        const float val = p.scale * fmaf(gs.eG[r], v1[q], v2[q]);
+                        if (O_F32) static_cast<float*>(p.o)[off] = val;
+                        else static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(val);
                     }
+                    off += ostride;
                 }
             }
         }
