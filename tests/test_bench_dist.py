@@ -1,0 +1,50 @@
+"""CPU (gloo) tests of the multi-rank logic of bench.py: the max-over-ranks timing, the whole-job
+throughput, and that the reference arm runs on rank 0 only."""
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, ws, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(ws),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        t = bench.max_over_ranks(10.0 + 5.0 * rank, ws)  # each rank's elapsed ms
+        bench.barrier(ws)
+        q.put((rank, t, bench.job_throughput(1000, ws, t)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws", [2])
+def test_max_over_ranks_and_throughput(ws):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_worker, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(ws))
+    slowest = 10.0 + 5.0 * (ws - 1)
+    for rank, t, thr in res:
+        assert t == slowest  # every rank sees the max
+        assert abs(thr - ws * 1000 / (slowest * 1e-3)) < 1e-6
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0 and out.stdout.strip() == ""
