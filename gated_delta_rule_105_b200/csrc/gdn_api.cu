@@ -117,9 +117,13 @@ static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, gdn_dtype o_d
     const bool use_tc = tc_ok && choice != GDN_KERNEL_SIMT;
     if (use_tc) {
         st = launch_tc(p, gdn2, o_dt == GDN_F32, err, stream);
-        if (st == GDN_OK) t_last_kernel = GDN_KERNEL_TC;
-        else if (st == GDN_ERR_CUDA) fail(st, "tcgen05 kernel launch: %s", tc_last_error());
-        return st;
+        if (st == GDN_OK) {
+            t_last_kernel = GDN_KERNEL_TC;
+            return st;
+        }
+        fail(st, "tcgen05 kernel: %s", tc_last_error());
+        if (st != GDN_ERR_UNSUPPORTED || choice == GDN_KERNEL_TC) return st;
+        // AUTO: a configuration the tcgen05 build cannot take runs on the SIMT kernel
     }
     st = gdn2 ? launch_simt<true>(p, dt, o_dt, err, stream) : launch_simt<false>(p, dt, o_dt, err, stream);
     if (st == GDN_OK) t_last_kernel = GDN_KERNEL_SIMT;

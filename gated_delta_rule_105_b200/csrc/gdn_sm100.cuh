@@ -189,6 +189,14 @@ __device__ __forceinline__ uint32_t taddr(uint32_t base, uint32_t lane, uint32_t
     return base + (lane << 16) + col;
 }
 
+// 32 lanes x 8 consecutive 32-bit columns: thread t of the warp gets lane (lane_base + t).
+__device__ __forceinline__ void tmem_ld8(uint32_t ta, float (&v)[8]) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(ta)
+                 : "memory");
+}
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane (lane_base + t).
 __device__ __forceinline__ void tmem_ld32(uint32_t ta, float (&v)[32]) {
     uint32_t* r = reinterpret_cast<uint32_t*>(v);
@@ -247,6 +255,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ void split_bf16(float x, float& hi, float& lo) {
     hi = __bfloat162float(__float2bfloat16_rn(x));
     lo = x - hi;
+}
+// Packed hi/lo split of a pair: hi = bf16x2(x0, x1), lo = bf16x2(x0 - hi0, x1 - hi1).
+__device__ __forceinline__ void split_pack_bf16(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h2);
+    const __nv_bfloat162 l2 = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h2);
+    lo = *reinterpret_cast<const uint32_t*>(&l2);
 }
 // Writes 32 values as bf16 into 16-byte chunks c0 .. c0+3 of line `line` of a 128B-swizzled region.
 __device__ __forceinline__ void st_half_line_bf16(uint8_t* region, uint32_t line, int c0, const float (&x)[32],

@@ -20,11 +20,11 @@
 // This is the WY form of the intra-chunk dependency with one state handed from chunk to chunk
 // (GatedDeltaNet data-flow walkthrough, yfxerp.com/news/367755, section "Chunked parallelism").
 //
-// Warp roles (16 warps): 0 TMA producer and gate prep; 1 issues the h-independent MMAs (S1, W^T) one chunk
+// Warp roles (20 warps): 0 TMA producer and gate prep; 1 issues the h-independent MMAs (S1, W^T) one chunk
 // ahead; 2 issues the serial MMAs (U^T, O^T, h^T); 3 idle; 4-7 and 8-11 (two prep warpgroups, one per half
-// of the 64 chunk columns) build A, P, T', T'' and -W^T, the first of them also (I+A)^-1; 12-15 (epilogue
-// warpgroup) split U into bf16 operands, refresh the bf16 copy of h^T and re-scale the fp32 state by the
-// next chunk's decay, and write o and hT.
+// of the 64 chunk columns) build A, P, T', T'' and -W^T, the first of them also (I+A)^-1; 12-15 (state
+// warpgroup) split U into bf16 operands, refresh the bf16 copy of h^T, re-scale the fp32 state by the next
+// chunk's decay and write hT; 16-19 (output warpgroup) write o.
 // All mbarrier waits are bounded: on time-out the CTA sets the error word and drains to the exit.
 #pragma once
 
@@ -34,7 +34,8 @@
 
 namespace gdn {
 
-constexpr int kTcThreads = 512;
+constexpr int kTcThreads = 640;
+
 constexpr int kTcDV = 128;  // value columns per CTA
 constexpr int kTcDK = 128;  // key dimension handled by this kernel
 
@@ -96,8 +97,8 @@ enum TcBar : int {
     B_HM_READY = 26,  // fp32 state in TMEM re-scaled by the next chunk's decay (128)
 };
 
-// TMEM columns.  U^T is accumulated in fp32 at TM_U, then replaced in place by its bf16 hi (TM_U .. +31)
-// and lo (TM_U + 32 .. +63) halves, two values per column; (U diag f)^T hi/lo sit at TM_UF likewise.
+// TMEM columns.  U^T is accumulated in fp32 at TM_U; the state warpgroup then writes U as bf16 hi/lo pairs
+// (two values per column) to TM_UF and U diag f, also as hi/lo pairs, in place over TM_U.
 constexpr uint32_t TM_S1 = 0, TM_W = 64, TM_U = 128, TM_UF = 192, TM_O1 = 256, TM_O2 = 320, TM_H = 384,
                    TM_COLS = 512;
 
@@ -115,70 +116,65 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-// Fragments of a 16x16 fp32 block at (r0, c0) of the [64][68] scratch.
+// 16x16 blocks of the [64][68] fp32 scratch, as tf32 mma.sync fragments.  A block is named by its logical
+// origin (r0, c0); `tr` = it is stored transposed in the mirrored position (element (r, c) of the logical
+// block at scratch row c0 + c, column r0 + r).
 struct Frag16 {
     uint32_t a[2][4];  // as the A operand: k-halves 0, 1
 };
-__device__ __forceinline__ void load_a16(const float* S, int r0, int c0, int lane, Frag16& f) {
+__device__ __forceinline__ float blk(const float* S, int r0, int c0, int r, int c, bool tr) {
+    return tr ? S[(c0 + c) * TcSmem::AS_LD + r0 + r] : S[(r0 + r) * TcSmem::AS_LD + c0 + c];
+}
+__device__ __forceinline__ void load_a16(const float* S, int r0, int c0, bool tr, int lane, Frag16& f) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int kh = 0; kh < 2; ++kh) {
-        const int c = c0 + 8 * kh;
-        f.a[kh][0] = f2tf32(S[(r0 + g) * TcSmem::AS_LD + c + t]);
-        f.a[kh][1] = f2tf32(S[(r0 + g + 8) * TcSmem::AS_LD + c + t]);
-        f.a[kh][2] = f2tf32(S[(r0 + g) * TcSmem::AS_LD + c + t + 4]);
-        f.a[kh][3] = f2tf32(S[(r0 + g + 8) * TcSmem::AS_LD + c + t + 4]);
+        f.a[kh][0] = f2tf32(blk(S, r0, c0, g, 8 * kh + t, tr));
+        f.a[kh][1] = f2tf32(blk(S, r0, c0, g + 8, 8 * kh + t, tr));
+        f.a[kh][2] = f2tf32(blk(S, r0, c0, g, 8 * kh + t + 4, tr));
+        f.a[kh][3] = f2tf32(blk(S, r0, c0, g + 8, 8 * kh + t + 4, tr));
     }
 }
-// acc (16x16 as two 16x8 n-halves) += A-frag(16x16) * B(16x16 block at (r0, c0) of the scratch).
-__device__ __forceinline__ void mma16(float (&acc)[2][4], const Frag16& A, const float* S, int r0, int c0, int lane) {
+// acc (16x16 as two 16x8 n-halves) += A-frag(16x16) * B (16x16 block (r0, c0), transposed if tr).
+__device__ __forceinline__ void mma16(float (&acc)[2][4], const Frag16& A, const float* S, int r0, int c0, bool tr,
+                                      int lane) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh) {
 #pragma unroll
         for (int kh = 0; kh < 2; ++kh) {
             uint32_t b[2];
-            b[0] = f2tf32(S[(r0 + 8 * kh + t) * TcSmem::AS_LD + c0 + 8 * nh + g]);
-            b[1] = f2tf32(S[(r0 + 8 * kh + t + 4) * TcSmem::AS_LD + c0 + 8 * nh + g]);
+            b[0] = f2tf32(blk(S, r0, c0, 8 * kh + t, 8 * nh + g, tr));
+            b[1] = f2tf32(blk(S, r0, c0, 8 * kh + t + 4, 8 * nh + g, tr));
             mma_tf32(acc[nh], A.a[kh], b);
         }
     }
 }
-__device__ __forceinline__ void store16(float* S, int r0, int c0, int lane, const float (&acc)[2][4], float sgn) {
+// Stores sgn * acc into the 16x16 block (r0, c0), transposed if tr.
+__device__ __forceinline__ void store16(float* S, int r0, int c0, bool tr, int lane, const float (&acc)[2][4],
+                                        float sgn) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh) {
-        const int c = c0 + 8 * nh + 2 * t;
-        S[(r0 + g) * TcSmem::AS_LD + c] = sgn * acc[nh][0];
-        S[(r0 + g) * TcSmem::AS_LD + c + 1] = sgn * acc[nh][1];
-        S[(r0 + g + 8) * TcSmem::AS_LD + c] = sgn * acc[nh][2];
-        S[(r0 + g + 8) * TcSmem::AS_LD + c + 1] = sgn * acc[nh][3];
+        const int c = 8 * nh + 2 * t;
+        float* p00 = tr ? &S[(c0 + c) * TcSmem::AS_LD + r0 + g] : &S[(r0 + g) * TcSmem::AS_LD + c0 + c];
+        const int dc = tr ? TcSmem::AS_LD : 1, dr = tr ? 1 : TcSmem::AS_LD;
+        p00[0] = sgn * acc[nh][0];
+        p00[dc] = sgn * acc[nh][1];
+        p00[8 * dr] = sgn * acc[nh][2];
+        p00[8 * dr + dc] = sgn * acc[nh][3];
     }
 }
 
-// (I + A)^-1 in place for a strictly lower-triangular 64x64 A held in the [64][68] fp32 scratch, by the
-// 4 warps of the prep warpgroup.  Diagonal 16x16 blocks by forward substitution (one column per lane);
-// off-diagonal blocks by T_ij = -T_ii (sum_{k=j}^{i-1} A_ik T_kj), distance by distance, on tf32 MMAs.
-// Every A block an off-diagonal step needs is read into registers before any block is overwritten.
+// (I + A)^-1 for a strictly lower-triangular 64x64 A in the [64][68] fp32 scratch (upper triangle 0), by
+// the 4 warps of one warpgroup.  On return the diagonal 16x16 blocks hold T_ii in place, each
+// off-diagonal block T_ij (i > j) is stored transposed in the upper-triangle block (j, i), and the lower
+// off-diagonal blocks of A are left intact.  Steps: the four diagonal blocks by forward substitution (one
+// column per lane); T_10 = -T_11 A_10 T_00 and T_32 = -T_33 A_32 T_22; then the lower-left 32x32 quarter
+// T_c = -T_b (A_c T_a), where T_a, T_b are the inverses of the two diagonal 32x32 quarters -- each block
+// product on tf32 MMAs, at most two per warp per step.
 __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane, uint32_t bar_id) {
     using namespace sm100;
-    // A blocks each warp needs: warp 0: A10 A20 A21 A30 A31 A32; warp 1: A21 A31 A32; warp 2: A32.
-    Frag16 a10, a20, a21, a30, a31, a32;
-    if (wid == 0) {
-        load_a16(S, 16, 0, lane, a10);
-        load_a16(S, 32, 0, lane, a20);
-        load_a16(S, 32, 16, lane, a21);
-        load_a16(S, 48, 0, lane, a30);
-        load_a16(S, 48, 16, lane, a31);
-        load_a16(S, 48, 32, lane, a32);
-    } else if (wid == 1) {
-        load_a16(S, 32, 16, lane, a21);
-        load_a16(S, 48, 16, lane, a31);
-        load_a16(S, 48, 32, lane, a32);
-    } else if (wid == 2) {
-        load_a16(S, 48, 32, lane, a32);
-    }
-    // diagonal block wid: lane c (< 16) computes column c of (I + A_bb)^-1
     {
         const int b0 = 16 * wid, c = lane & 15;
         float t[16];
@@ -195,57 +191,59 @@ __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane,
             for (int r = 0; r < 16; ++r) S[(b0 + r) * TcSmem::AS_LD + b0 + c] = t[r];
         }
     }
-    named_bar_sync(bar_id, 128);  // every diagonal inverse (and every A-block read) done
-    // off-diagonal blocks, within one warp each: X = sum_k A_ik T_kj, parked in slot (i, j); T_ij = -T_ii X
-    auto finish = [&](int i, int j, const float (&x)[2][4]) {
-        __syncwarp();
-        store16(S, 16 * i, 16 * j, lane, x, 1.f);
-        __syncwarp();
-        Frag16 tii;
-        load_a16(S, 16 * i, 16 * i, lane, tii);
-        float y[2][4] = {};
-        mma16(y, tii, S, 16 * i, 16 * j, lane);
-        __syncwarp();
-        store16(S, 16 * i, 16 * j, lane, y, -1.f);
-        __syncwarp();
-    };
-    if (wid == 0) {
-        {
-            float x[2][4] = {};
-            mma16(x, a10, S, 0, 0, lane);
-            finish(1, 0, x);
-        }
-        {
-            float x[2][4] = {};
-            mma16(x, a20, S, 0, 0, lane);
-            mma16(x, a21, S, 16, 0, lane);
-            finish(2, 0, x);
-        }
-        {
-            float x[2][4] = {};
-            mma16(x, a30, S, 0, 0, lane);
-            mma16(x, a31, S, 16, 0, lane);
-            mma16(x, a32, S, 32, 0, lane);
-            finish(3, 0, x);
-        }
-    } else if (wid == 1) {
-        {
-            float x[2][4] = {};
-            mma16(x, a21, S, 16, 16, lane);
-            finish(2, 1, x);
-        }
-        {
-            float x[2][4] = {};
-            mma16(x, a31, S, 16, 16, lane);
-            mma16(x, a32, S, 32, 16, lane);
-            finish(3, 1, x);
-        }
-    } else if (wid == 2) {
+    named_bar_sync(bar_id, 128);
+    // T_10 (warp 0) and T_32 (warp 1): X = A_ij T_jj, then T_ij = -T_ii X
+    if (wid < 2) {
+        const int i = 1 + 2 * wid, j = 2 * wid;
+        Frag16 f;
+        load_a16(S, 16 * i, 16 * j, false, lane, f);
         float x[2][4] = {};
-        mma16(x, a32, S, 32, 32, lane);
-        finish(3, 2, x);
+        mma16(x, f, S, 16 * j, 16 * j, false, lane);
+        store16(S, 16 * i, 16 * j, true, lane, x, 1.f);
+        __syncwarp();
+        load_a16(S, 16 * i, 16 * i, false, lane, f);
+        float y[2][4] = {};
+        mma16(y, f, S, 16 * i, 16 * j, true, lane);
+        __syncwarp();
+        store16(S, 16 * i, 16 * j, true, lane, y, -1.f);
     }
     named_bar_sync(bar_id, 128);
+    // X = A_c T_a for the blocks (p, q), p in {2, 3}, q in {0, 1}; one block per warp, parked in (p, q)
+    const int p = 2 + (wid >> 1), q = wid & 1;
+    {
+        Frag16 f;
+        float x[2][4] = {};
+        load_a16(S, 16 * p, 16 * q, false, lane, f);  // A_pq T_qq
+        mma16(x, f, S, 16 * q, 16 * q, false, lane);
+        if (q == 0) {  // + A_p1 T_10
+            load_a16(S, 16 * p, 16, false, lane, f);
+            mma16(x, f, S, 16, 0, true, lane);
+        }
+        store16(S, 16 * p, 16 * q, true, lane, x, 1.f);
+    }
+    named_bar_sync(bar_id, 128);
+    // T_c = -T_b X: T_2q = -T_22 X_2q ; T_3q = -(T_32 X_2q + T_33 X_3q)
+    {
+        Frag16 f;
+        float y[2][4] = {};
+        if (p == 2) {
+            load_a16(S, 32, 32, false, lane, f);
+            mma16(y, f, S, 32, 16 * q, true, lane);
+        } else {
+            load_a16(S, 48, 32, true, lane, f);
+            mma16(y, f, S, 32, 16 * q, true, lane);
+            load_a16(S, 48, 48, false, lane, f);
+            mma16(y, f, S, 48, 16 * q, true, lane);
+        }
+        named_bar_sync(bar_id, 128);  // every X block has been read
+        store16(S, 16 * p, 16 * q, true, lane, y, -1.f);
+    }
+    named_bar_sync(bar_id, 128);
+}
+// Element (r, s) of T = (I + A)^-1 as left by invert_unit_lower64.
+__device__ __forceinline__ float t_elem(const float* S, int r, int s) {
+    if (s > r) return 0.f;
+    return ((r >> 4) == (s >> 4)) ? S[r * TcSmem::AS_LD + s] : S[s * TcSmem::AS_LD + r];
 }
 
 // ------------------------------------------------------------------------------------------ the kernel
@@ -457,8 +455,6 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const uint32_t kq = sbase + L::KQ + st * L::KQ_STAGE;
                 if (!mbar_wait(&bars[B_PREP + st], (c >> 1) & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[B_V_FULL], c & 1, abort_flag, err)) break;
-                // the previous chunk's O^T MMAs read U from TM_U, which U^T below overwrites
-                if (c >= 1 && !mbar_wait(&bars[B_O_FULL], (c - 1) & 1, abort_flag, err)) break;
                 tc_fence_after();
                 // U^T = V^T (T''_hi + T''_lo)^T - h^T W^T ; the first half does not need the state
 #pragma unroll
@@ -486,14 +482,16 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (!mbar_wait(&bars[B_HM_READY], c & 1, abort_flag, err)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_bf16_tmem_a(tmem + TM_H, tmem + TM_UF + (kk >> 2) * 32 + (kk & 3) * 8,
-                                     desc_mn_sw128(kq + (kk & 3) * 2048, 16384), id_h, 1);
+                for (int kk = 0; kk < 8; ++kk) {  // kk < 4: hi, else lo; s-step ks covers values 16 ks .. 16 ks + 15
+                    const int ks = kk & 3;
+                    const uint32_t a = tmem + TM_U + (ks >> 1) * 32 + (kk >> 2) * 16 + (ks & 1) * 8;
+                    umma_bf16_tmem_a(tmem + TM_H, a, desc_mn_sw128(kq + ks * 2048, 16384), id_h, 1);
+                }
                 umma_commit(&bars[B_H_FULL]);
 #pragma unroll
                 for (int kk = 0; kk < 12; ++kk) {
                     const int part = kk >> 2, ks = kk & 3;  // 0: Uhi Phi, 1: Uhi Plo, 2: Ulo Phi
-                    const uint32_t a = tmem + TM_U + (part == 2 ? 32 : 0) + ks * 8;
+                    const uint32_t a = tmem + TM_UF + (part == 2 ? 32 : 0) + ks * 8;
                     const uint32_t b = sbase + (part == 1 ? L::PL : L::PH) + st * 8192 + ks * 32;
                     umma_bf16_tmem_a(tmem + TM_O2, a, desc_k_sw128(b), id_o, kk > 0);
                 }
@@ -518,45 +516,37 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const int st = c & 1;
             warp_wait(&bars[B_S1_FULL], c & 1, abort_flag, err);
             tc_fence_after();
-            float s1[32];
-            tmem_ld32(taddr(tmem, 32 * wid, TM_S1 + 32 * wsel), s1);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&bars[B_S1_FREE]);
             warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err);
             const TcGate& gs = gates[c & 3];
+            if (t >= 64 && c >= 2) warp_wait(&bars[B_P_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err);
             // Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1): a running product from the highest column of
-            // this half at or below r, started there with one exp2
+            // this half at or below r, started there with one exp2; 8 columns at a time, highest first
             {
                 const int r = t & 63;
                 const int s_hi = 32 * wsel + 31;
                 const int top = r < s_hi ? r : s_hi;
                 float run = (top == r) ? 1.f : ex2_approx(gs.G[r] - gs.G[top]);
-                if (t < 64) {  // A row r: beta_r Gamma_rs (k_r . k_s), s < r
-                    const float br = gs.beta[r];
-                    float arow[32];
+                const float br = (t < 64) ? gs.beta[r] : 1.f;
+#pragma unroll 1
+                for (int ch = 3; ch >= 0; --ch) {
+                    float s8[8];
+                    tmem_ld8(taddr(tmem, 32 * wid, TM_S1 + 32 * wsel + 8 * ch), s8);
+                    tmem_wait_ld();
+                    float x[8];
 #pragma unroll
-                    for (int q = 31; q >= 0; --q) {
-                        const int s = 32 * wsel + q;
-                        arow[q] = (s < r) ? br * run * s1[q] : 0.f;
+                    for (int q = 7; q >= 0; --q) {
+                        const int s = 32 * wsel + 8 * ch + q;
+                        x[q] = (t < 64 ? (s < r) : (s <= r)) ? br * run * s8[q] : 0.f;
                         if (s <= top && s > 0) run *= gs.a[s];
                     }
-#pragma unroll
-                    for (int q = 0; q < 32; q += 4)
-                        *reinterpret_cast<float4*>(&sA[r * L::AS_LD + 32 * wsel + q]) =
-                            make_float4(arow[q], arow[q + 1], arow[q + 2], arow[q + 3]);
-                } else {  // P row r: Gamma_rs (q_r . k_s), s <= r, split into bf16 hi + lo
-                    if (c >= 2) warp_wait(&bars[B_P_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err);
-#pragma unroll
-                    for (int ch = 3; ch >= 0; --ch) {
+                    if (t < 64) {  // A row r: beta_r Gamma_rs (k_r . k_s), s < r
+                        float* dst = &sA[r * L::AS_LD + 32 * wsel + 8 * ch];
+                        *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
+                        *reinterpret_cast<float4*>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
+                    } else {  // P row r: Gamma_rs (q_r . k_s), s <= r, bf16 hi + lo
                         float xh[8], xl[8];
 #pragma unroll
-                        for (int q = 7; q >= 0; --q) {
-                            const int qq = 8 * ch + q, s = 32 * wsel + qq;
-                            const float x = (s <= r) ? run * s1[qq] : 0.f;
-                            if (s <= top && s > 0) run *= gs.a[s];
-                            split_bf16(x, xh[q], xl[q]);
-                        }
+                        for (int q = 0; q < 8; ++q) split_bf16(x[q], xh[q], xl[q]);
                         const uint32_t off = sw128(r, 4 * wsel + ch);
                         *reinterpret_cast<uint4*>(sm + L::PH + st * 8192 + off) =
                             make_uint4(pack_bf16(xh[0], xh[1]), pack_bf16(xh[2], xh[3]), pack_bf16(xh[4], xh[5]),
@@ -567,6 +557,8 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&bars[B_S1_FREE]);
             named_bar_sync(1, 256);
             if (wsel == 0) invert_unit_lower64(sA, wid, lane, 3);
             named_bar_sync(1, 256);
@@ -578,7 +570,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const int s = 16 * qd + 8 * ch + q;
-                        const float tb = sA[r * L::AS_LD + s] * gs.beta[s];
+                        const float tb = t_elem(sA, r, s) * gs.beta[s];
                         x1[q] = tb * gs.eG[s];
                         split_bf16(tb, xh[q], xl[q]);
                     }
@@ -609,8 +601,8 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_before();
             mbar_arrive(&bars[B_PREP + st]);
         }
-    } else if (warp >= 12) {
-        // ================================================================ epilogue warpgroup
+    } else if (warp >= 12 && warp < 16) {
+        // ================================================================ state warpgroup
         const int j = tid & 127;  // value column (TMEM lane)
         const uint32_t lane_base = 32 * (warp & 3);
         // initial state: bf16 copy and fp32 master pre-scaled by the first chunk's decay
@@ -642,40 +634,26 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (!warp_wait(&bars[B_U_FULL], c & 1, abort_flag, err)) break;
             if (!warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err)) break;
             tc_fence_after();
-            {
-                float u[64];
-                {
-                    float v[32];
-                    tmem_ld32(taddr(tmem, lane_base, TM_U), v);
-                    tmem_wait_ld();
+            // U (for O2) as bf16 hi/lo pairs in TM_UF: hi of values 0-63 in columns 0-31, lo in 32-63.
+            // U diag f (for h^T) in place in TM_U, per 32 values: [hi 0-31 | lo 0-31 | hi 32-63 | lo 32-63],
+            // 16 columns each -- every column is read (as fp32) before it is overwritten.
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float u[32];
+                tmem_ld32(taddr(tmem, lane_base, TM_U + 32 * half), u);
+                tmem_wait_ld();
+                uint32_t hi[16], lo[16];
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) u[q] = v[q];
-                    tmem_ld32(taddr(tmem, lane_base, TM_U + 32), v);
-                    tmem_wait_ld();
+                for (int q = 0; q < 16; ++q) split_pack_bf16(u[2 * q], u[2 * q + 1], hi[q], lo[q]);
+                tmem_st16u(taddr(tmem, lane_base, TM_UF + 16 * half), hi);
+                tmem_st16u(taddr(tmem, lane_base, TM_UF + 32 + 16 * half), lo);
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) u[32 + q] = v[q];
+                for (int q = 0; q < 16; ++q) {
+                    const int s0 = 32 * half + 2 * q;
+                    split_pack_bf16(u[2 * q] * gs.f[s0], u[2 * q + 1] * gs.f[s0 + 1], hi[q], lo[q]);
                 }
-                // all of U is in registers before the first store overwrites its fp32 columns
-#pragma unroll
-                for (int part = 0; part < 4; ++part) {
-                    const int half = part & 1;      // which 32 values of u
-                    const bool scaled = part >= 2;  // U diag f
-                    uint32_t hi[16], lo[16];
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int s0 = 32 * half + 2 * q;
-                        const float x0 = scaled ? u[s0] * gs.f[s0] : u[s0];
-                        const float x1 = scaled ? u[s0 + 1] * gs.f[s0 + 1] : u[s0 + 1];
-                        float h0f, l0f, h1f, l1f;
-                        split_bf16(x0, h0f, l0f);
-                        split_bf16(x1, h1f, l1f);
-                        hi[q] = pack_bf16(h0f, h1f);
-                        lo[q] = pack_bf16(l0f, l1f);
-                    }
-                    const uint32_t base = scaled ? TM_UF : TM_U;
-                    tmem_st16u(taddr(tmem, lane_base, base + 16 * half), hi);
-                    tmem_st16u(taddr(tmem, lane_base, base + 32 + 16 * half), lo);
-                }
+                tmem_st16u(taddr(tmem, lane_base, TM_U + 32 * half), hi);
+                tmem_st16u(taddr(tmem, lane_base, TM_U + 32 * half + 16), lo);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -720,26 +698,34 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc_fence_before();
                 mbar_arrive(&bars[B_HM_READY]);
             }
-            // ---- output o_r = scale (2^G_r O1_r + O2_r)
+        }
+    } else if (warp >= 16) {
+        // ================================================================ output warpgroup
+        // o_r = scale (2^G_r O1_r + O2_r), read from TMEM 8 rows at a time
+        const int j = tid & 127;  // value column (TMEM lane)
+        const uint32_t lane_base = 32 * (warp & 3);
+        for (int c = 0; c < nc; ++c) {
+            const TcGate& gs = gates[c & 3];
+            if (!warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err)) break;
             if (!warp_wait(&bars[B_O_FULL], c & 1, abort_flag, err)) break;
             tc_fence_after();
             const int Lc = gs.L;
             const size_t tok0 = (size_t)row * T + bos + (size_t)c * kChunk;
             const size_t ostride = (size_t)H * dv;
             size_t off = (tok0 * H + h) * (size_t)dv + j0 + j;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float v1[32], v2[32];
-                tmem_ld32(taddr(tmem, lane_base, TM_O1 + 32 * half), v1);
-                tmem_ld32(taddr(tmem, lane_base, TM_O2 + 32 * half), v2);
+#pragma unroll 1
+            for (int r8 = 0; r8 < 64; r8 += 8) {
+                float v1[8], v2[8];
+                tmem_ld8(taddr(tmem, lane_base, TM_O1 + r8), v1);
+                tmem_ld8(taddr(tmem, lane_base, TM_O2 + r8), v2);
                 tmem_wait_ld();
-                if (half == 1) {
+                if (r8 == 56) {
                     tc_fence_before();
                     mbar_arrive(&bars[B_O_FREE]);
                 }
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int r = 32 * half + q;
+                for (int q = 0; q < 8; ++q) {
+                    const int r = r8 + q;
                     if (r < Lc) {
                         const float val = p.scale * fmaf(gs.eG[r], v1[q], v2[q]);
                         if (O_F32) static_cast<float*>(p.o)[off] = val;
