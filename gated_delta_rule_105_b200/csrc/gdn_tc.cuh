@@ -21,10 +21,12 @@
 // (GatedDeltaNet data-flow walkthrough, yfxerp.com/news/367755, section "Chunked parallelism").
 //
 // Warp roles (20 warps): 0 TMA producer and gate prep; 1 issues the h-independent MMAs (S1, W^T) one chunk
-// ahead; 2 issues the serial MMAs (U^T, O^T, h^T); 3 idle; 4-7 and 8-11 (two prep warpgroups, one per half
-// of the 64 chunk columns) build A, P, T', T'' and -W^T, the first of them also (I+A)^-1; 12-15 (state
-// warpgroup) split U into bf16 operands, refresh the bf16 copy of h^T, re-scale the fp32 state by the next
-// chunk's decay and write hT; 16-19 (output warpgroup) write o.
+// ahead; 2 issues the serial MMAs (U^T, O^T, h^T); 3 stores the output tiles by TMA; 4-7 and 8-11 (two prep
+// warpgroups) build A, P, (I+A)^-1, T', T'' and -W^T; 12-15 and 16-19 (state warpgroups, one per half of U,
+// of the key channels and of the chunk's rows) split U into bf16 operands, refresh the bf16 copy of h^T,
+// re-scale the fp32 state by the next chunk's decay, write hT and stage o.
+// The operands T', T'' and P are lower triangular: the MMAs that read them skip the blocks above the
+// diagonal (k-step ks of 16 tokens only reaches the output columns r >= 16 ks).
 // All mbarrier waits are bounded: on time-out the CTA sets the error word and drains to the exit.
 #pragma once
 
@@ -83,18 +85,19 @@ enum TcBar : int {
     B_GATE = 6,       // [4] gate stage written
     B_S1_FULL = 10,   // S1 in TMEM
     B_S1_FREE = 11,   // prep read S1 (256 arrivals)
-    B_TP_READY = 12,  // T' written (256)
+    B_TP_READY = 12,  // T' written (128)
     B_W_FULL = 13,    // W^T in TMEM
     B_PREP = 14,      // [2] T'', -W^T, P ready for the serial step (256)
-    B_P_FREE = 16,    // [2] O^T MMA reading P done
+    B_P_FREE = 16,    // [2] P, T'' stage free: O^T MMA done and the output staged there stored
     B_U_FULL = 18,    // U^T in TMEM (and -W^T, T'' no longer read)
-    B_U_CONV = 19,    // U, U.f split into bf16 hi/lo in TMEM (128)
+    B_U_CONV = 19,    // U, U.f split into bf16 hi/lo in TMEM (256)
     B_H_FULL = 20,    // h^T MMA done
-    B_H_READY = 21,   // bf16 h^T staged in shared memory (128)
+    B_H_READY = 21,   // bf16 h^T staged in shared memory (256)
     B_O_FULL = 22,    // O^T MMAs done
-    B_O_FREE = 23,    // O^T TMEM read (128)
+    B_O_FREE = 23,    // O^T TMEM read (256)
     B_DRAIN = 24,     // [2] final commit of each MMA issuer
-    B_HM_READY = 26,  // fp32 state in TMEM re-scaled by the next chunk's decay (128)
+    B_HM_READY = 26,  // fp32 state in TMEM re-scaled by the next chunk's decay (256)
+    B_O_STAGED = 27,  // output tile staged in shared memory (256)
 };
 
 // TMEM columns.  U^T is accumulated in fp32 at TM_U; the state warpgroup then writes U as bf16 hi/lo pairs
@@ -166,14 +169,48 @@ __device__ __forceinline__ void store16(float* S, int r0, int c0, bool tr, int l
     }
 }
 
+// Where the blocks of T go once final: T' = T diag(beta 2^G) as bf16, and T'' = T diag(beta) as a bf16 hi + lo
+// pair, each [r][s] K-major with 128-byte swizzle.  Only the blocks on and below the diagonal are written;
+// the MMAs that read these operands skip the zero blocks above it.
+struct TEmit {
+    uint8_t* tp;
+    uint8_t* tpp;
+    uint8_t* tppl;
+    const float* beta;
+    const float* eG;
+};
+// Emits sgn * acc, the final 16x16 block (r0, c0) of T held as an mma.sync accumulator.
+__device__ __forceinline__ void emit16(const TEmit& em, int r0, int c0, int lane, const float (&acc)[2][4], float sgn) {
+    using namespace sm100;
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        const int s = c0 + 8 * nh + 2 * t;
+        const float b0 = sgn * em.beta[s], b1 = sgn * em.beta[s + 1];
+        const float e0 = em.eG[s], e1 = em.eG[s + 1];
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const float x0 = acc[nh][2 * hr] * b0, x1 = acc[nh][2 * hr + 1] * b1;
+            const uint32_t off = sw128(r0 + g + 8 * hr, s >> 3) + (s & 7) * 2;
+            uint32_t hi, lo;
+            split_pack_bf16(x0, x1, hi, lo);
+            *reinterpret_cast<uint32_t*>(em.tp + off) = pack_bf16(x0 * e0, x1 * e1);
+            *reinterpret_cast<uint32_t*>(em.tpp + off) = hi;
+            *reinterpret_cast<uint32_t*>(em.tppl + off) = lo;
+        }
+    }
+}
+
 // (I + A)^-1 for a strictly lower-triangular 64x64 A in the [64][68] fp32 scratch (upper triangle 0), by
-// the 4 warps of one warpgroup.  On return the diagonal 16x16 blocks hold T_ii in place, each
-// off-diagonal block T_ij (i > j) is stored transposed in the upper-triangle block (j, i), and the lower
-// off-diagonal blocks of A are left intact.  Steps: the four diagonal blocks by forward substitution (one
-// column per lane); T_10 = -T_11 A_10 T_00 and T_32 = -T_33 A_32 T_22; then the lower-left 32x32 quarter
-// T_c = -T_b (A_c T_a), where T_a, T_b are the inverses of the two diagonal 32x32 quarters -- each block
-// product on tf32 MMAs, at most two per warp per step.
-__device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane, uint32_t bar_id) {
+// the 4 warps of one warpgroup; every block of T = (I + A)^-1 is emitted (TEmit) as soon as it is final.
+// Steps: the four diagonal 16x16 blocks by forward substitution (one column per lane), left in place for
+// the later steps; T_10 = -T_11 A_10 T_00 and T_32 = -T_33 A_32 T_22, stored transposed in the upper
+// blocks (0, 1) and (2, 3); then the lower-left 32x32 quarter T_c = -T_b (A_c T_a), where T_a, T_b are
+// the inverses of the two diagonal 32x32 quarters, with A_c T_a parked transposed in the upper blocks
+// (q, p).  Each block product runs on tf32 MMAs, at most two per warp per step.  The lower off-diagonal
+// blocks of A are left intact.  The code is unrolled: it is one chain of dependent shared-memory loads and
+// MMAs, which only unrolling lets the compiler overlap.
+__device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane, uint32_t bar_id, const TEmit& em) {
     using namespace sm100;
     {
         const int b0 = 16 * wid, c = lane & 15;
@@ -189,6 +226,18 @@ __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane,
         if (lane < 16) {
 #pragma unroll
             for (int r = 0; r < 16; ++r) S[(b0 + r) * TcSmem::AS_LD + b0 + c] = t[r];
+        }
+        // emit column c of T_ii: lanes 0-15 rows 0-7, lanes 16-31 rows 8-15
+        const int s = b0 + c, hr = lane >> 4;
+        const float bs = em.beta[s], es = em.eG[s];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            const float x = (hr ? t[8 + rr] : t[rr]) * bs;
+            const uint32_t off = sw128(b0 + 8 * hr + rr, s >> 3) + (s & 7) * 2;
+            const __nv_bfloat16 xh = __float2bfloat16_rn(x);
+            *reinterpret_cast<__nv_bfloat16*>(em.tp + off) = __float2bfloat16_rn(x * es);
+            *reinterpret_cast<__nv_bfloat16*>(em.tpp + off) = xh;
+            *reinterpret_cast<__nv_bfloat16*>(em.tppl + off) = __float2bfloat16_rn(x - __bfloat162float(xh));
         }
     }
     named_bar_sync(bar_id, 128);
@@ -206,6 +255,7 @@ __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane,
         mma16(y, f, S, 16 * i, 16 * j, true, lane);
         __syncwarp();
         store16(S, 16 * i, 16 * j, true, lane, y, -1.f);
+        emit16(em, 16 * i, 16 * j, lane, y, -1.f);
     }
     named_bar_sync(bar_id, 128);
     // X = A_c T_a for the blocks (p, q), p in {2, 3}, q in {0, 1}; one block per warp, parked in (p, q)
@@ -222,7 +272,7 @@ __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane,
         store16(S, 16 * p, 16 * q, true, lane, x, 1.f);
     }
     named_bar_sync(bar_id, 128);
-    // T_c = -T_b X: T_2q = -T_22 X_2q ; T_3q = -(T_32 X_2q + T_33 X_3q)
+    // T_c = -T_b X: T_2q = -T_22 X_2q ; T_3q = -(T_32 X_2q + T_33 X_3q); emitted only (not needed in S)
     {
         Frag16 f;
         float y[2][4] = {};
@@ -235,22 +285,16 @@ __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane,
             load_a16(S, 48, 48, false, lane, f);
             mma16(y, f, S, 48, 16 * q, true, lane);
         }
-        named_bar_sync(bar_id, 128);  // every X block has been read
-        store16(S, 16 * p, 16 * q, true, lane, y, -1.f);
+        emit16(em, 16 * p, 16 * q, lane, y, -1.f);
     }
-    named_bar_sync(bar_id, 128);
-}
-// Element (r, s) of T = (I + A)^-1 as left by invert_unit_lower64.
-__device__ __forceinline__ float t_elem(const float* S, int r, int s) {
-    if (s > r) return 0.f;
-    return ((r >> 4) == (s >> 4)) ? S[r * TcSmem::AS_LD + s] : S[s * TcSmem::AS_LD + r];
 }
 
 // ------------------------------------------------------------------------------------------ the kernel
 template <bool O_F32>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p, unsigned* err) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const FwdParams p,
+                  unsigned* err) {
     using namespace sm100;
     using L = TcSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -306,10 +350,10 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     if (tid == 0) {
         for (int b = 0; b < (int)L::N_BARS; ++b) {
-            const uint32_t cnt =
-                (b == B_S1_FREE || b == B_TP_READY || b == B_PREP || b == B_PREP + 1)
-                    ? 256u
-                    : ((b == B_U_CONV || b == B_O_FREE || b == B_H_READY || b == B_HM_READY) ? 128u : 1u);
+            const uint32_t cnt = (b == B_S1_FREE || b == B_PREP || b == B_PREP + 1 || b == B_U_CONV ||
+                                  b == B_H_READY || b == B_HM_READY || b == B_O_FREE || b == B_O_STAGED)
+                                     ? 256u
+                                     : (b == B_TP_READY ? 128u : 1u);
             mbar_init(&bars[b], cnt);
         }
         *abort_flag = 0;
@@ -317,6 +361,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_o);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, TM_COLS);
@@ -352,6 +397,18 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tma_load_3d(sm + L::V + 8192, &tm_v, &bars[B_V_FULL], j0 + 64, h, tok);
             }
             v_issued++;
+        };
+        // L2 prefetch of a later chunk's tiles, so that the load issued once a stage frees up hits L2
+        auto prefetch = [&](int c) {
+            if (lane == 0 && c < nc) {
+                const int tok = row * T + bos + c * kChunk;
+                tma_prefetch_3d(&tm_k, 0, h, tok);
+                tma_prefetch_3d(&tm_k, 64, h, tok);
+                tma_prefetch_3d(&tm_q, 0, h, tok);
+                tma_prefetch_3d(&tm_q, 64, h, tok);
+                tma_prefetch_3d(&tm_v, j0, h, tok);
+                tma_prefetch_3d(&tm_v, j0 + 64, h, tok);
+            }
         };
         auto make_gates = [&](int c) {
             TcGate& gs = gates[c & 3];
@@ -392,22 +449,17 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_GATE + (c & 3)]);
         };
-        load_kq(0);
-        make_gates(0);
-        if (nc > 1) {
-            load_kq(1);
-            make_gates(1);
-        }
-        load_v(0);
-        for (int c = 0; c < nc; ++c) {
-            if (c + 1 < nc) {
-                if (!warp_wait(&bars[B_V_EMPTY], c & 1, abort_flag, err)) break;
+        // iteration c loads V of chunk c + 1 and K/Q (+ gates) of chunk c + 2; the first two fill both stages
+        for (int c = -2; c < nc; ++c) {
+            if (c + 1 >= 0 && c + 1 < nc) {
+                if (c >= 0 && !warp_wait(&bars[B_V_EMPTY], c & 1, abort_flag, err)) break;
                 load_v(c + 1);
             }
             if (c + 2 < nc) {
-                if (!warp_wait(&bars[B_KQ_EMPTY + (c & 1)], (c >> 1) & 1, abort_flag, err)) break;
+                if (c >= 0 && !warp_wait(&bars[B_KQ_EMPTY + (c & 1)], (c >> 1) & 1, abort_flag, err)) break;
                 load_kq(c + 2);
                 make_gates(c + 2);
+                prefetch(c + 3);
             }
         }
         // drain: wait for every load this warp issued before the CTA may exit
@@ -416,28 +468,59 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (v_issued > 0) drain_wait(&bars[B_V_FULL], (v_issued - 1) & 1);
     } else if (warp == 1) {
         // ================================================================ h-independent MMAs (S1, W^T)
+        // Issued in readiness order.  S1 of chunk c + 1 needs its K/Q and the prep to have read S1 of chunk c,
+        // which it normally has before chunk c's T' is ready; W^T of chunk c needs T'.  While both are
+        // pending the thread sleeps on T' and checks the S1 conditions whenever it wakes.
         if (lane == 0) {
             const uint32_t id_s1 = idesc_bf16(128, 64, false, false);
             const uint32_t id_w = idesc_bf16(128, 64, true, false);
-            for (int c = 0; c < nc; ++c) {
-                const int st = c & 1;
-                const uint32_t kq = sbase + L::KQ + st * L::KQ_STAGE;
-                if (!mbar_wait(&bars[B_KQ_FULL + st], (c >> 1) & 1, abort_flag, err)) break;
-                if (c >= 1 && !mbar_wait(&bars[B_S1_FREE], (c - 1) & 1, abort_flag, err)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t a = kq + (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_bf16(tmem + TM_S1, desc_k_sw128(a), desc_k_sw128(a), id_s1, kk > 0);
+            const uint32_t n16 = 2u << 17;  // N += 16 in an instruction descriptor (N / 8 at bit 17)
+            int ns = 0, nw = 0;  // next chunk for S1, for W^T
+            long long last = clock64();
+            auto s1_ready = [&]() {
+                return mbar_test(&bars[B_KQ_FULL + (ns & 1)], (ns >> 1) & 1) &&
+                       (ns == 0 || mbar_test(&bars[B_S1_FREE], (ns - 1) & 1));
+            };
+            while (nw < nc) {
+                bool did = false;
+                // S1 may run ahead of W^T by one chunk; W^T(nw) needs S1(nw) first
+                const bool s1_due = ns < nc && ns <= nw + 1;
+                if (s1_due && s1_ready()) {
+                    tc_fence_after();
+                    const uint64_t d = desc_k_sw128(sbase + L::KQ + (ns & 1) * L::KQ_STAGE);
+#pragma unroll 1
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t a = d + (kk >> 2) * 1024 + (kk & 3) * 2;
+                        umma_bf16(tmem + TM_S1, a, a, id_s1, kk > 0);
+                    }
+                    umma_commit(&bars[B_S1_FULL]);
+                    ++ns;
+                    did = true;
+                } else if (nw < ns && mbar_try_wait_ns(&bars[B_TP_READY], nw & 1, s1_due ? 200u : kSuspendHintNs)) {
+                    tc_fence_after();
+                    const uint64_t da = desc_mn_sw128(sbase + L::KQ + (nw & 1) * L::KQ_STAGE, 16384);
+                    const uint64_t db = desc_k_sw128(sbase + L::TP);
+                    // k-step kk (tokens s in [16 kk, 16 kk + 16)) reaches only the rows r >= 16 kk of T'
+#pragma unroll 1
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + TM_W + 16 * kk, da + kk * 128, db + kk * 130, id_w - kk * n16, kk > 0);
+                    umma_commit(&bars[B_W_FULL]);
+                    ++nw;
+                    did = true;
+                } else if (nw == ns) {  // only S1 can make progress: sleep on its K/Q, then on S1_FREE
+                    mbar_try_wait(&bars[B_KQ_FULL + (ns & 1)], (ns >> 1) & 1);
+                    if (ns > 0) mbar_try_wait(&bars[B_S1_FREE], (ns - 1) & 1);
                 }
-                umma_commit(&bars[B_S1_FULL]);
-                if (!mbar_wait(&bars[B_TP_READY], c & 1, abort_flag, err)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem + TM_W, desc_mn_sw128(kq + kk * 2048, 16384),
-                              desc_k_sw128(sbase + L::TP + kk * 32), id_w, kk > 0);
-                umma_commit(&bars[B_W_FULL]);
+                if (did) {
+                    last = clock64();
+                } else {
+                    if (*abort_flag) break;
+                    if (clock64() - last > kWaitLimitCycles) {
+                        *abort_flag = 1;
+                        atomicOr(err, kErrTimeout);
+                        break;
+                    }
+                }
             }
             umma_commit(&bars[B_DRAIN]);
             drain_wait(&bars[B_DRAIN], 0);
@@ -445,153 +528,167 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         __syncwarp();
     } else if (warp == 2) {
         // ================================================================ serial MMAs (U^T, O^T, h^T)
+        // The k-step loops stay rolled (short code); descriptors advance by byte offset >> 4.
         if (lane == 0) {
             const uint32_t id_u1 = idesc_bf16(128, 64, true, false);
             const uint32_t id_u2 = idesc_bf16(128, 64, false, true);
             const uint32_t id_o = idesc_bf16(128, 64, false, false);
             const uint32_t id_h = idesc_bf16(128, 128, false, true);
+            const uint32_t n16 = 2u << 17;  // N += 16 in an instruction descriptor (N / 8 at bit 17)
+            const uint64_t d_v = desc_mn_sw128(sbase + L::V, 8192);
+            const uint64_t d_ht = desc_k_sw128(sbase + L::HT);
+            const uint64_t d_wt = desc_mn_sw128(sbase + L::WT, 8192);
             for (int c = 0; c < nc; ++c) {
                 const int st = c & 1;
                 const uint32_t kq = sbase + L::KQ + st * L::KQ_STAGE;
                 if (!mbar_wait(&bars[B_PREP + st], (c >> 1) & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[B_V_FULL], c & 1, abort_flag, err)) break;
                 tc_fence_after();
-                // U^T = V^T (T''_hi + T''_lo)^T - h^T W^T ; the first half does not need the state
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_bf16(tmem + TM_U, desc_mn_sw128(sbase + L::V + (kk & 3) * 2048, 8192),
-                              desc_k_sw128(sbase + (kk < 4 ? L::TPP : L::TPPL) + st * 8192 + (kk & 3) * 32), id_u1,
-                              kk > 0);
+                // U^T = V^T (T''_hi + T''_lo)^T - h^T W^T ; the first half does not need the state.  As T'' is
+                // lower triangular, k-step ks (tokens s in [16 ks, 16 ks + 16)) updates only columns r >= 16 ks.
+#pragma unroll 1
+                for (int kk = 0; kk < 8; ++kk) {
+                    const int ks = kk & 3;
+                    const uint64_t b = desc_k_sw128(sbase + (kk < 4 ? L::TPP : L::TPPL) + st * 8192) + ks * 130;
+                    umma_bf16(tmem + TM_U + 16 * ks, d_v + ks * 128, b, id_u1 - ks * n16, kk > 0);
+                }
                 if (!mbar_wait(&bars[B_H_READY], c & 1, abort_flag, err)) break;
                 tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_bf16(tmem + TM_U, desc_k_sw128(sbase + L::HT + (kk >> 2) * 16384 + (kk & 3) * 32),
-                              desc_mn_sw128(sbase + L::WT + kk * 2048, 8192), id_u2, 1);
+                    umma_bf16(tmem + TM_U, d_ht + (kk >> 2) * 1024 + (kk & 3) * 2, d_wt + kk * 128, id_u2, 1);
                 umma_commit(&bars[B_U_FULL]);
                 umma_commit(&bars[B_V_EMPTY]);
                 // O1^T = h^T Q^T (scaled by 2^G_r in the epilogue)
                 if (c >= 1 && !mbar_wait(&bars[B_O_FREE], (c - 1) & 1, abort_flag, err)) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_bf16(tmem + TM_O1, desc_k_sw128(sbase + L::HT + (kk >> 2) * 16384 + (kk & 3) * 32),
-                              desc_k_sw128(kq + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32), id_o, kk > 0);
+                const uint64_t d_q = desc_k_sw128(kq + 8192);
+#pragma unroll 1
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t o = (kk >> 2) * 1024 + (kk & 3) * 2;
+                    umma_bf16(tmem + TM_O1, d_ht + o, d_q + o, id_o, kk > 0);
+                }
                 // h^T += (U diag f)^T K  (hi and lo halves) ;  O2^T = U^T P^T  (hi*hi + hi*lo + lo*hi)
                 if (!mbar_wait(&bars[B_U_CONV], c & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[B_HM_READY], c & 1, abort_flag, err)) break;
                 tc_fence_after();
-#pragma unroll
+                const uint64_t d_k = desc_mn_sw128(kq, 16384);
+#pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk) {  // kk < 4: hi, else lo; s-step ks covers values 16 ks .. 16 ks + 15
                     const int ks = kk & 3;
                     const uint32_t a = tmem + TM_U + (ks >> 1) * 32 + (kk >> 2) * 16 + (ks & 1) * 8;
-                    umma_bf16_tmem_a(tmem + TM_H, a, desc_mn_sw128(kq + ks * 2048, 16384), id_h, 1);
+                    umma_bf16_tmem_a(tmem + TM_H, a, d_k + ks * 128, id_h, 1);
                 }
                 umma_commit(&bars[B_H_FULL]);
-#pragma unroll
-                for (int kk = 0; kk < 12; ++kk) {
+#pragma unroll 1
+                for (int kk = 0; kk < 12; ++kk) {  // P lower triangular: k-step ks reaches columns r >= 16 ks
                     const int part = kk >> 2, ks = kk & 3;  // 0: Uhi Phi, 1: Uhi Plo, 2: Ulo Phi
                     const uint32_t a = tmem + TM_UF + (part == 2 ? 32 : 0) + ks * 8;
-                    const uint32_t b = sbase + (part == 1 ? L::PL : L::PH) + st * 8192 + ks * 32;
-                    umma_bf16_tmem_a(tmem + TM_O2, a, desc_k_sw128(b), id_o, kk > 0);
+                    const uint64_t b = desc_k_sw128(sbase + (part == 1 ? L::PL : L::PH) + st * 8192) + ks * 130;
+                    umma_bf16_tmem_a(tmem + TM_O2 + 16 * ks, a, b, id_o - ks * n16, kk > 0);
                 }
                 umma_commit(&bars[B_O_FULL]);
                 umma_commit(&bars[B_KQ_EMPTY + st]);
-                umma_commit(&bars[B_P_FREE + st]);
             }
             umma_commit(&bars[B_DRAIN + 1]);
             drain_wait(&bars[B_DRAIN + 1], 0);
         }
         __syncwarp();
+    } else if (warp == 3) {
+        // ================================================================ output stores
+        // A full chunk's o tile is staged by the state warpgroups in the P and T'' buffers of its stage (free
+        // once its O^T MMAs are done) and leaves by TMA; a partial chunk is written directly by them.
+        if (lane == 0) {
+            for (int c = 0; c < nc; ++c) {
+                const int st = c & 1;
+                if (!mbar_wait(&bars[B_O_STAGED], c & 1, abort_flag, err)) break;
+                if (eos - bos - c * kChunk >= kChunk) {
+                    const int tok0 = row * T + bos + c * kChunk;
+                    const uint32_t rg[4] = {L::PH, L::PL, L::TPP, L::TPPL};
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) tma_store_3d(&tm_o, sm + rg[b] + st * 8192, j0, h, tok0 + 16 * b);
+                    bulk_commit();
+                    bulk_wait_read_all();
+                }
+                mbar_arrive(&bars[B_P_FREE + st]);
+            }
+            bulk_wait_all();
+        }
+        __syncwarp();
     } else if (warp >= 4 && warp < 12) {
         // ================================================================ prep warpgroups
-        // A timed-out wait does not break out here: the warpgroups finish the iteration (with whatever data)
-        // and leave together at the top of the next one, so no thread is left waiting at a named barrier.
-        const int wsel = (warp - 4) >> 2;      // 0: chunk columns 0-31, 1: columns 32-63
-        const int t = (tid - 128) & 127;       // row of S1 / line of W^T (TMEM lane)
+        // Per chunk: (1) A rows, split by column halves over the quadrant-0/1 warps of both warpgroups;
+        // (2) the first warpgroup inverts (I + A), writing T' (what the W^T MMA needs) and T'' as it goes,
+        // while the quadrant-2/3 warps of the second build P; (3) -W^T.  A timed-out wait does not break out
+        // here: the warpgroups finish the iteration and leave together at the top of the next.
+        const int wsel = (warp - 4) >> 2;      // warpgroup 0 or 1
+        const int t = (tid - 128) & 127;       // TMEM lane: row of S1 / line of W^T
         const int wid = warp & 3;
-        const int tp = tid - 128;              // 0..255 across both warpgroups
         for (int c = 0; c < nc; ++c) {
             if (named_bar_or(2, 256, *abort_flag != 0)) break;
             const int st = c & 1;
             warp_wait(&bars[B_S1_FULL], c & 1, abort_flag, err);
-            tc_fence_after();
             warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err);
+            tc_fence_after();
             const TcGate& gs = gates[c & 3];
-            if (t >= 64 && c >= 2) warp_wait(&bars[B_P_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err);
-            // Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1): a running product from the highest column of
-            // this half at or below r, started there with one exp2; 8 columns at a time, highest first
-            {
-                const int r = t & 63;
-                const int s_hi = 32 * wsel + 31;
+            // Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1): a running product down from the highest
+            // column at or below r of the columns handled, started there with one exp2; 8 columns at a time
+            auto row_pass = [&](int r, int s_lo, int s_hi, bool is_a) {
                 const int top = r < s_hi ? r : s_hi;
                 float run = (top == r) ? 1.f : ex2_approx(gs.G[r] - gs.G[top]);
-                const float br = (t < 64) ? gs.beta[r] : 1.f;
+                const float br = is_a ? gs.beta[r] : 1.f;
 #pragma unroll 1
-                for (int ch = 3; ch >= 0; --ch) {
+                for (int c8 = s_hi - 7; c8 >= s_lo; c8 -= 8) {
                     float s8[8];
-                    tmem_ld8(taddr(tmem, 32 * wid, TM_S1 + 32 * wsel + 8 * ch), s8);
+                    tmem_ld8(taddr(tmem, 32 * wid, TM_S1 + c8), s8);
                     tmem_wait_ld();
                     float x[8];
 #pragma unroll
                     for (int q = 7; q >= 0; --q) {
-                        const int s = 32 * wsel + 8 * ch + q;
-                        x[q] = (t < 64 ? (s < r) : (s <= r)) ? br * run * s8[q] : 0.f;
+                        const int s = c8 + q;
+                        x[q] = (is_a ? (s < r) : (s <= r)) ? br * run * s8[q] : 0.f;
                         if (s <= top && s > 0) run *= gs.a[s];
                     }
-                    if (t < 64) {  // A row r: beta_r Gamma_rs (k_r . k_s), s < r
-                        float* dst = &sA[r * L::AS_LD + 32 * wsel + 8 * ch];
+                    if (is_a) {  // A row r: beta_r Gamma_rs (k_r . k_s), s < r
+                        float* dst = &sA[r * L::AS_LD + c8];
                         *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
                         *reinterpret_cast<float4*>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
                     } else {  // P row r: Gamma_rs (q_r . k_s), s <= r, bf16 hi + lo
-                        float xh[8], xl[8];
+                        uint32_t hi[4], lo[4];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) split_bf16(x[q], xh[q], xl[q]);
-                        const uint32_t off = sw128(r, 4 * wsel + ch);
-                        *reinterpret_cast<uint4*>(sm + L::PH + st * 8192 + off) =
-                            make_uint4(pack_bf16(xh[0], xh[1]), pack_bf16(xh[2], xh[3]), pack_bf16(xh[4], xh[5]),
-                                       pack_bf16(xh[6], xh[7]));
-                        *reinterpret_cast<uint4*>(sm + L::PL + st * 8192 + off) =
-                            make_uint4(pack_bf16(xl[0], xl[1]), pack_bf16(xl[2], xl[3]), pack_bf16(xl[4], xl[5]),
-                                       pack_bf16(xl[6], xl[7]));
+                        for (int q = 0; q < 4; ++q) split_pack_bf16(x[2 * q], x[2 * q + 1], hi[q], lo[q]);
+                        const uint32_t off = sw128(r, c8 >> 3);
+                        *reinterpret_cast<uint4*>(sm + L::PH + st * 8192 + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<uint4*>(sm + L::PL + st * 8192 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                     }
                 }
+            };
+            // (1) A rows (lanes 0-63), columns [32 wsel, 32 wsel + 32); S1 is then read only by the P rows
+            if (wid < 2) row_pass(t, 32 * wsel, 32 * wsel + 31, true);
+            if (wsel == 0 || wid < 2) {
+                tc_fence_before();
+                mbar_arrive(&bars[B_S1_FREE]);
             }
-            tc_fence_before();
-            mbar_arrive(&bars[B_S1_FREE]);
             named_bar_sync(1, 256);
-            if (wsel == 0) invert_unit_lower64(sA, wid, lane, 3);
-            named_bar_sync(1, 256);
-            {  // T' = T diag(beta 2^G) (bf16) and T'' = T diag(beta) (bf16 hi + lo), [r][s] K-major
-                const int r = tp >> 2, qd = tp & 3;  // 16 columns [16 qd, 16 qd + 16) of row r
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    float x1[8], xh[8], xl[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int s = 16 * qd + 8 * ch + q;
-                        const float tb = t_elem(sA, r, s) * gs.beta[s];
-                        x1[q] = tb * gs.eG[s];
-                        split_bf16(tb, xh[q], xl[q]);
-                    }
-                    const uint32_t off = sw128(r, 2 * qd + ch);
-                    *reinterpret_cast<uint4*>(sm + L::TP + off) =
-                        make_uint4(pack_bf16(x1[0], x1[1]), pack_bf16(x1[2], x1[3]), pack_bf16(x1[4], x1[5]),
-                                   pack_bf16(x1[6], x1[7]));
-                    *reinterpret_cast<uint4*>(sm + L::TPP + st * 8192 + off) =
-                        make_uint4(pack_bf16(xh[0], xh[1]), pack_bf16(xh[2], xh[3]), pack_bf16(xh[4], xh[5]),
-                                   pack_bf16(xh[6], xh[7]));
-                    *reinterpret_cast<uint4*>(sm + L::TPPL + st * 8192 + off) =
-                        make_uint4(pack_bf16(xl[0], xl[1]), pack_bf16(xl[2], xl[3]), pack_bf16(xl[4], xl[5]),
-                                   pack_bf16(xl[6], xl[7]));
-                }
+            // (2) the inverse (first warpgroup), emitting T' and T''; P rows (lanes 64-127 of the second).
+            // T'' and P of chunk c go into the stage buffers of chunk c - 2, free once its output has left.
+            if (c >= 2 && (wsel == 0 || wid >= 2))
+                warp_wait(&bars[B_P_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err);
+            if (wsel == 0) {
+                const TEmit em{sm + L::TP, sm + L::TPP + st * 8192, sm + L::TPPL + st * 8192, gs.beta, gs.eG};
+                invert_unit_lower64(sA, wid, lane, 3, em);
+                fence_proxy_async();
+                mbar_arrive(&bars[B_TP_READY]);
+            } else if (wid >= 2) {
+                row_pass(t - 64, 0, 63, false);
+                tc_fence_before();
+                mbar_arrive(&bars[B_S1_FREE]);
             }
-            fence_proxy_async();
-            mbar_arrive(&bars[B_TP_READY]);
+            // (3) -W^T line i = t, columns r of this warpgroup's half
             warp_wait(&bars[B_W_FULL], c & 1, abort_flag, err);
             if (c >= 1) warp_wait(&bars[B_U_FULL], (c - 1) & 1, abort_flag, err);
             tc_fence_after();
-            {  // -W^T line i = t, columns r of this half
+            {
                 float v[32];
                 tmem_ld32(taddr(tmem, 32 * wid, TM_W + 32 * wsel), v);
                 tmem_wait_ld();
@@ -601,15 +698,19 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_before();
             mbar_arrive(&bars[B_PREP + st]);
         }
-    } else if (warp >= 12 && warp < 16) {
-        // ================================================================ state warpgroup
+    } else if (warp >= 12) {
+        // ================================================================ state / output warpgroups
+        // Warpgroups 12-15 (half 0) and 16-19 (half 1) share the serial-chain work: each splits half of U
+        // into bf16 operands, refreshes half of the state (key channels [64 half, 64 half + 64)) and then
+        // stages half of the chunk's output rows for the TMA store.
+        const int half = (warp - 12) >> 2;
         const int j = tid & 127;  // value column (TMEM lane)
         const uint32_t lane_base = 32 * (warp & 3);
         // initial state: bf16 copy and fp32 master pre-scaled by the first chunk's decay
         if (warp_wait(&bars[B_GATE + 0], 0, abort_flag, err)) {
             const float g0 = gates[0].gamma;
 #pragma unroll 1
-            for (int piece = 0; piece < 4; ++piece) {
+            for (int piece = 2 * half; piece < 2 * half + 2; ++piece) {
                 float v[32];
                 const float* hp = p.h0 ? p.h0 + state_base + (size_t)(32 * piece) * dv + j : nullptr;
 #pragma unroll
@@ -630,15 +731,13 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         for (int c = 0; c < nc; ++c) {
             const TcGate& gs = gates[c & 3];
-            // ---- U: fp32 accumulator -> bf16 hi/lo pairs for U and U diag f
+            // ---- U (values [32 half, 32 half + 32)): fp32 accumulator -> bf16 hi/lo pairs.
+            // U (for O2) goes to TM_UF (hi of values 0-63 in columns 0-31, lo in 32-63); U diag f (for h^T)
+            // in place over its own fp32 columns of TM_U as [hi | lo], 16 columns each.
             if (!warp_wait(&bars[B_U_FULL], c & 1, abort_flag, err)) break;
             if (!warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err)) break;
             tc_fence_after();
-            // U (for O2) as bf16 hi/lo pairs in TM_UF: hi of values 0-63 in columns 0-31, lo in 32-63.
-            // U diag f (for h^T) in place in TM_U, per 32 values: [hi 0-31 | lo 0-31 | hi 32-63 | lo 32-63],
-            // 16 columns each -- every column is read (as fp32) before it is overwritten.
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
+            {
                 float u[32];
                 tmem_ld32(taddr(tmem, lane_base, TM_U + 32 * half), u);
                 tmem_wait_ld();
@@ -658,7 +757,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[B_U_CONV]);
-            // ---- state refresh: bf16 copy for the next chunk's MMAs, fp32 master times the next decay
+            // ---- state refresh (key channels of this half)
             if (!warp_wait(&bars[B_H_FULL], c & 1, abort_flag, err)) break;
             const bool last = c + 1 == nc;
             if (!last && !warp_wait(&bars[B_GATE + ((c + 1) & 3)], ((c + 1) >> 2) & 1, abort_flag, err)) break;
@@ -666,7 +765,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const float gn = last ? 1.f : gates[(c + 1) & 3].gamma;
             // pass 1: the bf16 copy (what the next chunk's first MMAs wait for), or hT after the last chunk
 #pragma unroll 1
-            for (int piece = 0; piece < 4; ++piece) {
+            for (int piece = 2 * half; piece < 2 * half + 2; ++piece) {
                 float v[32];
                 tmem_ld32(taddr(tmem, lane_base, TM_H + 32 * piece), v);
                 tmem_wait_ld();
@@ -686,7 +785,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mbar_arrive(&bars[B_H_READY]);
                 // pass 2: the fp32 master times the next chunk's decay (needed only by the next h^T MMA)
 #pragma unroll 1
-                for (int piece = 0; piece < 4; ++piece) {
+                for (int piece = 2 * half; piece < 2 * half + 2; ++piece) {
                     float v[32];
                     tmem_ld32(taddr(tmem, lane_base, TM_H + 32 * piece), v);
                     tmem_wait_ld();
@@ -698,42 +797,42 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc_fence_before();
                 mbar_arrive(&bars[B_HM_READY]);
             }
-        }
-    } else if (warp >= 16) {
-        // ================================================================ output warpgroup
-        // o_r = scale (2^G_r O1_r + O2_r), read from TMEM 8 rows at a time
-        const int j = tid & 127;  // value column (TMEM lane)
-        const uint32_t lane_base = 32 * (warp & 3);
-        for (int c = 0; c < nc; ++c) {
-            const TcGate& gs = gates[c & 3];
-            if (!warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err)) break;
+            // ---- output rows [32 half, 32 half + 32): o_r = scale (2^G_r O1_r + O2_r), 8 rows at a time
             if (!warp_wait(&bars[B_O_FULL], c & 1, abort_flag, err)) break;
             tc_fence_after();
             const int Lc = gs.L;
+            const int st = c & 1;
             const size_t tok0 = (size_t)row * T + bos + (size_t)c * kChunk;
             const size_t ostride = (size_t)H * dv;
-            size_t off = (tok0 * H + h) * (size_t)dv + j0 + j;
+            size_t off = ((tok0 + 32 * half) * H + h) * (size_t)dv + j0 + j;
+            const uint32_t rg0 = half ? L::TPP : L::PH, rg1 = half ? L::TPPL : L::PL;
 #pragma unroll 1
-            for (int r8 = 0; r8 < 64; r8 += 8) {
+            for (int r8 = 32 * half; r8 < 32 * half + 32; r8 += 8) {
                 float v1[8], v2[8];
                 tmem_ld8(taddr(tmem, lane_base, TM_O1 + r8), v1);
                 tmem_ld8(taddr(tmem, lane_base, TM_O2 + r8), v2);
                 tmem_wait_ld();
-                if (r8 == 56) {
+                if (r8 == 32 * half + 24) {
                     tc_fence_before();
                     mbar_arrive(&bars[B_O_FREE]);
                 }
+                uint8_t* stg = sm + ((r8 & 16) ? rg1 : rg0) + st * 8192;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const int r = r8 + q;
-                    if (r < Lc) {
-                        const float val = p.scale * fmaf(gs.eG[r], v1[q], v2[q]);
+                    const float val = p.scale * fmaf(gs.eG[r], v1[q], v2[q]);
+                    if (Lc == kChunk) {  // staged for the TMA store: row r & 15 of a [16][128] box
+                        if (O_F32) reinterpret_cast<float*>(stg)[(r & 15) * kTcDV + j] = val;
+                        else reinterpret_cast<__nv_bfloat16*>(stg)[(r & 15) * kTcDV + j] = __float2bfloat16_rn(val);
+                    } else if (r < Lc) {
                         if (O_F32) static_cast<float*>(p.o)[off] = val;
                         else static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(val);
                     }
                     off += ostride;
                 }
             }
+            fence_proxy_async();
+            mbar_arrive(&bars[B_O_STAGED]);
         }
     }
     tc_fence_before();
@@ -781,15 +880,30 @@ inline bool make_map(CUtensorMap* map, const void* base, int d, int H, long long
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over the [rows, H, dv] output (fp32 or bf16), box 128 x 1 x 16 (one CTA's columns, 16 tokens),
+// no swizzle: the store source is a row-major [16][128] tile.
+inline bool make_out_map(CUtensorMap* map, void* base, int dv, int H, long long rows, bool f32) {
+    PFN_encodeTiled enc = get_encode_fn();
+    if (!enc) return false;
+    const cuuint64_t es = f32 ? 4 : 2;
+    const cuuint64_t dims[3] = {(cuuint64_t)dv, (cuuint64_t)H, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)dv * es, (cuuint64_t)dv * H * es};
+    const cuuint32_t box[3] = {(cuuint32_t)kTcDV, 1, 16};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, unsigned* err, cudaStream_t stream) {
     if (gdn2) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "GDN-2 has no tcgen05 kernel yet");
         return GDN_ERR_UNSUPPORTED;
     }
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     const long long rows = (long long)p.B * p.T;
     if (!make_map(&mq, p.q, p.dk, p.H, rows) || !make_map(&mk, p.k, p.dk, p.H, rows) ||
-        !make_map(&mv, p.v, p.dv, p.H, rows)) {
+        !make_map(&mv, p.v, p.dv, p.H, rows) || !make_out_map(&mo, p.o, p.dv, p.H, rows, o_f32)) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "cuTensorMapEncodeTiled failed");
         return GDN_ERR_CUDA;
     }
@@ -800,7 +914,7 @@ inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, unsigned*
         return GDN_ERR_CUDA;
     }
     const unsigned grid = (unsigned)(p.dv / kTcDV) * p.H * p.n_seq;
-    kern<<<grid, kTcThreads, TcSmem::ALLOC, stream>>>(mq, mk, mv, p, err);
+    kern<<<grid, kTcThreads, TcSmem::ALLOC, stream>>>(mq, mk, mv, mo, p, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "%s", cudaGetErrorString(e));
