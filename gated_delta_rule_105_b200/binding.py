@@ -140,13 +140,30 @@ def _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype):
     return B, T, H, dk, dv, n_seq, o, hT
 
 
+def workspace_bytes(B, T, H, dk, dv, BT=64, n_seqs=0) -> int:
+    """Device workspace (bytes) a call with these sizes can use: the tensor-core path of bf16 inputs keeps the
+    WY factors of every chunk there; 0 when no path needs any."""
+    return int(load_library().gdn_workspace_bytes(B, T, H, dk, dv, BT, n_seqs))
+
+
+def _workspace(q, B, T, H, dk, dv, BT, n_seqs, workspace):
+    if workspace is not None:
+        _check_dev("workspace", workspace, torch.uint8)
+        return workspace
+    if q.dtype != torch.bfloat16:
+        return None
+    nbytes = workspace_bytes(B, T, H, dk, dv, BT, n_seqs)
+    return torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes > 0 else None
+
+
 def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, output_final_state=True, cu_seqlens=None, BT=64,
-                  o=None, hT=None, o_dtype=None):
+                  o=None, hT=None, o_dtype=None, workspace=None):
     """Chunked gated delta rule forward through ``gdn_chunk_fwd`` of the C ABI.
 
     q, k [B,T,H,dk] and v [B,T,H,dv] (fp32 or bf16), g, beta [B,T,H] fp32, h0 [N,H,dk,dv] fp32 or None,
     cu_seqlens int32 [N+1] (B == 1) or None.  Returns (o [B,T,H,dv], hT [N,H,dk,dv] fp32); o is in
-    ``o_dtype`` (float32, or q's dtype -- the default).
+    ``o_dtype`` (float32, or q's dtype -- the default).  ``workspace`` (uint8 on the device, at least
+    :func:`workspace_bytes`) is allocated per call when not given.
     """
     B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype)
     _check_dev("g", g, torch.float32)
@@ -155,10 +172,12 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, output_final_state=True
         raise ValueError("g and beta must be [B,T,H]")
     scale = dk ** -0.5 if scale is None else float(scale)
     stream = torch.cuda.current_stream(q.device).cuda_stream
+    n_seqs = 0 if cu_seqlens is None else n_seq
+    ws = _workspace(q, B, T, H, dk, dv, BT, n_seqs, workspace)
     st = load_library().gdn_chunk_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(o), _ptr(hT),
         B, T, H, dk, dv, BT, _dtype_code(q), _dtype_code(o), _ptr(cu_seqlens),
-        0 if cu_seqlens is None else n_seq, None, 0, ctypes.c_void_p(stream))
+        n_seqs, _ptr(ws), 0 if ws is None else ws.numel(), ctypes.c_void_p(stream))
     _raise_on(st)
     return o, hT
 

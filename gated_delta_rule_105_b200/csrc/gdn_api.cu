@@ -105,7 +105,8 @@ static gdn_status launch_simt(const FwdParams& p, gdn_dtype dt, gdn_dtype o_dt, 
     return launch_simt_io<__nv_bfloat16, __nv_bfloat16, GDN2>(p, err, stream);
 }
 
-static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, gdn_dtype o_dt, cudaStream_t stream) {
+static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, gdn_dtype o_dt, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
     const int choice = g_kernel_choice.load();
     const bool tc_ok = dt == GDN_BF16 && tc_supported(p, gdn2, o_dt == GDN_F32);
     if (choice == GDN_KERNEL_TC && !tc_ok)
@@ -116,7 +117,7 @@ static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, gdn_dtype o_d
     if (p.n_seq == 0 || p.H == 0) return GDN_OK;
     const bool use_tc = tc_ok && choice != GDN_KERNEL_SIMT;
     if (use_tc) {
-        st = launch_tc(p, gdn2, o_dt == GDN_F32, err, stream);
+        st = launch_tc(p, gdn2, o_dt == GDN_F32, ws, ws_bytes, err, stream);
         if (st == GDN_OK) {
             t_last_kernel = GDN_KERNEL_TC;
             return st;
@@ -136,7 +137,12 @@ using namespace gdn;
 
 extern "C" {
 
-size_t gdn_workspace_bytes(int, int, int, int, int, int, int) { return 0; }
+size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs) {
+    // the tcgen05 path (bf16 inputs) keeps T' and T'' of every chunk and head; the SIMT path needs nothing
+    if (B < 1 || T < 1 || H < 1 || BT != kChunk || dk != kTcDK || dv < kTcDV || dv % kTcDV != 0 || n_seqs < 0)
+        return 0;
+    return tc_workspace_bytes(B, T, H, n_seqs);
+}
 
 gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float scale, const float* h0, void* o, float* hT, int B, int T, int H, int dk, int dv,
@@ -147,7 +153,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
                                  o_dt, cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
     if (st != GDN_OK) return st;
     FwdParams p{q, k, v, g, beta, nullptr, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
-    return run(p, false, dt, o_dt, stream);
+    return run(p, false, dt, o_dt, workspace, ws_bytes, stream);
 }
 
 gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* b,
@@ -159,7 +165,7 @@ gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const flo
                                  cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
     if (st != GDN_OK) return st;
     FwdParams p{q, k, v, g, b, w, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
-    return run(p, true, dt, o_dt, stream);
+    return run(p, true, dt, o_dt, workspace, ws_bytes, stream);
 }
 
 gdn_status gdn_set_kernel(gdn_kernel kernel) {

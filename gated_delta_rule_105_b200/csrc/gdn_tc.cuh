@@ -1,30 +1,28 @@
-// tcgen05 (5th-generation tensor core) chunked forward kernel for the gated delta rule, bf16 inputs.
+// tcgen05 (5th-generation tensor core) chunked forward of the gated delta rule, bf16 inputs: two kernels.
 //
-// One CTA owns one (sequence n, head h, block of 128 value columns j) and walks the sequence's chunks of
-// C = 64 tokens.  Every contraction is an M = 128 tcgen05.mma with bf16 operands in 128B-swizzled shared
-// memory and an fp32 accumulator in tensor memory.  The state is kept transposed, h^T [j][i] (value column
-// j on the 128 TMEM lanes, key channel i on 128 columns), fp32 in TMEM for the whole sequence.
+// Per chunk of C = 64 tokens (r, s = token rows; G = chunk-local cumulative gate in base 2;
+// f_s = 2^(G_last - G_s)):
+//   A   = strict_lower(beta_r 2^(G_r - G_s) k_r . k_s) ;  T = (I + A)^-1
+//   T'  = T diag(beta 2^G) ;  T'' = T diag(beta)
+//   W   = T' K ;  U = T'' V - W h                  (the corrected values)
+//   P   = lower(2^(G_r - G_s) q_r . k_s)
+//   O   = scale (diag(2^G) Q h + P U)              (read-out)
+//   h  <- 2^(G_last) h + K^T diag(f) U
+// This is the WY form of the intra-chunk dependency with one state handed from chunk to chunk
+// (GatedDeltaNet data-flow walkthrough, yfxerp.com/news/367755, section "Chunked parallelism").
 //
-// Per chunk (r, s = token rows; G = chunk-local cumulative gate in base 2; f_s = 2^(G_last - G_s)):
-//   S1  = [K; Q] K^T                          (rows 0-63: K K^T, rows 64-127: Q K^T)
-//   A   = strict_lower(beta_r 2^(G_r - G_s) S1_K) ;  P = lower(2^(G_r - G_s) S1_Q)
-//   T   = (I + A)^-1 ; T' = T diag(beta 2^G) ; T'' = T diag(beta)
-//   W^T = K^T T'^T
-//   U^T = V^T T''^T - h^T W^T                 (= (T'' V - W h)^T, the corrected values)
-//   O^T = diag(2^G) applied to h^T Q^T, + U^T P^T   (read-out, scaled by `scale` on the way out)
-//   h^T <- 2^(G_last) h^T + (U diag f)^T K
+// The WY kernel (gdn_tc_wy_kernel) computes, for every (chunk, head) at once, A from K K^T, the inverse and
+// T', T'' (T'' as a bf16 hi + lo pair), and writes them to the workspace in the exact shared-memory form
+// the MMAs read (24 KB per chunk and head).  Nothing in it depends on the state, so it runs fully parallel.
+// The main kernel (gdn_tc_fwd_kernel) then walks each sequence's chunks: one CTA owns one (sequence n,
+// head h, block of 128 value columns j); the state is kept transposed, h^T [j][i] (value column j on the 128
+// TMEM lanes, key channel i on 128 columns), fp32 in TMEM for the whole sequence.  Every contraction is an
+// M = 128 tcgen05.mma with bf16 operands in 128B-swizzled shared memory (or U in TMEM) and an fp32
+// accumulator in TMEM.
 // Precision: every bf16 operand whose rounding would reach the output at the bf16-ulp level is avoided or
 // split.  U and U diag f are kept as bf16 hi + lo pairs (in TMEM, as the A operand), P and T'' likewise
 // (in shared memory); 2^G_r is applied to the fp32 accumulator of h^T Q^T instead of to Q.  The remaining
 // bf16 operands are h^T, W^T, T' and the inputs themselves.
-// This is the WY form of the intra-chunk dependency with one state handed from chunk to chunk
-// (GatedDeltaNet data-flow walkthrough, yfxerp.com/news/367755, section "Chunked parallelism").
-//
-// Warp roles (20 warps): 0 TMA producer and gate prep; 1 issues the h-independent MMAs (S1, W^T) one chunk
-// ahead; 2 issues the serial MMAs (U^T, O^T, h^T); 3 stores the output tiles by TMA; 4-7 and 8-11 (two prep
-// warpgroups) build A, P, (I+A)^-1, T', T'' and -W^T; 12-15 and 16-19 (state warpgroups, one per half of U,
-// of the key channels and of the chunk's rows) split U into bf16 operands, refresh the bf16 copy of h^T,
-// re-scale the fp32 state by the next chunk's decay, write hT and stage o.
 // The operands T', T'' and P are lower triangular: the MMAs that read them skip the blocks above the
 // diagonal (k-step ks of 16 tokens only reaches the output columns r >= 16 ks).
 // All mbarrier waits are bounded: on time-out the CTA sets the error word and drains to the exit.
@@ -36,12 +34,13 @@
 
 namespace gdn {
 
-constexpr int kTcThreads = 640;
+constexpr int kTcThreads = 512;  // main kernel: 16 warps
+constexpr int kWyThreads = 128;  // WY kernel: one warpgroup
+constexpr int kTcDV = 128;       // value columns per CTA
+constexpr int kTcDK = 128;       // key dimension handled by these kernels
+constexpr uint32_t kWyUnit = 24576;  // workspace bytes per (chunk, head): T' | T''_hi | T''_lo, 8 KB each
 
-constexpr int kTcDV = 128;  // value columns per CTA
-constexpr int kTcDK = 128;  // key dimension handled by this kernel
-
-struct TcGate {  // one chunk's gate data, written by the producer warp
+struct TcGate {  // one chunk's gate data
     float G[64];     // log2(e) * chunk-local cumulative g
     float beta[64];  // beta (0 past the end of the sequence)
     float f[64];     // 2^(G_last - G_s)
@@ -53,59 +52,91 @@ struct TcGate {  // one chunk's gate data, written by the producer warp
 };
 static_assert(sizeof(TcGate) % 16 == 0, "gate stage size");
 
-// Shared-memory map (bytes from a 1024-aligned base).
-struct TcSmem {
-    static constexpr uint32_t KQ = 0;  // 2 stages x [K ch0-63 | Q ch0-63 | K ch64-127 | Q ch64-127], 8 KB each
-    static constexpr uint32_t KQ_STAGE = 32768;
-    static constexpr uint32_t V = KQ + 2 * KQ_STAGE;  // V tile: j 0-63 | j 64-127, 8 KB each (MN-major A)
-    static constexpr uint32_t TPP = V + 16384;        // T'' hi [2]: [r][s] K-major, 8 KB each
-    static constexpr uint32_t TPPL = TPP + 16384;     // T'' lo [2]
-    static constexpr uint32_t TP = TPPL + 16384;      // T': [r][s] K-major, 8 KB
-    static constexpr uint32_t PH = TP + 8192;         // P hi [2]: [r][s] K-major, 8 KB each
-    static constexpr uint32_t PL = PH + 16384;        // P lo [2]
-    static constexpr uint32_t WT = PL + 16384;        // -W^T: lines i (128) x 64 r, MN-major B, 16 KB
-    static constexpr uint32_t HT = WT + 16384;        // h^T bf16: [j][i] K-major, panels i 0-63 | 64-127, 16 KB each
-    static constexpr uint32_t AS = HT + 32768;        // A, then (I+A)^-1, fp32 [64][68]
-    static constexpr uint32_t AS_LD = 68;
-    static constexpr uint32_t GATE = AS + 64 * AS_LD * 4;  // 4 x TcGate
-    static constexpr uint32_t BARS = GATE + 4 * sizeof(TcGate);
-    static constexpr uint32_t N_BARS = 32;
-    static constexpr uint32_t MISC = BARS + 8 * N_BARS;  // tmem base, abort flag
-    static constexpr uint32_t END = MISC + 64;
-    static constexpr uint32_t ALLOC = END + 1024;  // slack for the 1024-byte alignment of the base
-};
-static_assert(TcSmem::ALLOC <= 232448, "shared memory budget");
+// Workspace slot of chunk c of a sequence that starts at global token offset `start` (row * T + bos) and
+// is sequence number n: n + floor((start + 64 c) / 64).  Slots of different chunks never coincide, and
+// all are below ceil(B T / 64) + (number of sequences).
+__host__ __device__ inline long long wy_slot(int n, long long start, int c) { return n + (start >> 6) + c; }
+inline long long wy_slots(int B, int T, int n_seqs) {
+    return ((long long)B * T + kChunk - 1) / kChunk + (n_seqs > B ? n_seqs : B);
+}
 
-// Barrier indices.
-enum TcBar : int {
-    B_KQ_FULL = 0,    // [2] TMA K/Q landed (tx)
-    B_KQ_EMPTY = 2,   // [2] serial MMAs of the stage's chunk done
-    B_V_FULL = 4,     // V landed (tx)
-    B_V_EMPTY = 5,    // U^T MMA reading V done
-    B_GATE = 6,       // [4] gate stage written
-    B_S1_FULL = 10,   // S1 in TMEM
-    B_S1_FREE = 11,   // prep read S1 (256 arrivals)
-    B_TP_READY = 12,  // T' written (128)
-    B_W_FULL = 13,    // W^T in TMEM
-    B_PREP = 14,      // [2] T'', -W^T, P ready for the serial step (256)
-    B_P_FREE = 16,    // [2] P, T'' stage free: O^T MMA done and the output staged there stored
-    B_U_FULL = 18,    // U^T in TMEM (and -W^T, T'' no longer read)
-    B_U_CONV = 19,    // U, U.f split into bf16 hi/lo in TMEM (256)
-    B_H_FULL = 20,    // h^T MMA done
-    B_H_READY = 21,   // bf16 h^T staged in shared memory (256)
-    B_O_FULL = 22,    // O^T MMAs done
-    B_O_FREE = 23,    // O^T TMEM read (256)
-    B_DRAIN = 24,     // [2] final commit of each MMA issuer
-    B_HM_READY = 26,  // fp32 state in TMEM re-scaled by the next chunk's decay (256)
-    B_O_STAGED = 27,  // output tile staged in shared memory (256)
-};
+// One chunk's gates, by one warp (lane l: tokens 2l, 2l+1).  tok0 = global token index of row 0.
+__device__ __forceinline__ void tc_make_gates(TcGate& gs, const FwdParams& p, size_t tok0, int Lc, int h, int lane) {
+    using namespace sm100;
+    float gv[2], bv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int r = 2 * lane + u;
+        const size_t tok = (tok0 + r) * p.H + h;
+        gv[u] = r < Lc ? p.g[tok] : 0.f;
+        bv[u] = r < Lc ? p.beta[tok] : 0.f;
+    }
+    const float pair = gv[0] + gv[1];
+    float incl = pair;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    const float excl = incl - pair;
+    const float G0 = (excl + gv[0]) * kLog2e, G1 = incl * kLog2e;
+    const float Glast = __shfl_sync(0xffffffffu, G1, 31);
+    gs.G[2 * lane] = G0;
+    gs.G[2 * lane + 1] = G1;
+    gs.beta[2 * lane] = bv[0];
+    gs.beta[2 * lane + 1] = bv[1];
+    gs.f[2 * lane] = ex2_approx(Glast - G0);
+    gs.f[2 * lane + 1] = ex2_approx(Glast - G1);
+    gs.eG[2 * lane] = ex2_approx(G0);
+    gs.eG[2 * lane + 1] = ex2_approx(G1);
+    gs.a[2 * lane] = ex2_approx(gv[0] * kLog2e);
+    gs.a[2 * lane + 1] = ex2_approx(gv[1] * kLog2e);
+    if (lane == 0) {
+        gs.gamma = ex2_approx(Glast);
+        gs.L = Lc;
+    }
+}
 
-// TMEM columns.  U^T is accumulated in fp32 at TM_U; the state warpgroup then writes U as bf16 hi/lo pairs
-// (two values per column) to TM_UF and U diag f, also as hi/lo pairs, in place over TM_U.
-constexpr uint32_t TM_S1 = 0, TM_W = 64, TM_U = 128, TM_UF = 192, TM_O1 = 256, TM_O2 = 320, TM_H = 384,
-                   TM_COLS = 512;
+// One row r of A (IS_A: beta_r Gamma_rs (k_r . k_s), s < r, fp32 into `arow`) or of P (Gamma_rs (q_r . k_s),
+// s <= r, bf16 hi + lo into the 128B-swizzled `ph`, `pl`), columns [s_lo, s_hi], from the dot products in
+// TMEM (`ta` = this warp's lanes, column of s = 0).  Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1) is a
+// running product down from the highest column at or below r, started there with one exp2.
+template <bool IS_A>
+__device__ __forceinline__ void tc_row_pass(uint32_t ta, const TcGate& gs, int r, int s_lo, int s_hi, float* arow,
+                                            uint8_t* ph, uint8_t* pl) {
+    using namespace sm100;
+    const int top = r < s_hi ? r : s_hi;
+    float run = (top == r) ? 1.f : ex2_approx(gs.G[r] - gs.G[top]);
+    const float br = IS_A ? gs.beta[r] : 1.f;
+#pragma unroll 1
+    for (int c8 = s_hi - 7; c8 >= s_lo; c8 -= 8) {
+        float s8[8];
+        tmem_ld8(ta + c8, s8);
+        tmem_wait_ld();
+        float x[8];
+#pragma unroll
+        for (int q = 7; q >= 0; --q) {
+            const int s = c8 + q;
+            x[q] = (IS_A ? (s < r) : (s <= r)) ? br * run * s8[q] : 0.f;
+            if (s <= top && s > 0) run *= gs.a[s];
+        }
+        if (IS_A) {
+            *reinterpret_cast<float4*>(arow + c8) = make_float4(x[0], x[1], x[2], x[3]);
+            *reinterpret_cast<float4*>(arow + c8 + 4) = make_float4(x[4], x[5], x[6], x[7]);
+        } else {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) split_pack_bf16(x[2 * q], x[2 * q + 1], hi[q], lo[q]);
+            const uint32_t off = sw128(r, c8 >> 3);
+            *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    }
+}
 
-// ------------------------------------------------------------------------------------------ small helpers
+// ------------------------------------------------------------------------------------------ the inverse
+constexpr int kAsLd = 68;  // row stride (floats) of the [64][68] fp32 scratch holding A, then T
+
 __device__ __forceinline__ uint32_t f2tf32(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -119,14 +150,14 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-// 16x16 blocks of the [64][68] fp32 scratch, as tf32 mma.sync fragments.  A block is named by its logical
-// origin (r0, c0); `tr` = it is stored transposed in the mirrored position (element (r, c) of the logical
-// block at scratch row c0 + c, column r0 + r).
+// 16x16 blocks of the scratch, as tf32 mma.sync fragments.  A block is named by its logical origin (r0, c0);
+// `tr` = it is stored transposed in the mirrored position (element (r, c) of the logical block at scratch
+// row c0 + c, column r0 + r).
 struct Frag16 {
     uint32_t a[2][4];  // as the A operand: k-halves 0, 1
 };
 __device__ __forceinline__ float blk(const float* S, int r0, int c0, int r, int c, bool tr) {
-    return tr ? S[(c0 + c) * TcSmem::AS_LD + r0 + r] : S[(r0 + r) * TcSmem::AS_LD + c0 + c];
+    return tr ? S[(c0 + c) * kAsLd + r0 + r] : S[(r0 + r) * kAsLd + c0 + c];
 }
 __device__ __forceinline__ void load_a16(const float* S, int r0, int c0, bool tr, int lane, Frag16& f) {
     const int g = lane >> 2, t = lane & 3;
@@ -160,8 +191,8 @@ __device__ __forceinline__ void store16(float* S, int r0, int c0, bool tr, int l
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh) {
         const int c = 8 * nh + 2 * t;
-        float* p00 = tr ? &S[(c0 + c) * TcSmem::AS_LD + r0 + g] : &S[(r0 + g) * TcSmem::AS_LD + c0 + c];
-        const int dc = tr ? TcSmem::AS_LD : 1, dr = tr ? 1 : TcSmem::AS_LD;
+        float* p00 = tr ? &S[(c0 + c) * kAsLd + r0 + g] : &S[(r0 + g) * kAsLd + c0 + c];
+        const int dc = tr ? kAsLd : 1, dr = tr ? 1 : kAsLd;
         p00[0] = sgn * acc[nh][0];
         p00[dc] = sgn * acc[nh][1];
         p00[8 * dr] = sgn * acc[nh][2];
@@ -219,13 +250,13 @@ __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane,
         for (int r = 0; r < 16; ++r) {
             float acc = (r == c) ? 1.f : 0.f;
 #pragma unroll
-            for (int s = 0; s < r; ++s) acc = fmaf(-S[(b0 + r) * TcSmem::AS_LD + b0 + s], t[s], acc);
+            for (int s = 0; s < r; ++s) acc = fmaf(-S[(b0 + r) * kAsLd + b0 + s], t[s], acc);
             t[r] = (r < c) ? 0.f : acc;
         }
         __syncwarp();
         if (lane < 16) {
 #pragma unroll
-            for (int r = 0; r < 16; ++r) S[(b0 + r) * TcSmem::AS_LD + b0 + c] = t[r];
+            for (int r = 0; r < 16; ++r) S[(b0 + r) * kAsLd + b0 + c] = t[r];
         }
         // emit column c of T_ii: lanes 0-15 rows 0-7, lanes 16-31 rows 8-15
         const int s = b0 + c, hr = lane >> 4;
@@ -289,12 +320,207 @@ __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane,
     }
 }
 
-// ------------------------------------------------------------------------------------------ the kernel
+// Validated sequence bounds of sequence n: row in q/k/v, first token bos and end eos within the row.
+// Returns false (and sets the error word) for a malformed cu_seqlens entry.
+__device__ __forceinline__ bool tc_seq_bounds(const FwdParams& p, int n, int& row, int& bos, int& eos, unsigned* err) {
+    if (p.cu_seqlens) {
+        row = 0;
+        bos = p.cu_seqlens[n];
+        eos = p.cu_seqlens[n + 1];
+        if (bos < 0 || eos < bos || eos > p.T) {
+            atomicOr(err, kErrSeqlens);
+            return false;
+        }
+    } else {
+        row = n;
+        bos = 0;
+        eos = p.T;
+    }
+    return true;
+}
+
+// ------------------------------------------------------------------------------------------ the WY kernel
+// Shared-memory map (bytes from a 1024-aligned base).  The S1 MMA reads a 128-row A operand per 64-channel
+// panel (rows 0-63: the K tile; rows 64-127: whatever follows it, results unused), so each K panel is
+// followed by 8 KB of other data: the T' and T''_hi emission areas.
+struct WySmem {
+    static constexpr uint32_t K0 = 0;        // K channels 0-63, [64 tokens][128 B] swizzled
+    static constexpr uint32_t TP = 8192;     // T'
+    static constexpr uint32_t K1 = 16384;    // K channels 64-127
+    static constexpr uint32_t TPP = 24576;   // T''_hi
+    static constexpr uint32_t TPPL = 32768;  // T''_lo
+    static constexpr uint32_t AS = 40960;    // A, then (I+A)^-1, fp32 [64][68]
+    static constexpr uint32_t GATE = AS + 64 * kAsLd * 4;
+    static constexpr uint32_t BARS = GATE + sizeof(TcGate);  // [0] K landed, [1] S1 done
+    static constexpr uint32_t MISC = BARS + 16;              // tmem base, abort flag, unit info
+    static constexpr uint32_t END = MISC + 64;
+    static constexpr uint32_t ALLOC = END + 1024;
+};
+
+// One CTA per (workspace slot, head): finds the (sequence, chunk) of its slot, builds A, inverts I + A and
+// writes T', T''_hi, T''_lo of that chunk to the workspace.
+__global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                               const FwdParams p, uint8_t* ws, unsigned* err) {
+    using namespace sm100;
+    using L = WySmem;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 16);
+    int* info = reinterpret_cast<int*>(sm + L::MISC + 32);  // row, start token, chunk, valid rows
+    TcGate& gs = *reinterpret_cast<TcGate*>(sm + L::GATE);
+    float* sA = reinterpret_cast<float*>(sm + L::AS);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long slot = blockIdx.x / p.H;
+    const int h = blockIdx.x % p.H;
+
+    if (tid == 0) {
+        // the sequence n whose slot range holds `slot`: largest n with wy_slot(n, start_n, 0) <= slot
+        int lo = 0, hi = p.n_seq - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            const long long st0 = p.cu_seqlens ? (long long)p.cu_seqlens[mid] : (long long)mid * p.T;
+            if (wy_slot(mid, st0, 0) <= slot) lo = mid;
+            else hi = mid - 1;
+        }
+        int row, bos, eos, Lc = 0, c = 0;
+        if (tc_seq_bounds(p, lo, row, bos, eos, err)) {
+            const long long start = (long long)row * p.T + bos;
+            const long long cc = slot - wy_slot(lo, start, 0);
+            if (cc >= 0 && cc * kChunk < eos - bos) {
+                c = (int)cc;
+                Lc = min(kChunk, eos - bos - c * kChunk);
+            }
+            info[1] = (int)(start + (long long)c * kChunk);
+        }
+        info[2] = Lc;
+        if (Lc > 0) {
+            mbar_init(&bars[0], 1);
+            mbar_init(&bars[1], 1);
+            *abort_flag = 0;
+            fence_barrier_init();
+            mbar_expect_tx(&bars[0], 16384);
+            tma_load_3d(sm + L::K0, &tm_k, &bars[0], 0, h, info[1]);
+            tma_load_3d(sm + L::K1, &tm_k, &bars[0], 64, h, info[1]);
+        }
+    }
+    __syncthreads();
+    const int tok0 = info[1], Lc = info[2];
+    if (Lc == 0) return;  // unused slot
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 64);
+        tmem_relinquish();
+    }
+    if (warp == 1) tc_make_gates(gs, p, (size_t)tok0, Lc, h, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        // S1 = K K^T (rows 64-127 of the A operand are other data; their results are never read)
+        if (mbar_wait(&bars[0], 0, abort_flag, err)) {
+            tc_fence_after();
+            const uint64_t d = desc_k_sw128(smem_u32(sm));
+            const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll 1
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t a = d + (kk >> 2) * 1024 + (kk & 3) * 2;
+                umma_bf16(tmem, a, a, id, kk > 0);
+            }
+            umma_commit(&bars[1]);
+        }
+    }
+    __syncwarp();
+    const bool ok = warp_wait(&bars[1], 0, abort_flag, err);
+    tc_fence_after();
+    if (ok && warp < 2) tc_row_pass<true>(taddr(tmem, 32 * warp, 0), gs, tid, 0, 63, sA + tid * kAsLd, nullptr, nullptr);
+    tc_fence_before();
+    const bool all_ok = __syncthreads_and(ok) != 0;  // one outcome for the CTA: the inverse has barriers
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
+    if (!all_ok) return;
+    const TEmit em{sm + L::TP, sm + L::TPP, sm + L::TPPL, gs.beta, gs.eG};
+    invert_unit_lower64(sA, warp, lane, 1, em);
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+        uint8_t* dst = ws + ((size_t)slot * p.H + h) * kWyUnit;
+        bulk_store(dst, sm + L::TP, 8192);
+        bulk_store(dst + 8192, sm + L::TPP, 8192);
+        bulk_store(dst + 16384, sm + L::TPPL, 8192);
+        bulk_commit();
+        bulk_wait_all();
+    }
+}
+
+// ------------------------------------------------------------------------------------------ the main kernel
+// Shared-memory map (bytes from a 1024-aligned base).
+struct TcSmem {
+    static constexpr uint32_t KQ = 0;  // 2 stages x [K ch0-63 | Q ch0-63 | K ch64-127 | Q ch64-127], 8 KB each
+    static constexpr uint32_t KQ_STAGE = 32768;
+    static constexpr uint32_t V = KQ + 2 * KQ_STAGE;  // V tile: j 0-63 | j 64-127, 8 KB each (MN-major A)
+    static constexpr uint32_t TW = V + 16384;         // 2 stages x [T''_hi | T''_lo], [r][s] K-major, 8 KB each
+    static constexpr uint32_t TP = TW + 32768;        // T': [r][s] K-major, 8 KB
+    static constexpr uint32_t PH = TP + 8192;         // P hi [2]: [r][s] K-major, 8 KB each
+    static constexpr uint32_t PL = PH + 16384;        // P lo [2]
+    static constexpr uint32_t WT = PL + 16384;        // -W^T: lines i (128) x 64 r, MN-major B, 16 KB
+    static constexpr uint32_t HT = WT + 16384;        // h^T bf16: [j][i] K-major, panels i 0-63 | 64-127, 16 KB each
+    static constexpr uint32_t OS = HT + 32768;        // output staging, rows 32-63: 2 x [16][128]
+    static constexpr uint32_t GATE = OS + 16384;      // 4 x TcGate
+    static constexpr uint32_t BARS = GATE + 4 * sizeof(TcGate);
+    static constexpr uint32_t N_BARS = 40;
+    static constexpr uint32_t MISC = BARS + 8 * N_BARS;  // tmem base, abort flag
+    static constexpr uint32_t END = MISC + 64;
+    static constexpr uint32_t ALLOC = END + 1024;  // slack for the 1024-byte alignment of the base
+};
+static_assert(TcSmem::ALLOC <= 232448, "shared memory budget");
+
+// Barrier indices.
+enum TcBar : int {
+    B_KQ_FULL = 0,     // [2] TMA K/Q landed (tx)
+    B_KQ_EMPTY = 2,    // [2] serial MMAs of the stage's chunk done
+    B_V_FULL = 4,      // V landed (tx)
+    B_V_EMPTY = 5,     // U^T MMA reading V done
+    B_GATE = 6,        // [4] gate stage written
+    B_S1_FULL = 10,    // S1 in TMEM
+    B_S1_FREE = 11,    // P rows read S1 (64)
+    B_TP_FULL = 12,    // T' landed (tx)
+    B_W_FULL = 13,     // W^T in TMEM (and T' read)
+    B_PREP = 14,       // [2] -W^T written (128)
+    B_P_FREE = 16,     // [2] P stage free: O^T MMA done and the output rows staged there stored
+    B_U_FULL = 18,     // U^T in TMEM (and -W^T no longer read)
+    B_U_CONV = 19,     // U, U.f split into bf16 hi/lo in TMEM (256)
+    B_H_FULL = 20,     // h^T MMA done
+    B_H_READY = 21,    // bf16 h^T staged in shared memory (256)
+    B_O_FULL = 22,     // O^T MMAs done
+    B_O_FREE = 23,     // O^T TMEM read (128)
+    B_DRAIN = 24,      // [2] final commit of each MMA issuer
+    B_HM_READY = 26,   // fp32 state in TMEM re-scaled by the next chunk's decay (256)
+    B_O_STAGED = 27,   // output tile staged in shared memory (128)
+    B_TW_FULL = 28,    // [2] T''_hi, T''_lo landed (tx)
+    B_TW_EMPTY = 30,   // [2] U^T MMA reading T'' done
+    B_P_READY = 32,    // [2] P written (64)
+    B_OS_FREE = 34,    // output staging rows 32-63 stored
+};
+
+// TMEM columns.  U^T is accumulated in fp32 at TM_U; the state warpgroups then write U as bf16 hi/lo pairs
+// (two values per column) to TM_UF and U diag f, also as hi/lo pairs, in place over TM_U.
+constexpr uint32_t TM_S1 = 0, TM_W = 64, TM_U = 128, TM_UF = 192, TM_O1 = 256, TM_O2 = 320, TM_H = 384,
+                   TM_COLS = 512;
+
+// Warp roles (16 warps): 0 TMA producer (K, Q, V, T', T'') and gates; 1 issues S1 and W^T; 2 issues the
+// serial MMAs (U^T, O^T, h^T); 3 stores the output tiles by TMA; 4-7 (prep / output warpgroup) stage o,
+// write -W^T and, in quadrants 2-3, P; 8-11 and 12-15 (state warpgroups, one per half of U and of the key
+// channels) split U into bf16 operands, refresh the bf16 copy of h^T, re-scale the fp32 state by the next
+// chunk's decay and write hT.
 template <bool O_F32>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const FwdParams p,
-                  unsigned* err) {
+                  const uint8_t* ws, unsigned* err) {
     using namespace sm100;
     using L = TcSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -303,7 +529,6 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 16);
     TcGate* gates = reinterpret_cast<TcGate*>(sm + L::GATE);
-    float* sA = reinterpret_cast<float*>(sm + L::AS);
 
     // Waits for in-flight copies or MMAs before exit even after an abort (bounded, error word only).
     auto drain_wait = [&](uint64_t* bar, uint32_t parity) {
@@ -323,21 +548,12 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int j0 = tile * kTcDV;
 
     int row, bos, eos;
-    if (p.cu_seqlens) {
-        row = 0;
-        bos = p.cu_seqlens[n];
-        eos = p.cu_seqlens[n + 1];
-        if (bos < 0 || eos < bos || eos > T) {
-            if (tid == 0) atomicOr(err, kErrSeqlens);
-            return;
-        }
-    } else {
-        row = n;
-        bos = 0;
-        eos = T;
-    }
+    if (!tc_seq_bounds(p, n, row, bos, eos, err)) return;
     const int nc = (eos - bos + kChunk - 1) / kChunk;
     const size_t state_base = ((size_t)n * H + h) * kTcDK * (size_t)dv + j0;
+    const long long seq_start = (long long)row * T + bos;
+    // workspace unit of chunk c: T' at +0, T''_hi | T''_lo at +8 KB
+    auto wy_unit = [&](int c) { return ws + ((size_t)wy_slot(n, seq_start, c) * H + h) * kWyUnit; };
 
     if (nc == 0) {  // empty sequence: hT = h0
         if (p.hT)
@@ -350,10 +566,10 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     if (tid == 0) {
         for (int b = 0; b < (int)L::N_BARS; ++b) {
-            const uint32_t cnt = (b == B_S1_FREE || b == B_PREP || b == B_PREP + 1 || b == B_U_CONV ||
-                                  b == B_H_READY || b == B_HM_READY || b == B_O_FREE || b == B_O_STAGED)
-                                     ? 256u
-                                     : (b == B_TP_READY ? 128u : 1u);
+            uint32_t cnt = 1;
+            if (b == B_U_CONV || b == B_H_READY || b == B_HM_READY) cnt = 256;
+            if (b == B_PREP || b == B_PREP + 1 || b == B_O_FREE || b == B_O_STAGED) cnt = 128;
+            if (b == B_S1_FREE || b == B_P_READY || b == B_P_READY + 1) cnt = 64;
             mbar_init(&bars[b], cnt);
         }
         *abort_flag = 0;
@@ -374,153 +590,102 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t sbase = smem_u32(sm);
 
     if (warp == 0) {
-        // ================================================================ producer: TMA + gates
-        int kq_issued[2] = {0, 0}, v_issued = 0;
-        auto load_kq = [&](int c) {
-            const int st = c & 1;
-            if (lane == 0) {
-                uint8_t* dst = sm + L::KQ + st * L::KQ_STAGE;
-                const int tok = row * T + bos + c * kChunk;
-                mbar_expect_tx(&bars[B_KQ_FULL + st], 32768);
-                tma_load_3d(dst + 0, &tm_k, &bars[B_KQ_FULL + st], 0, h, tok);
-                tma_load_3d(dst + 8192, &tm_q, &bars[B_KQ_FULL + st], 0, h, tok);
-                tma_load_3d(dst + 16384, &tm_k, &bars[B_KQ_FULL + st], 64, h, tok);
-                tma_load_3d(dst + 24576, &tm_q, &bars[B_KQ_FULL + st], 64, h, tok);
-            }
-            kq_issued[st]++;
-        };
-        auto load_v = [&](int c) {
-            if (lane == 0) {
-                const int tok = row * T + bos + c * kChunk;
-                mbar_expect_tx(&bars[B_V_FULL], 16384);
-                tma_load_3d(sm + L::V, &tm_v, &bars[B_V_FULL], j0, h, tok);
-                tma_load_3d(sm + L::V + 8192, &tm_v, &bars[B_V_FULL], j0 + 64, h, tok);
-            }
-            v_issued++;
-        };
-        // L2 prefetch of a later chunk's tiles, so that the load issued once a stage frees up hits L2
-        auto prefetch = [&](int c) {
+        // ================================================================ producer: TMA, bulk copies, gates
+        int kq_issued[2] = {0, 0}, tw_issued[2] = {0, 0}, v_issued = 0, tp_issued = 0;
+        auto prefetch = [&](int c) {  // L2 prefetch of a later chunk, so the load issued later hits L2
             if (lane == 0 && c < nc) {
-                const int tok = row * T + bos + c * kChunk;
+                const int tok = (int)(seq_start + c * kChunk);
                 tma_prefetch_3d(&tm_k, 0, h, tok);
                 tma_prefetch_3d(&tm_k, 64, h, tok);
                 tma_prefetch_3d(&tm_q, 0, h, tok);
                 tma_prefetch_3d(&tm_q, 64, h, tok);
                 tma_prefetch_3d(&tm_v, j0, h, tok);
                 tma_prefetch_3d(&tm_v, j0 + 64, h, tok);
+                bulk_prefetch_l2(wy_unit(c), kWyUnit);
             }
         };
-        auto make_gates = [&](int c) {
-            TcGate& gs = gates[c & 3];
-            const int c0 = bos + c * kChunk;
-            const int Lc = min(kChunk, eos - c0);
-            float gv[2], bv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int r = 2 * lane + u;
-                const size_t tok = ((size_t)row * T + c0 + r) * H + h;
-                gv[u] = r < Lc ? p.g[tok] : 0.f;
-                bv[u] = r < Lc ? p.beta[tok] : 0.f;
-            }
-            const float pair = gv[0] + gv[1];
-            float incl = pair;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, incl, d);
-                if (lane >= d) incl += y;
-            }
-            const float excl = incl - pair;
-            const float G0 = (excl + gv[0]) * kLog2e, G1 = incl * kLog2e;
-            const float Glast = __shfl_sync(0xffffffffu, G1, 31);
-            gs.G[2 * lane] = G0;
-            gs.G[2 * lane + 1] = G1;
-            gs.beta[2 * lane] = bv[0];
-            gs.beta[2 * lane + 1] = bv[1];
-            gs.f[2 * lane] = ex2_approx(Glast - G0);
-            gs.f[2 * lane + 1] = ex2_approx(Glast - G1);
-            gs.eG[2 * lane] = ex2_approx(G0);
-            gs.eG[2 * lane + 1] = ex2_approx(G1);
-            gs.a[2 * lane] = ex2_approx(gv[0] * kLog2e);
-            gs.a[2 * lane + 1] = ex2_approx(gv[1] * kLog2e);
-            if (lane == 0) {
-                gs.gamma = ex2_approx(Glast);
-                gs.L = Lc;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_GATE + (c & 3)]);
-        };
-        // iteration c loads V of chunk c + 1 and K/Q (+ gates) of chunk c + 2; the first two fill both stages
+        // iteration c: T' of chunk c + 1 (once W^T of chunk c is done with it), V of chunk c + 1, T'' and
+        // K/Q (+ gates) of chunk c + 2; the iterations before 0 fill the stages
         for (int c = -2; c < nc; ++c) {
-            if (c + 1 >= 0 && c + 1 < nc) {
+            const int c1 = c + 1, c2 = c + 2;
+            if (c1 >= 0 && c1 < nc) {
+                if (c >= 0 && !warp_wait(&bars[B_W_FULL], c & 1, abort_flag, err)) break;
+                if (lane == 0) {
+                    mbar_expect_tx(&bars[B_TP_FULL], 8192);
+                    bulk_load(sm + L::TP, wy_unit(c1), 8192, &bars[B_TP_FULL]);
+                }
+                tp_issued++;
                 if (c >= 0 && !warp_wait(&bars[B_V_EMPTY], c & 1, abort_flag, err)) break;
-                load_v(c + 1);
+                if (lane == 0) {
+                    const int tok = (int)(seq_start + c1 * kChunk);
+                    mbar_expect_tx(&bars[B_V_FULL], 16384);
+                    tma_load_3d(sm + L::V, &tm_v, &bars[B_V_FULL], j0, h, tok);
+                    tma_load_3d(sm + L::V + 8192, &tm_v, &bars[B_V_FULL], j0 + 64, h, tok);
+                }
+                v_issued++;
             }
-            if (c + 2 < nc) {
-                if (c >= 0 && !warp_wait(&bars[B_KQ_EMPTY + (c & 1)], (c >> 1) & 1, abort_flag, err)) break;
-                load_kq(c + 2);
-                make_gates(c + 2);
-                prefetch(c + 3);
+            if (c2 < nc) {
+                const int st = c2 & 1;
+                if (c >= 0 && !warp_wait(&bars[B_TW_EMPTY + st], (c >> 1) & 1, abort_flag, err)) break;
+                if (lane == 0) {
+                    mbar_expect_tx(&bars[B_TW_FULL + st], 16384);
+                    bulk_load(sm + L::TW + st * 16384, wy_unit(c2) + 8192, 16384, &bars[B_TW_FULL + st]);
+                }
+                tw_issued[st]++;
+                if (c >= 0 && !warp_wait(&bars[B_KQ_EMPTY + st], (c >> 1) & 1, abort_flag, err)) break;
+                if (lane == 0) {
+                    uint8_t* dst = sm + L::KQ + st * L::KQ_STAGE;
+                    const int tok = (int)(seq_start + c2 * kChunk);
+                    mbar_expect_tx(&bars[B_KQ_FULL + st], 32768);
+                    tma_load_3d(dst + 0, &tm_k, &bars[B_KQ_FULL + st], 0, h, tok);
+                    tma_load_3d(dst + 8192, &tm_q, &bars[B_KQ_FULL + st], 0, h, tok);
+                    tma_load_3d(dst + 16384, &tm_k, &bars[B_KQ_FULL + st], 64, h, tok);
+                    tma_load_3d(dst + 24576, &tm_q, &bars[B_KQ_FULL + st], 64, h, tok);
+                }
+                kq_issued[st]++;
+                tc_make_gates(gates[c2 & 3], p, (size_t)(seq_start + c2 * kChunk), min(kChunk, eos - bos - c2 * kChunk),
+                              h, lane);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_GATE + (c2 & 3)]);
+                prefetch(c2 + 1);
             }
         }
         // drain: wait for every load this warp issued before the CTA may exit
-        for (int st = 0; st < 2; ++st)
+        for (int st = 0; st < 2; ++st) {
             if (kq_issued[st] > 0) drain_wait(&bars[B_KQ_FULL + st], (kq_issued[st] - 1) & 1);
+            if (tw_issued[st] > 0) drain_wait(&bars[B_TW_FULL + st], (tw_issued[st] - 1) & 1);
+        }
         if (v_issued > 0) drain_wait(&bars[B_V_FULL], (v_issued - 1) & 1);
+        if (tp_issued > 0) drain_wait(&bars[B_TP_FULL], (tp_issued - 1) & 1);
     } else if (warp == 1) {
-        // ================================================================ h-independent MMAs (S1, W^T)
-        // Issued in readiness order.  S1 of chunk c + 1 needs its K/Q and the prep to have read S1 of chunk c,
-        // which it normally has before chunk c's T' is ready; W^T of chunk c needs T'.  While both are
-        // pending the thread sleeps on T' and checks the S1 conditions whenever it wakes.
+        // ================================================================ S1 = [K; Q] K^T and W^T = K^T T'^T
         if (lane == 0) {
             const uint32_t id_s1 = idesc_bf16(128, 64, false, false);
             const uint32_t id_w = idesc_bf16(128, 64, true, false);
             const uint32_t n16 = 2u << 17;  // N += 16 in an instruction descriptor (N / 8 at bit 17)
-            int ns = 0, nw = 0;  // next chunk for S1, for W^T
-            long long last = clock64();
-            auto s1_ready = [&]() {
-                return mbar_test(&bars[B_KQ_FULL + (ns & 1)], (ns >> 1) & 1) &&
-                       (ns == 0 || mbar_test(&bars[B_S1_FREE], (ns - 1) & 1));
-            };
-            while (nw < nc) {
-                bool did = false;
-                // S1 may run ahead of W^T by one chunk; W^T(nw) needs S1(nw) first
-                const bool s1_due = ns < nc && ns <= nw + 1;
-                if (s1_due && s1_ready()) {
-                    tc_fence_after();
-                    const uint64_t d = desc_k_sw128(sbase + L::KQ + (ns & 1) * L::KQ_STAGE);
+            const uint64_t d_tp = desc_k_sw128(sbase + L::TP);
+            for (int c = 0; c < nc; ++c) {
+                const int st = c & 1;
+                if (!mbar_wait(&bars[B_KQ_FULL + st], (c >> 1) & 1, abort_flag, err)) break;
+                if (c >= 1 && !mbar_wait(&bars[B_S1_FREE], (c - 1) & 1, abort_flag, err)) break;
+                tc_fence_after();
+                const uint64_t d = desc_k_sw128(sbase + L::KQ + st * L::KQ_STAGE);
 #pragma unroll 1
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t a = d + (kk >> 2) * 1024 + (kk & 3) * 2;
-                        umma_bf16(tmem + TM_S1, a, a, id_s1, kk > 0);
-                    }
-                    umma_commit(&bars[B_S1_FULL]);
-                    ++ns;
-                    did = true;
-                } else if (nw < ns && mbar_try_wait_ns(&bars[B_TP_READY], nw & 1, s1_due ? 200u : kSuspendHintNs)) {
-                    tc_fence_after();
-                    const uint64_t da = desc_mn_sw128(sbase + L::KQ + (nw & 1) * L::KQ_STAGE, 16384);
-                    const uint64_t db = desc_k_sw128(sbase + L::TP);
-                    // k-step kk (tokens s in [16 kk, 16 kk + 16)) reaches only the rows r >= 16 kk of T'
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t a = d + (kk >> 2) * 1024 + (kk & 3) * 2;
+                    umma_bf16(tmem + TM_S1, a, a, id_s1, kk > 0);
+                }
+                umma_commit(&bars[B_S1_FULL]);
+                // W^T: T' of this chunk has landed and -W^T of the previous one has been read out of TMEM
+                if (!mbar_wait(&bars[B_TP_FULL], c & 1, abort_flag, err)) break;
+                if (c >= 1 && !mbar_wait(&bars[B_PREP + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, err)) break;
+                tc_fence_after();
+                const uint64_t da = desc_mn_sw128(sbase + L::KQ + st * L::KQ_STAGE, 16384);
+                // k-step kk (tokens s in [16 kk, 16 kk + 16)) reaches only the rows r >= 16 kk of T'
 #pragma unroll 1
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + TM_W + 16 * kk, da + kk * 128, db + kk * 130, id_w - kk * n16, kk > 0);
-                    umma_commit(&bars[B_W_FULL]);
-                    ++nw;
-                    did = true;
-                } else if (nw == ns) {  // only S1 can make progress: sleep on its K/Q, then on S1_FREE
-                    mbar_try_wait(&bars[B_KQ_FULL + (ns & 1)], (ns >> 1) & 1);
-                    if (ns > 0) mbar_try_wait(&bars[B_S1_FREE], (ns - 1) & 1);
-                }
-                if (did) {
-                    last = clock64();
-                } else {
-                    if (*abort_flag) break;
-                    if (clock64() - last > kWaitLimitCycles) {
-                        *abort_flag = 1;
-                        atomicOr(err, kErrTimeout);
-                        break;
-                    }
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + TM_W + 16 * kk, da + kk * 128, d_tp + kk * 130, id_w - kk * n16, kk > 0);
+                umma_commit(&bars[B_W_FULL]);
             }
             umma_commit(&bars[B_DRAIN]);
             drain_wait(&bars[B_DRAIN], 0);
@@ -534,7 +699,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint32_t id_u2 = idesc_bf16(128, 64, false, true);
             const uint32_t id_o = idesc_bf16(128, 64, false, false);
             const uint32_t id_h = idesc_bf16(128, 128, false, true);
-            const uint32_t n16 = 2u << 17;  // N += 16 in an instruction descriptor (N / 8 at bit 17)
+            const uint32_t n16 = 2u << 17;
             const uint64_t d_v = desc_mn_sw128(sbase + L::V, 8192);
             const uint64_t d_ht = desc_k_sw128(sbase + L::HT);
             const uint64_t d_wt = desc_mn_sw128(sbase + L::WT, 8192);
@@ -543,15 +708,18 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const uint32_t kq = sbase + L::KQ + st * L::KQ_STAGE;
                 if (!mbar_wait(&bars[B_PREP + st], (c >> 1) & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[B_V_FULL], c & 1, abort_flag, err)) break;
+                if (!mbar_wait(&bars[B_TW_FULL + st], (c >> 1) & 1, abort_flag, err)) break;
                 tc_fence_after();
                 // U^T = V^T (T''_hi + T''_lo)^T - h^T W^T ; the first half does not need the state.  As T'' is
                 // lower triangular, k-step ks (tokens s in [16 ks, 16 ks + 16)) updates only columns r >= 16 ks.
+                const uint64_t d_t = desc_k_sw128(sbase + L::TW + st * 16384);
 #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk) {
                     const int ks = kk & 3;
-                    const uint64_t b = desc_k_sw128(sbase + (kk < 4 ? L::TPP : L::TPPL) + st * 8192) + ks * 130;
-                    umma_bf16(tmem + TM_U + 16 * ks, d_v + ks * 128, b, id_u1 - ks * n16, kk > 0);
+                    umma_bf16(tmem + TM_U + 16 * ks, d_v + ks * 128, d_t + (kk >> 2) * 512 + ks * 130,
+                              id_u1 - ks * n16, kk > 0);
                 }
+                umma_commit(&bars[B_TW_EMPTY + st]);
                 if (!mbar_wait(&bars[B_H_READY], c & 1, abort_flag, err)) break;
                 tc_fence_after();
 #pragma unroll 1
@@ -580,6 +748,8 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     umma_bf16_tmem_a(tmem + TM_H, a, d_k + ks * 128, id_h, 1);
                 }
                 umma_commit(&bars[B_H_FULL]);
+                if (!mbar_wait(&bars[B_P_READY + st], (c >> 1) & 1, abort_flag, err)) break;
+                tc_fence_after();
 #pragma unroll 1
                 for (int kk = 0; kk < 12; ++kk) {  // P lower triangular: k-step ks reaches columns r >= 16 ks
                     const int part = kk >> 2, ks = kk & 3;  // 0: Uhi Phi, 1: Uhi Plo, 2: Ulo Phi
@@ -596,114 +766,121 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         __syncwarp();
     } else if (warp == 3) {
         // ================================================================ output stores
-        // A full chunk's o tile is staged by the state warpgroups in the P and T'' buffers of its stage (free
-        // once its O^T MMAs are done) and leaves by TMA; a partial chunk is written directly by them.
+        // A full chunk's o tile is staged by the prep / output warpgroup, rows 0-31 in the P buffers of its
+        // stage (free once its O^T MMAs are done), rows 32-63 in OS, and leaves by TMA; a partial chunk is
+        // written directly by that warpgroup.
         if (lane == 0) {
             for (int c = 0; c < nc; ++c) {
                 const int st = c & 1;
                 if (!mbar_wait(&bars[B_O_STAGED], c & 1, abort_flag, err)) break;
                 if (eos - bos - c * kChunk >= kChunk) {
-                    const int tok0 = row * T + bos + c * kChunk;
-                    const uint32_t rg[4] = {L::PH, L::PL, L::TPP, L::TPPL};
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) tma_store_3d(&tm_o, sm + rg[b] + st * 8192, j0, h, tok0 + 16 * b);
+                    const int tok0 = (int)(seq_start + c * kChunk);
+                    tma_store_3d(&tm_o, sm + L::PH + st * 8192, j0, h, tok0);
+                    tma_store_3d(&tm_o, sm + L::PL + st * 8192, j0, h, tok0 + 16);
+                    tma_store_3d(&tm_o, sm + L::OS, j0, h, tok0 + 32);
+                    tma_store_3d(&tm_o, sm + L::OS + 8192, j0, h, tok0 + 48);
                     bulk_commit();
                     bulk_wait_read_all();
                 }
                 mbar_arrive(&bars[B_P_FREE + st]);
+                mbar_arrive(&bars[B_OS_FREE]);
             }
             bulk_wait_all();
         }
         __syncwarp();
-    } else if (warp >= 4 && warp < 12) {
-        // ================================================================ prep warpgroups
-        // Per chunk: (1) A rows, split by column halves over the quadrant-0/1 warps of both warpgroups;
-        // (2) the first warpgroup inverts (I + A), writing T' (what the W^T MMA needs) and T'' as it goes,
-        // while the quadrant-2/3 warps of the second build P; (3) -W^T.  A timed-out wait does not break out
-        // here: the warpgroups finish the iteration and leave together at the top of the next.
-        const int wsel = (warp - 4) >> 2;      // warpgroup 0 or 1
-        const int t = (tid - 128) & 127;       // TMEM lane: row of S1 / line of W^T
+    } else if (warp < 8) {
+        // ================================================================ prep / output warpgroup
+        // Iteration k: (1) the output tile of chunk k - 2 (its O^T MMAs are done by the time chunk k - 1's
+        // U^T is), read from TMEM first so the next O^T MMAs can start, then staged for the TMA store: rows
+        // 0-31 in the P buffers of its stage, rows 32-63 in OS; a partial chunk is written directly.
+        // (2) -W^T of chunk k, line i = t, from TMEM into shared memory.  (3) The P rows of chunk k (the
+        // quadrant-2/3 warps, whose TMEM lanes hold Q K^T).  The warps run independently; a timed-out wait
+        // does not break out, the warp finishes the iteration and leaves at the top of the next.
+        const int t = tid - 128;  // TMEM lane: value column j of O^T / line of W^T / row of S1
         const int wid = warp & 3;
-        for (int c = 0; c < nc; ++c) {
-            if (named_bar_or(2, 256, *abort_flag != 0)) break;
-            const int st = c & 1;
-            warp_wait(&bars[B_S1_FULL], c & 1, abort_flag, err);
-            warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err);
-            tc_fence_after();
-            const TcGate& gs = gates[c & 3];
-            // Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1): a running product down from the highest
-            // column at or below r of the columns handled, started there with one exp2; 8 columns at a time
-            auto row_pass = [&](int r, int s_lo, int s_hi, bool is_a) {
-                const int top = r < s_hi ? r : s_hi;
-                float run = (top == r) ? 1.f : ex2_approx(gs.G[r] - gs.G[top]);
-                const float br = is_a ? gs.beta[r] : 1.f;
+        const uint32_t lane_base = 32 * wid;
+        for (int k = 0; k < nc + 2; ++k) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            if (k >= 2) {
+                const int c = k - 2, st = c & 1;
+                warp_wait(&bars[B_O_FULL], c & 1, abort_flag, err);
+                if (c >= 1) warp_wait(&bars[B_OS_FREE], (c - 1) & 1, abort_flag, err);
+                tc_fence_after();
+                const TcGate& gs = gates[c & 3];
+                const int Lc = gs.L;
+                const size_t tok0 = (size_t)(seq_start + (long long)c * kChunk);
+                const size_t ostride = (size_t)H * dv;
+                size_t off = (tok0 * H + h) * (size_t)dv + j0 + t;
 #pragma unroll 1
-                for (int c8 = s_hi - 7; c8 >= s_lo; c8 -= 8) {
-                    float s8[8];
-                    tmem_ld8(taddr(tmem, 32 * wid, TM_S1 + c8), s8);
+                for (int r32 = 0; r32 < 64; r32 += 32) {
+                    float v1[32], v2[32];
+                    tmem_ld32(taddr(tmem, lane_base, TM_O1 + r32), v1);
+                    tmem_ld32(taddr(tmem, lane_base, TM_O2 + r32), v2);
                     tmem_wait_ld();
-                    float x[8];
-#pragma unroll
-                    for (int q = 7; q >= 0; --q) {
-                        const int s = c8 + q;
-                        x[q] = (is_a ? (s < r) : (s <= r)) ? br * run * s8[q] : 0.f;
-                        if (s <= top && s > 0) run *= gs.a[s];
+                    if (r32 == 32) {
+                        tc_fence_before();
+                        mbar_arrive(&bars[B_O_FREE]);
                     }
-                    if (is_a) {  // A row r: beta_r Gamma_rs (k_r . k_s), s < r
-                        float* dst = &sA[r * L::AS_LD + c8];
-                        *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
-                        *reinterpret_cast<float4*>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
-                    } else {  // P row r: Gamma_rs (q_r . k_s), s <= r, bf16 hi + lo
-                        uint32_t hi[4], lo[4];
+                    uint8_t* const stg0 = sm + (r32 ? L::OS : L::PH + st * 8192);
+                    uint8_t* const stg1 = sm + (r32 ? L::OS + 8192 : L::PL + st * 8192);
+                    const float4* eg4 = reinterpret_cast<const float4*>(gs.eG + r32);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) split_pack_bf16(x[2 * q], x[2 * q + 1], hi[q], lo[q]);
-                        const uint32_t off = sw128(r, c8 >> 3);
-                        *reinterpret_cast<uint4*>(sm + L::PH + st * 8192 + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                        *reinterpret_cast<uint4*>(sm + L::PL + st * 8192 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 e = eg4[q4];
+                        const float ev[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int q = 4 * q4 + u, r = r32 + q;
+                            const float val = p.scale * fmaf(ev[u], v1[q], v2[q]);
+                            uint8_t* stg = (q & 16) ? stg1 : stg0;
+                            if (Lc == kChunk) {  // staged for the TMA store: row r & 15 of a [16][128] box
+                                if (O_F32) reinterpret_cast<float*>(stg)[(r & 15) * kTcDV + t] = val;
+                                else reinterpret_cast<__nv_bfloat16*>(stg)[(r & 15) * kTcDV + t] = __float2bfloat16_rn(val);
+                            } else if (r < Lc) {
+                                if (O_F32) static_cast<float*>(p.o)[off] = val;
+                                else static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(val);
+                            }
+                            off += ostride;
+                        }
                     }
                 }
-            };
-            // (1) A rows (lanes 0-63), columns [32 wsel, 32 wsel + 32); S1 is then read only by the P rows
-            if (wid < 2) row_pass(t, 32 * wsel, 32 * wsel + 31, true);
-            if (wsel == 0 || wid < 2) {
-                tc_fence_before();
-                mbar_arrive(&bars[B_S1_FREE]);
-            }
-            named_bar_sync(1, 256);
-            // (2) the inverse (first warpgroup), emitting T' and T''; P rows (lanes 64-127 of the second).
-            // T'' and P of chunk c go into the stage buffers of chunk c - 2, free once its output has left.
-            if (c >= 2 && (wsel == 0 || wid >= 2))
-                warp_wait(&bars[B_P_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err);
-            if (wsel == 0) {
-                const TEmit em{sm + L::TP, sm + L::TPP + st * 8192, sm + L::TPPL + st * 8192, gs.beta, gs.eG};
-                invert_unit_lower64(sA, wid, lane, 3, em);
                 fence_proxy_async();
-                mbar_arrive(&bars[B_TP_READY]);
-            } else if (wid >= 2) {
-                row_pass(t - 64, 0, 63, false);
-                tc_fence_before();
-                mbar_arrive(&bars[B_S1_FREE]);
+                mbar_arrive(&bars[B_O_STAGED]);
             }
-            // (3) -W^T line i = t, columns r of this warpgroup's half
+            if (k >= nc) continue;
+            const int c = k, st = c & 1;
             warp_wait(&bars[B_W_FULL], c & 1, abort_flag, err);
             if (c >= 1) warp_wait(&bars[B_U_FULL], (c - 1) & 1, abort_flag, err);
             tc_fence_after();
-            {
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
                 float v[32];
-                tmem_ld32(taddr(tmem, 32 * wid, TM_W + 32 * wsel), v);
+                tmem_ld32(taddr(tmem, lane_base, TM_W + 32 * half), v);
                 tmem_wait_ld();
-                st_half_line_bf16(sm + L::WT, t, 4 * wsel, v, -1.f);
+                st_half_line_bf16(sm + L::WT, t, 4 * half, v, -1.f);
             }
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bars[B_PREP + st]);
+            if (wid >= 2) {
+                warp_wait(&bars[B_S1_FULL], c & 1, abort_flag, err);
+                warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err);
+                if (c >= 2) warp_wait(&bars[B_P_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err);
+                tc_fence_after();
+                // rows 0-31 need columns 0-31 only: the O^T MMA never reads the blocks above the diagonal
+                tc_row_pass<false>(taddr(tmem, lane_base, TM_S1), gates[c & 3], t - 64, 0, wid == 2 ? 31 : 63, nullptr,
+                                   sm + L::PH + st * 8192, sm + L::PL + st * 8192);
+                fence_proxy_async();
+                mbar_arrive(&bars[B_P_READY + st]);
+                tc_fence_before();
+                mbar_arrive(&bars[B_S1_FREE]);
+            }
         }
-    } else if (warp >= 12) {
-        // ================================================================ state / output warpgroups
-        // Warpgroups 12-15 (half 0) and 16-19 (half 1) share the serial-chain work: each splits half of U
-        // into bf16 operands, refreshes half of the state (key channels [64 half, 64 half + 64)) and then
-        // stages half of the chunk's output rows for the TMA store.
-        const int half = (warp - 12) >> 2;
+    } else {
+        // ================================================================ state warpgroups
+        // Warpgroups 8-11 (half 0) and 12-15 (half 1) share the serial-chain work: each splits half of U
+        // into bf16 operands and refreshes half of the state (key channels [64 half, 64 half + 64)).
+        const int half = (warp - 8) >> 2;
         const int j = tid & 127;  // value column (TMEM lane)
         const uint32_t lane_base = 32 * (warp & 3);
         // initial state: bf16 copy and fp32 master pre-scaled by the first chunk's decay
@@ -797,42 +974,6 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc_fence_before();
                 mbar_arrive(&bars[B_HM_READY]);
             }
-            // ---- output rows [32 half, 32 half + 32): o_r = scale (2^G_r O1_r + O2_r), 8 rows at a time
-            if (!warp_wait(&bars[B_O_FULL], c & 1, abort_flag, err)) break;
-            tc_fence_after();
-            const int Lc = gs.L;
-            const int st = c & 1;
-            const size_t tok0 = (size_t)row * T + bos + (size_t)c * kChunk;
-            const size_t ostride = (size_t)H * dv;
-            size_t off = ((tok0 + 32 * half) * H + h) * (size_t)dv + j0 + j;
-            const uint32_t rg0 = half ? L::TPP : L::PH, rg1 = half ? L::TPPL : L::PL;
-#pragma unroll 1
-            for (int r8 = 32 * half; r8 < 32 * half + 32; r8 += 8) {
-                float v1[8], v2[8];
-                tmem_ld8(taddr(tmem, lane_base, TM_O1 + r8), v1);
-                tmem_ld8(taddr(tmem, lane_base, TM_O2 + r8), v2);
-                tmem_wait_ld();
-                if (r8 == 32 * half + 24) {
-                    tc_fence_before();
-                    mbar_arrive(&bars[B_O_FREE]);
-                }
-                uint8_t* stg = sm + ((r8 & 16) ? rg1 : rg0) + st * 8192;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int r = r8 + q;
-                    const float val = p.scale * fmaf(gs.eG[r], v1[q], v2[q]);
-                    if (Lc == kChunk) {  // staged for the TMA store: row r & 15 of a [16][128] box
-                        if (O_F32) reinterpret_cast<float*>(stg)[(r & 15) * kTcDV + j] = val;
-                        else reinterpret_cast<__nv_bfloat16*>(stg)[(r & 15) * kTcDV + j] = __float2bfloat16_rn(val);
-                    } else if (r < Lc) {
-                        if (O_F32) static_cast<float*>(p.o)[off] = val;
-                        else static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(val);
-                    }
-                    off += ostride;
-                }
-            }
-            fence_proxy_async();
-            mbar_arrive(&bars[B_O_STAGED]);
         }
     }
     tc_fence_before();
@@ -846,6 +987,10 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // ------------------------------------------------------------------------------------------ host side
 inline bool tc_supported(const FwdParams& p, bool gdn2, bool /*o_f32*/) {
     return !gdn2 && p.dk == kTcDK && p.dv % kTcDV == 0 && p.T > 0;
+}
+// Workspace bytes the tcgen05 path needs (the WY kernel's output).
+inline size_t tc_workspace_bytes(int B, int T, int H, int n_seqs) {
+    return (size_t)wy_slots(B, T, n_seqs) * (size_t)H * kWyUnit;
 }
 
 static thread_local char t_tc_msg[256];
@@ -895,9 +1040,15 @@ inline bool make_out_map(CUtensorMap* map, void* base, int dv, int H, long long 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, unsigned* err, cudaStream_t stream) {
+inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, void* ws, size_t ws_bytes, unsigned* err,
+                            cudaStream_t stream) {
     if (gdn2) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "GDN-2 has no tcgen05 kernel yet");
+        return GDN_ERR_UNSUPPORTED;
+    }
+    const size_t need = tc_workspace_bytes(p.B, p.T, p.H, p.n_seq);
+    if (!ws || ws_bytes < need) {
+        snprintf(t_tc_msg, sizeof(t_tc_msg), "the tcgen05 path needs %zu bytes of workspace (got %zu)", need, ws_bytes);
         return GDN_ERR_UNSUPPORTED;
     }
     CUtensorMap mq, mk, mv, mo;
@@ -907,14 +1058,31 @@ inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, unsigned*
         snprintf(t_tc_msg, sizeof(t_tc_msg), "cuTensorMapEncodeTiled failed");
         return GDN_ERR_CUDA;
     }
+    cudaError_t e = cudaFuncSetAttribute(gdn_tc_wy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)WySmem::ALLOC);
+    if (e != cudaSuccess) {
+        snprintf(t_tc_msg, sizeof(t_tc_msg), "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        return GDN_ERR_CUDA;
+    }
+    const long long wy_grid = (long long)(wy_slots(p.B, p.T, p.n_seq)) * p.H;
+    if (wy_grid > 0x7fffffffLL) {
+        snprintf(t_tc_msg, sizeof(t_tc_msg), "too many chunks for one launch");
+        return GDN_ERR_UNSUPPORTED;
+    }
+    gdn_tc_wy_kernel<<<(unsigned)wy_grid, kWyThreads, WySmem::ALLOC, stream>>>(mk, p, static_cast<uint8_t*>(ws), err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        snprintf(t_tc_msg, sizeof(t_tc_msg), "WY kernel: %s", cudaGetErrorString(e));
+        return GDN_ERR_CUDA;
+    }
     auto kern = o_f32 ? gdn_tc_fwd_kernel<true> : gdn_tc_fwd_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TcSmem::ALLOC);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TcSmem::ALLOC);
     if (e != cudaSuccess) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         return GDN_ERR_CUDA;
     }
     const unsigned grid = (unsigned)(p.dv / kTcDV) * p.H * p.n_seq;
-    kern<<<grid, kTcThreads, TcSmem::ALLOC, stream>>>(mq, mk, mv, mo, p, err);
+    kern<<<grid, kTcThreads, TcSmem::ALLOC, stream>>>(mq, mk, mv, mo, p, static_cast<const uint8_t*>(ws), err);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "%s", cudaGetErrorString(e));

@@ -37,6 +37,14 @@
  * Every pointer must be 16-byte aligned.  The library never allocates, frees or synchronises inside a
  * *_fwd call: the caller owns every buffer, and work is enqueued on `stream` (asynchronous).
  *
+ * Workspace: the tensor-core path (bf16 inputs, dk == 128, dv a multiple of 128) first computes the WY
+ * factors of every (chunk, head) -- T' = T diag(beta e^G) and T'' = T diag(beta) with T = (I + A)^-1 --
+ * into `workspace`, then runs the chunk recurrence that reads them; it needs gdn_workspace_bytes() bytes
+ * (24 KB per chunk slot and head; slots = ceil(B T / 64) + number of sequences).  The workspace is scratch:
+ * its contents are undefined before and after a call, and it must not be shared by calls in flight at the
+ * same time.  With a smaller (or NULL) workspace, AUTO runs the SIMT kernel and TC returns
+ * GDN_ERR_UNSUPPORTED.
+ *
  * Errors
  *   Arguments are checked on the host before anything is enqueued; a failed check returns
  *   GDN_ERR_INVALID_ARG (bad pointer, size, alignment) or GDN_ERR_UNSUPPORTED (a shape or option outside
@@ -72,7 +80,8 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype; /* dtype of q, k, v (dt) a
  * forces the tcgen05 kernel (bf16 only; GDN_ERR_UNSUPPORTED otherwise). */
 typedef enum { GDN_KERNEL_AUTO = 0, GDN_KERNEL_SIMT = 1, GDN_KERNEL_TC = 2 } gdn_kernel;
 
-/* Bytes of caller-provided device workspace a call with these sizes needs (0: pass NULL, 0). */
+/* Bytes of caller-provided device workspace the tensor-core path needs for these sizes (see Workspace
+ * above); 0 when only the SIMT kernel can take them (then pass NULL, 0).  n_seqs as for the *_fwd calls. */
 size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs);
 
 /* Gated delta rule forward; see the header comment for the definition, layouts and errors. */

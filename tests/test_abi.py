@@ -89,7 +89,12 @@ def test_status_strings_and_kernel_choice(lib):
         assert lib.gdn_status_string(s).decode() not in ("", "unknown status")
     assert lib.gdn_set_kernel(9) == 1
     assert lib.gdn_set_kernel(0) == 0
-    assert lib.gdn_workspace_bytes(4, 4096, 16, 128, 256, 64, 0) == 0
+    # the tensor-core path keeps 24 KB of WY factors per (chunk slot, head); slots = ceil(B T / 64) + sequences
+    assert lib.gdn_workspace_bytes(4, 4096, 16, 128, 256, 64, 0) == (256 + 4) * 16 * 24576
+    assert lib.gdn_workspace_bytes(1, 65536, 16, 128, 256, 64, 16) == (1024 + 16) * 16 * 24576
+    assert lib.gdn_workspace_bytes(1, 100, 2, 128, 128, 64, 0) == (2 + 1) * 2 * 24576
+    assert lib.gdn_workspace_bytes(4, 4096, 16, 64, 64, 64, 0) == 0  # shapes only the SIMT kernel takes
+    assert lib.gdn_workspace_bytes(4, 0, 16, 128, 256, 64, 0) == 0
 
 
 def test_binding_refuses_cpu_tensors(lib):
