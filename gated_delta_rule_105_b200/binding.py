@@ -56,6 +56,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_last_error.restype = ctypes.c_char_p
     lib.gdn_debug_umma_selftest.argtypes = [vp, vp, vp, i, vp]
     lib.gdn_debug_umma_selftest.restype = i
+    lib.gdn_profile_enable.argtypes = [i]
+    lib.gdn_profile_enable.restype = i
+    lib.gdn_profile_take.argtypes = [i, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
+    lib.gdn_profile_take.restype = i
     _lib = lib
     return lib
 
@@ -102,6 +106,25 @@ def check_error(stream=None) -> None:
     """Synchronise the stream and raise if a kernel reported a device-side error."""
     s = torch.cuda.current_stream() if stream is None else stream
     _raise_on(load_library().gdn_check_error(ctypes.c_void_p(s.cuda_stream)))
+
+
+PROFILE_KERNELS = {"gdn_simt_fwd_kernel": 0, "gdn_tc_wy_kernel": 1, "gdn_tc_fwd_kernel": 2}
+
+
+def profile_enable(on: bool = True) -> None:
+    """Bracket every library kernel launch with CUDA events on its stream (see ``gdn_profile_take``)."""
+    _raise_on(load_library().gdn_profile_enable(1 if on else 0))
+
+
+def profile_take() -> dict:
+    """{kernel name: (launches, total device ms)} of the launches recorded since the last take."""
+    out = {}
+    for name, kid in PROFILE_KERNELS.items():
+        n, ms = ctypes.c_int(0), ctypes.c_double(0.0)
+        _raise_on(load_library().gdn_profile_take(kid, ctypes.byref(n), ctypes.byref(ms)))
+        if n.value:
+            out[name] = (n.value, ms.value)
+    return out
 
 
 def umma_selftest(A, B, mode):

@@ -7,6 +7,7 @@
 
 #include "gdn.h"
 #include "gdn_common.cuh"
+#include "gdn_prof.cuh"
 #include "gdn_simt.cuh"
 #include "gdn_tc.cuh"
 #include "gdn_tc_selftest.cuh"
@@ -86,7 +87,9 @@ static gdn_status launch_simt_dk(const FwdParams& p, unsigned* err, cudaStream_t
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     dim3 grid(p.dv / DVT, p.H, p.n_seq);
+    ProfScope prof(PK_SIMT, stream);
     kern<<<grid, kSimtThreads, L::bytes, stream>>>(p, err);
+    prof.done();
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "SIMT kernel launch: %s", cudaGetErrorString(e));
     return GDN_OK;
@@ -202,6 +205,19 @@ const char* gdn_status_string(gdn_status s) {
 }
 
 const char* gdn_last_error(void) { return t_msg; }
+
+gdn_status gdn_profile_enable(int on) {
+    prof_state().on.store(on != 0);
+    return GDN_OK;
+}
+
+gdn_status gdn_profile_take(int kernel, int* launches, double* total_ms) {
+    t_msg[0] = 0;
+    if (kernel < 0 || kernel >= PK_COUNT) return fail(GDN_ERR_INVALID_ARG, "kernel id must be 0..%d", PK_COUNT - 1);
+    if (!launches || !total_ms) return fail(GDN_ERR_INVALID_ARG, "NULL output pointer");
+    if (!prof_take(kernel, launches, total_ms)) return fail(GDN_ERR_CUDA, "a recorded launch event failed");
+    return GDN_OK;
+}
 
 gdn_status gdn_debug_umma_selftest(const float* A, const float* B, float* D, int mode, cudaStream_t stream) {
     t_msg[0] = 0;

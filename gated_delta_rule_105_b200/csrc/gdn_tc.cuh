@@ -1069,7 +1069,9 @@ inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, void* ws,
         snprintf(t_tc_msg, sizeof(t_tc_msg), "too many chunks for one launch");
         return GDN_ERR_UNSUPPORTED;
     }
+    ProfScope prof_wy(PK_TC_WY, stream);
     gdn_tc_wy_kernel<<<(unsigned)wy_grid, kWyThreads, WySmem::ALLOC, stream>>>(mk, p, static_cast<uint8_t*>(ws), err);
+    prof_wy.done();
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "WY kernel: %s", cudaGetErrorString(e));
@@ -1082,7 +1084,9 @@ inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, void* ws,
         return GDN_ERR_CUDA;
     }
     const unsigned grid = (unsigned)(p.dv / kTcDV) * p.H * p.n_seq;
+    ProfScope prof_main(PK_TC_MAIN, stream);
     kern<<<grid, kTcThreads, TcSmem::ALLOC, stream>>>(mq, mk, mv, mo, p, static_cast<const uint8_t*>(ws), err);
+    prof_main.done();
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "%s", cudaGetErrorString(e));

@@ -122,6 +122,15 @@ const char* gdn_last_error(void);
  * the MMA k-step loop, and writes D = A B (fp32, row-major [M][N], device).  Asynchronous on `stream`. */
 gdn_status gdn_debug_umma_selftest(const float* A, const float* B, float* D, int mode, cudaStream_t stream);
 
+/* Per-kernel device timing, a measurement aid (off by default; process-wide).  While enabled, every kernel
+ * launch made by gdn_chunk_fwd / gdn2_chunk_fwd is bracketed by two CUDA events recorded on its stream.
+ * gdn_profile_take(kernel, &launches, &total_ms) waits for the recorded events of one kernel -- 0: SIMT
+ * kernel, 1: tensor-core WY kernel, 2: tensor-core chunk kernel -- returns how many launches they cover and
+ * their summed device time in milliseconds, and forgets them.  Errors: GDN_ERR_INVALID_ARG for an unknown
+ * kernel id or NULL outputs, GDN_ERR_CUDA if an event failed. */
+gdn_status gdn_profile_enable(int on);
+gdn_status gdn_profile_take(int kernel, int* launches, double* total_ms);
+
 #ifdef __cplusplus
 }
 #endif
