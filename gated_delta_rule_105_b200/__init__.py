@@ -5,7 +5,9 @@ The compute lives in ``libgdn.so`` (hand-written sm_100a CUDA behind a C ABI dec
 synthetic inputs of the shapes the method is measured on.
 """
 from .binding import (GdnError, check_error, chunk_gated_delta_rule, gdn2_chunk_fwd, gdn_chunk_fwd,
-                      last_kernel, load_library, profile_enable, profile_take, set_kernel, workspace_bytes)
+                      gdn_chunk_fwd_noalloc, last_kernel, load_library, profile_enable, profile_take, set_kernel,
+                      workspace_bytes)
 
 __all__ = ["GdnError", "check_error", "chunk_gated_delta_rule", "gdn2_chunk_fwd", "gdn_chunk_fwd",
-           "last_kernel", "load_library", "profile_enable", "profile_take", "set_kernel", "workspace_bytes"]
+           "gdn_chunk_fwd_noalloc", "last_kernel", "load_library", "profile_enable", "profile_take", "set_kernel",
+           "workspace_bytes"]

@@ -42,6 +42,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_workspace_bytes.restype = sz
     lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [i] * 8 + [vp, i, vp, sz, vp]
     lib.gdn_chunk_fwd.restype = i
+    lib.gdn_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [i] * 8 + [vp, i, vp]
+    lib.gdn_chunk_fwd_noalloc.restype = i
     lib.gdn2_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, f, fp, vp, fp] + [i] * 8 + [vp, i, vp, sz, vp]
     lib.gdn2_chunk_fwd.restype = i
     lib.gdn_set_kernel.argtypes = [i]
@@ -201,6 +203,25 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, output_final_state=True
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(o), _ptr(hT),
         B, T, H, dk, dv, BT, _dtype_code(q), _dtype_code(o), _ptr(cu_seqlens),
         n_seqs, _ptr(ws), 0 if ws is None else ws.numel(), ctypes.c_void_p(stream))
+    _raise_on(st)
+    return o, hT
+
+
+def gdn_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, h0=None, output_final_state=True, cu_seqlens=None,
+                          BT=64, o=None, hT=None, o_dtype=None):
+    """As :func:`gdn_chunk_fwd`, through ``gdn_chunk_fwd_noalloc``: no workspace is allocated (the library's
+    static scratch serves the tensor-core path; calls must not overlap on the device)."""
+    B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype)
+    _check_dev("g", g, torch.float32)
+    _check_dev("beta", beta, torch.float32)
+    if g.shape != (B, T, H) or beta.shape != (B, T, H):
+        raise ValueError("g and beta must be [B,T,H]")
+    scale = dk ** -0.5 if scale is None else float(scale)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    st = load_library().gdn_chunk_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(o), _ptr(hT),
+        B, T, H, dk, dv, BT, _dtype_code(q), _dtype_code(o), _ptr(cu_seqlens),
+        0 if cu_seqlens is None else n_seq, ctypes.c_void_p(stream))
     _raise_on(st)
     return o, hT
 

@@ -17,6 +17,10 @@ namespace gdn {
 __device__ unsigned int g_err_word;
 
 static thread_local char t_msg[512];
+
+// Scratch for gdn_chunk_fwd_noalloc: reserved once per process and device when the module loads, so that
+// entry point never allocates.  Its size is GDN_STATIC_WS_BYTES (gdn.h).
+static __device__ __align__(256) uint8_t g_static_ws[GDN_STATIC_WS_BYTES];
 static thread_local gdn_kernel t_last_kernel = GDN_KERNEL_AUTO;
 static std::atomic<int> g_kernel_choice{GDN_KERNEL_AUTO};
 
@@ -159,6 +163,21 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
     return run(p, false, dt, o_dt, workspace, ws_bytes, stream);
 }
 
+gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                 float scale, const float* h0, void* o, float* hT, int B, int T, int H, int dk,
+                                 int dv, int BT, gdn_dtype dt, gdn_dtype o_dt, const int32_t* cu_seqlens,
+                                 int n_seqs, cudaStream_t stream) {
+    int n_seq = 0;
+    gdn_status st = check_common(q, k, v, g, beta, nullptr, false, scale, h0, o, hT, B, T, H, dk, dv, BT, dt,
+                                 o_dt, cu_seqlens, n_seqs, nullptr, 0, &n_seq);
+    if (st != GDN_OK) return st;
+    void* ws = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ws, g_static_ws);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "static scratch: %s", cudaGetErrorString(e));
+    FwdParams p{q, k, v, g, beta, nullptr, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
+    return run(p, false, dt, o_dt, ws, (size_t)GDN_STATIC_WS_BYTES, stream);
+}
+
 gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* b,
                           const float* w, float scale, const float* h0, void* o, float* hT, int B, int T, int H,
                           int dk, int dv, int BT, gdn_dtype dt, gdn_dtype o_dt, const int32_t* cu_seqlens,
@@ -222,7 +241,7 @@ gdn_status gdn_profile_take(int kernel, int* launches, double* total_ms) {
 gdn_status gdn_debug_umma_selftest(const float* A, const float* B, float* D, int mode, cudaStream_t stream) {
     t_msg[0] = 0;
     if (!A || !B || !D) return fail(GDN_ERR_INVALID_ARG, "NULL pointer");
-    if (mode < 0 || mode > 4) return fail(GDN_ERR_INVALID_ARG, "mode must be 0..4 (got %d)", mode);
+    if (mode < 0 || mode > 5) return fail(GDN_ERR_INVALID_ARG, "mode must be 0..5 (got %d)", mode);
     gdn_status st;
     unsigned* err = err_word_ptr(&st);
     if (!err) return st;

@@ -20,9 +20,10 @@
 // M = 128 tcgen05.mma with bf16 operands in 128B-swizzled shared memory (or U in TMEM) and an fp32
 // accumulator in TMEM.
 // Precision: every bf16 operand whose rounding would reach the output at the bf16-ulp level is avoided or
-// split.  U and U diag f are kept as bf16 hi + lo pairs (in TMEM, as the A operand), P and T'' likewise
-// (in shared memory); 2^G_r is applied to the fp32 accumulator of h^T Q^T instead of to Q.  The remaining
-// bf16 operands are h^T, W^T, T' and the inputs themselves.
+// split.  U diag f (in TMEM, as the A operand of the h^T MMA) and T'' are bf16 hi + lo pairs; the read-out
+// product U^T P^T runs on kind::tf32 with U in fp32 straight from TMEM and P stored as tf32; 2^G_r is
+// applied to the fp32 accumulator of h^T Q^T instead of to Q.  The remaining bf16 operands are h^T, W^T,
+// T' and the inputs themselves.
 // The operands T', T'' and P are lower triangular: the MMAs that read them skip the blocks above the
 // diagonal (k-step ks of 16 tokens only reaches the output columns r >= 16 ks).
 // All mbarrier waits are bounded: on time-out the CTA sets the error word and drains to the exit.
@@ -97,9 +98,17 @@ __device__ __forceinline__ void tc_make_gates(TcGate& gs, const FwdParams& p, si
     }
 }
 
+// fp32 -> tf32 (round to nearest, ties away), returned as the fp32 bit pattern with the low 13 bits clear.
+__device__ __forceinline__ uint32_t f2tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
 // One row r of A (IS_A: beta_r Gamma_rs (k_r . k_s), s < r, fp32 into `arow`) or of P (Gamma_rs (q_r . k_s),
-// s <= r, bf16 hi + lo into the 128B-swizzled `ph`, `pl`), columns [s_lo, s_hi], from the dot products in
-// TMEM (`ta` = this warp's lanes, column of s = 0).  Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1) is a
+// s <= r, rounded to tf32 and stored as fp32 in the 128B-swizzled K-major layout of a kind::tf32 operand:
+// columns 0-31 in `ph`, 32-63 in `pl`), columns [s_lo, s_hi], from the dot products in TMEM (`ta` = this
+// warp's lanes, column of s = 0).  Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1) is a
 // running product down from the highest column at or below r, started there with one exp2.
 template <bool IS_A>
 __device__ __forceinline__ void tc_row_pass(uint32_t ta, const TcGate& gs, int r, int s_lo, int s_hi, float* arow,
@@ -124,12 +133,12 @@ __device__ __forceinline__ void tc_row_pass(uint32_t ta, const TcGate& gs, int r
             *reinterpret_cast<float4*>(arow + c8) = make_float4(x[0], x[1], x[2], x[3]);
             *reinterpret_cast<float4*>(arow + c8 + 4) = make_float4(x[4], x[5], x[6], x[7]);
         } else {
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) split_pack_bf16(x[2 * q], x[2 * q + 1], hi[q], lo[q]);
-            const uint32_t off = sw128(r, c8 >> 3);
-            *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            uint8_t* panel = (c8 & 32) ? pl : ph;
+            const uint32_t ch = (c8 & 31) >> 2;  // 16-byte chunk of 4 fp32
+            *reinterpret_cast<uint4*>(panel + sw128(r, ch)) =
+                make_uint4(f2tf32(x[0]), f2tf32(x[1]), f2tf32(x[2]), f2tf32(x[3]));
+            *reinterpret_cast<uint4*>(panel + sw128(r, ch + 1)) =
+                make_uint4(f2tf32(x[4]), f2tf32(x[5]), f2tf32(x[6]), f2tf32(x[7]));
         }
     }
 }
@@ -137,11 +146,6 @@ __device__ __forceinline__ void tc_row_pass(uint32_t ta, const TcGate& gs, int r
 // ------------------------------------------------------------------------------------------ the inverse
 constexpr int kAsLd = 68;  // row stride (floats) of the [64][68] fp32 scratch holding A, then T
 
-__device__ __forceinline__ uint32_t f2tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
 // D(16x8) += A(16x8) B(8x8), tf32 inputs, fp32 accumulate (legacy warp-level MMA, used only for the
 // 16x16 blocks of the triangular inverse).
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
@@ -342,19 +346,19 @@ __device__ __forceinline__ bool tc_seq_bounds(const FwdParams& p, int n, int& ro
 // ------------------------------------------------------------------------------------------ the WY kernel
 // Shared-memory map (bytes from a 1024-aligned base).  The S1 MMA reads a 128-row A operand per 64-channel
 // panel (rows 0-63: the K tile; rows 64-127: whatever follows it, results unused), so each K panel is
-// followed by 8 KB of other data: the T' and T''_hi emission areas.
+// followed by 8 KB of other data: the T' and T''_hi emission areas.  T''_lo reuses the first K panel.
 struct WySmem {
-    static constexpr uint32_t K0 = 0;        // K channels 0-63, [64 tokens][128 B] swizzled
+    static constexpr uint32_t K0 = 0;        // K channels 0-63, [64 tokens][128 B] swizzled; then T''_lo
     static constexpr uint32_t TP = 8192;     // T'
     static constexpr uint32_t K1 = 16384;    // K channels 64-127
     static constexpr uint32_t TPP = 24576;   // T''_hi
-    static constexpr uint32_t TPPL = 32768;  // T''_lo
-    static constexpr uint32_t AS = 40960;    // A, then (I+A)^-1, fp32 [64][68]
+    static constexpr uint32_t TPPL = K0;     // written by the inverse, once S1 has been computed from K
+    static constexpr uint32_t AS = 32768;    // A, then (I+A)^-1, fp32 [64][68]
     static constexpr uint32_t GATE = AS + 64 * kAsLd * 4;
     static constexpr uint32_t BARS = GATE + sizeof(TcGate);  // [0] K landed, [1] S1 done
     static constexpr uint32_t MISC = BARS + 16;              // tmem base, abort flag, unit info
     static constexpr uint32_t END = MISC + 64;
-    static constexpr uint32_t ALLOC = END + 1024;
+    static constexpr uint32_t ALLOC = END + 1024;  // 4 CTAs per SM
 };
 
 // One CTA per (workspace slot, head): finds the (sequence, chunk) of its slot, builds A, inverts I + A and
@@ -506,8 +510,8 @@ enum TcBar : int {
     B_OS_FREE = 34,    // output staging rows 32-63 stored
 };
 
-// TMEM columns.  U^T is accumulated in fp32 at TM_U; the state warpgroups then write U as bf16 hi/lo pairs
-// (two values per column) to TM_UF and U diag f, also as hi/lo pairs, in place over TM_U.
+// TMEM columns.  U^T is accumulated in fp32 at TM_U and read there, as tf32, by the O2 MMA; the state
+// warpgroups write U diag f as bf16 hi/lo pairs (two values per column) to TM_UF for the h^T MMA.
 constexpr uint32_t TM_S1 = 0, TM_W = 64, TM_U = 128, TM_UF = 192, TM_O1 = 256, TM_O2 = 320, TM_H = 384,
                    TM_COLS = 512;
 
@@ -699,6 +703,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint32_t id_u2 = idesc_bf16(128, 64, false, true);
             const uint32_t id_o = idesc_bf16(128, 64, false, false);
             const uint32_t id_h = idesc_bf16(128, 128, false, true);
+            const uint32_t id_o2 = idesc_tf32(128, 64, false, false);
             const uint32_t n16 = 2u << 17;
             const uint64_t d_v = desc_mn_sw128(sbase + L::V, 8192);
             const uint64_t d_ht = desc_k_sw128(sbase + L::HT);
@@ -744,18 +749,20 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk) {  // kk < 4: hi, else lo; s-step ks covers values 16 ks .. 16 ks + 15
                     const int ks = kk & 3;
-                    const uint32_t a = tmem + TM_U + (ks >> 1) * 32 + (kk >> 2) * 16 + (ks & 1) * 8;
+                    const uint32_t a = tmem + TM_UF + (ks >> 1) * 32 + (kk >> 2) * 16 + (ks & 1) * 8;
                     umma_bf16_tmem_a(tmem + TM_H, a, d_k + ks * 128, id_h, 1);
                 }
                 umma_commit(&bars[B_H_FULL]);
                 if (!mbar_wait(&bars[B_P_READY + st], (c >> 1) & 1, abort_flag, err)) break;
                 tc_fence_after();
+                // O2^T = U^T P^T on kind::tf32: U fp32 straight from TM_U, P fp32 (tokens 0-31 in PH, 32-63 in
+                // PL); k-step ks8 covers 8 tokens and, P being lower triangular, only columns r >= 16 (ks8 / 2)
 #pragma unroll 1
-                for (int kk = 0; kk < 12; ++kk) {  // P lower triangular: k-step ks reaches columns r >= 16 ks
-                    const int part = kk >> 2, ks = kk & 3;  // 0: Uhi Phi, 1: Uhi Plo, 2: Ulo Phi
-                    const uint32_t a = tmem + TM_UF + (part == 2 ? 32 : 0) + ks * 8;
-                    const uint64_t b = desc_k_sw128(sbase + (part == 1 ? L::PL : L::PH) + st * 8192) + ks * 130;
-                    umma_bf16_tmem_a(tmem + TM_O2 + 16 * ks, a, b, id_o - ks * n16, kk > 0);
+                for (int ks8 = 0; ks8 < 8; ++ks8) {
+                    const int r0 = 16 * (ks8 >> 1);
+                    const uint64_t b = desc_k_sw128(sbase + ((ks8 & 4) ? L::PL : L::PH) + st * 8192) +
+                                       ((r0 * 128 + (ks8 & 3) * 32) >> 4);
+                    umma_tf32_tmem_a(tmem + TM_O2 + r0, tmem + TM_U + 8 * ks8, b, id_o2 - (r0 >> 4) * n16, ks8 > 0);
                 }
                 umma_commit(&bars[B_O_FULL]);
                 umma_commit(&bars[B_KQ_EMPTY + st]);
@@ -908,9 +915,8 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         for (int c = 0; c < nc; ++c) {
             const TcGate& gs = gates[c & 3];
-            // ---- U (values [32 half, 32 half + 32)): fp32 accumulator -> bf16 hi/lo pairs.
-            // U (for O2) goes to TM_UF (hi of values 0-63 in columns 0-31, lo in 32-63); U diag f (for h^T)
-            // in place over its own fp32 columns of TM_U as [hi | lo], 16 columns each.
+            // ---- U diag f (values [32 half, 32 half + 32)) as bf16 hi/lo pairs for the h^T MMA, to TM_UF
+            // ([hi | lo], 16 columns each per half).  U itself stays fp32 in TM_U: the O2 MMA reads it as tf32.
             if (!warp_wait(&bars[B_U_FULL], c & 1, abort_flag, err)) break;
             if (!warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err)) break;
             tc_fence_after();
@@ -920,16 +926,12 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tmem_wait_ld();
                 uint32_t hi[16], lo[16];
 #pragma unroll
-                for (int q = 0; q < 16; ++q) split_pack_bf16(u[2 * q], u[2 * q + 1], hi[q], lo[q]);
-                tmem_st16u(taddr(tmem, lane_base, TM_UF + 16 * half), hi);
-                tmem_st16u(taddr(tmem, lane_base, TM_UF + 32 + 16 * half), lo);
-#pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const int s0 = 32 * half + 2 * q;
                     split_pack_bf16(u[2 * q] * gs.f[s0], u[2 * q + 1] * gs.f[s0 + 1], hi[q], lo[q]);
                 }
-                tmem_st16u(taddr(tmem, lane_base, TM_U + 32 * half), hi);
-                tmem_st16u(taddr(tmem, lane_base, TM_U + 32 * half + 16), lo);
+                tmem_st16u(taddr(tmem, lane_base, TM_UF + 32 * half), hi);
+                tmem_st16u(taddr(tmem, lane_base, TM_UF + 32 * half + 16), lo);
             }
             tmem_wait_st();
             tc_fence_before();

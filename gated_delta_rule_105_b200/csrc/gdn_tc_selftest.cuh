@@ -7,6 +7,7 @@
 // mode 2: A K-major  [128 x 64],                                     B MN-major [K=64  x N=128] (N blocks 8 KB apart)
 // mode 3: A K-major  [128 x 128] (two panels),                       B MN-major [K=128 x N=64]
 // mode 4: A in tensor memory [128 x 64] (bf16 pairs per column),      B K-major  [N=64  x K=64]
+// mode 5: kind::tf32, A in tensor memory [128 x 32] (fp32, one per column), B K-major fp32  [N=64 x K=32]
 #pragma once
 
 #include "gdn_sm100.cuh"
@@ -22,6 +23,7 @@ __host__ __device__ inline SelftestShape selftest_shape(int mode) {
         case 1: return {128, 64, 64};
         case 2: return {128, 128, 64};
         case 4: return {128, 64, 64};
+        case 5: return {128, 64, 32};
         default: return {128, 64, 128};
     }
 }
@@ -49,7 +51,7 @@ __global__ void __launch_bounds__(128) gdn_umma_selftest_kernel(const float* A, 
             uint8_t* p = sA + blk * 8192 + sw128(k, mm / 8) + (mm % 8) * 2;
             *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(A[m * s.K + k]);
         }
-    } else if (mode != 4) {
+    } else if (mode < 4) {
         // K-major: line = m, 64 K per line, K panel p at p * 16384
         for (int e = tid; e < s.M * s.K; e += 128) {
             const int m = e / s.K, k = e % s.K;
@@ -59,7 +61,12 @@ __global__ void __launch_bounds__(128) gdn_umma_selftest_kernel(const float* A, 
         }
     }
     // ---- stage B
-    if (mode == 2 || mode == 3) {
+    if (mode == 5) {  // K-major fp32: line = n, 32 K per 128-byte line
+        for (int e = tid; e < s.K * s.N; e += 128) {
+            const int k = e / s.N, n = e % s.N;
+            *reinterpret_cast<float*>(sB + sw128(n, k / 4) + (k % 4) * 4) = B[k * s.N + n];
+        }
+    } else if (mode == 2 || mode == 3) {
         // MN-major: line = k, 64 N per line, N block b at b * 8192 (mode 2); mode 3 has one N block of 128 lines
         for (int e = tid; e < s.K * s.N; e += 128) {
             const int k = e / s.N, n = e % s.N;
@@ -100,7 +107,23 @@ __global__ void __launch_bounds__(128) gdn_umma_selftest_kernel(const float* A, 
         __syncthreads();
         tc_fence_after();
     }
-    if (tid == 0) {
+    if (mode == 5) {  // A rows into tensor memory columns 64..95, one fp32 per column
+        const int m = warp * 32 + (tid % 32);
+        float row[32];
+        for (int c = 0; c < 32; ++c) row[c] = A[m * s.K + c];
+        tmem_st32(taddr(tb, warp * 32, 64), row);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    if (tid == 0 && mode == 5) {
+        const uint32_t b0 = smem_u32(sB);
+        for (int kk = 0; kk < s.K / 8; ++kk)
+            umma_tf32_tmem_a(tb, tb + 64 + kk * 8, desc_k_sw128(b0 + kk * 32), idesc_tf32(s.M, s.N, false, false),
+                             kk > 0 ? 1u : 0u);
+        umma_commit(&bar);
+    } else if (tid == 0) {
         const uint32_t idesc = idesc_bf16(s.M, s.N, mode == 1, mode == 2 || mode == 3);
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
         for (int kk = 0; kk < s.K / 16; ++kk) {

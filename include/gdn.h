@@ -91,6 +91,22 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          const int32_t* cu_seqlens, int n_seqs,
                          void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* Size of the scratch array compiled into the library for gdn_chunk_fwd_noalloc: 128 MiB of device memory,
+ * reserved per process and device when the library's device code is loaded. */
+#define GDN_STATIC_WS_BYTES (128u * 1024u * 1024u)
+
+/* gdn_chunk_fwd without a caller workspace and without any allocation: the tensor-core path uses the
+ * library's static scratch (GDN_STATIC_WS_BYTES).  A call that needs more scratch than that (see
+ * gdn_workspace_bytes) runs as gdn_chunk_fwd with a too-small workspace would: AUTO takes the SIMT kernel,
+ * TC returns GDN_ERR_UNSUPPORTED.  All calls of this entry point in a process share the one scratch per
+ * device, so they must not overlap on the device: issue them on one stream, or order them (events,
+ * synchronisation); concurrent callers use gdn_chunk_fwd with their own workspaces.  Arguments, layouts
+ * and errors are otherwise those of gdn_chunk_fwd. */
+gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                 float scale, const float* h0, void* o, float* hT,
+                                 int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt, gdn_dtype o_dt,
+                                 const int32_t* cu_seqlens, int n_seqs, cudaStream_t stream);
+
 /* Gated Delta Rule-2 forward; g, b are [B,T,H,dk] and w is [B,T,H,dv], all fp32. */
 gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* b,
                           const float* w, float scale, const float* h0, void* o, float* hT,
@@ -114,12 +130,14 @@ const char* gdn_status_string(gdn_status status);
 /* Description of the most recent failure on the calling thread ("" if none). */
 const char* gdn_last_error(void);
 
-/* Diagnostic (no counterpart on the pages): checks the tensor-core operand layouts the tcgen05 kernel uses.
- * One CTA stages A (row-major [M][K] fp32, device) and B (row-major [K][N] fp32, device) as bf16 in shared
- * memory in the layout selected by `mode` (0: A K-major 128x128, B K-major, N=64; 1: A MN-major 128x64,
- * B K-major, N=64; 2: A K-major 128x64, B MN-major, N=128; 3: A K-major 128x128, B MN-major, N=64; 4: A
- * 128x64 in tensor memory, B K-major, N=64), runs
- * the MMA k-step loop, and writes D = A B (fp32, row-major [M][N], device).  Asynchronous on `stream`. */
+/* Diagnostic (no counterpart on the pages): checks the tensor-core operand layouts the tcgen05 kernels use.
+ * One CTA stages A (row-major [M][K] fp32, device) and B (row-major [K][N] fp32, device) in shared or tensor
+ * memory in the layout selected by `mode` -- bf16 operands: 0: A K-major 128x128, B K-major, N=64; 1: A
+ * MN-major 128x64, B K-major, N=64; 2: A K-major 128x64, B MN-major, N=128; 3: A K-major 128x128, B
+ * MN-major, N=64; 4: A 128x64 in tensor memory, B K-major, N=64; tf32 operands (fp32 storage): 5: A 128x32
+ * in tensor memory, B K-major, N=64 -- runs the MMA k-step loop, and writes D = A B (fp32, row-major
+ * [M][N], device).  Mode outside 0..5: GDN_ERR_INVALID_ARG.
+ * Asynchronous on `stream`. */
 gdn_status gdn_debug_umma_selftest(const float* A, const float* B, float* D, int mode, cudaStream_t stream);
 
 /* Per-kernel device timing, a measurement aid (off by default; process-wide).  While enabled, every kernel

@@ -27,7 +27,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["gdn_chunk_fwd", "gdn2_chunk_fwd", "gdn_workspace_bytes", "gdn_check_error", "gdn_status_string",
-              "gdn_last_error", "gdn_set_kernel", "gdn_last_kernel", "gdn_debug_umma_selftest"]:
+              "gdn_last_error", "gdn_set_kernel", "gdn_last_kernel", "gdn_debug_umma_selftest",
+              "gdn_chunk_fwd_noalloc", "gdn_profile_enable", "gdn_profile_take"]:
         assert n in names
 
 
@@ -103,3 +104,20 @@ def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(1, 4, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         gdn_chunk_fwd(q, q, q, torch.zeros(1, 4, 1), torch.zeros(1, 4, 1))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(q=A + 8), 1), (dict(B=0), 1), (dict(BT=32), 2), (dict(dk=96), 2), (dict(dv=320), 2),
+    (dict(dt=7), 2), (dict(scale=float("nan")), 1), (dict(cu=A, B=2, n_seqs=2), 1), (dict(n_seqs=3), 1),
+])
+def test_noalloc_entry_checks_arguments_before_touching_the_device(lib, kw, status):
+    args = dict(q=A, k=A, v=A, g=A, beta=A, scale=0.125, h0=None, o=A, hT=None, B=1, T=64, H=1, dk=64, dv=64,
+                BT=64, dt=1, odt=0, cu=None, n_seqs=0)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    st = lib.gdn_chunk_fwd_noalloc(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]), vp(args["beta"]),
+                                   args["scale"], vp(args["h0"]), vp(args["o"]), vp(args["hT"]), args["B"], args["T"],
+                                   args["H"], args["dk"], args["dv"], args["BT"], args["dt"], args["odt"],
+                                   vp(args["cu"]), args["n_seqs"], None)
+    assert st == status
+    assert lib.gdn_last_error().decode() != ""
