@@ -21,7 +21,7 @@
 // accumulator in TMEM.
 // Precision: every bf16 operand whose rounding would reach the output at the bf16-ulp level is avoided or
 // split.  U diag f (in TMEM, as the A operand of the h^T MMA) and T'' are bf16 hi + lo pairs; the read-out
-// product U^T P^T runs on kind::tf32 with U in fp32 straight from TMEM and P stored as tf32; 2^G_r is
+// product U^T P^T runs on kind::tf32 with U rounded to tf32 in TMEM and P stored as tf32; 2^G_r is
 // applied to the fp32 accumulator of h^T Q^T instead of to Q.  The remaining bf16 operands are h^T, W^T,
 // T' and the inputs themselves.
 // The operands T', T'' and P are lower triangular: the MMAs that read them skip the blocks above the
@@ -508,6 +508,7 @@ enum TcBar : int {
     B_TW_EMPTY = 30,   // [2] U^T MMA reading T'' done
     B_P_READY = 32,    // [2] P written (64)
     B_OS_FREE = 34,    // output staging rows 32-63 stored
+    B_U_RND = 35,      // U in TMEM rounded to tf32 in place, for the O2 MMA (256)
 };
 
 // TMEM columns.  U^T is accumulated in fp32 at TM_U and read there, as tf32, by the O2 MMA; the state
@@ -571,7 +572,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (tid == 0) {
         for (int b = 0; b < (int)L::N_BARS; ++b) {
             uint32_t cnt = 1;
-            if (b == B_U_CONV || b == B_H_READY || b == B_HM_READY) cnt = 256;
+            if (b == B_U_CONV || b == B_U_RND || b == B_H_READY || b == B_HM_READY) cnt = 256;
             if (b == B_PREP || b == B_PREP + 1 || b == B_O_FREE || b == B_O_STAGED) cnt = 128;
             if (b == B_S1_FREE || b == B_P_READY || b == B_P_READY + 1) cnt = 64;
             mbar_init(&bars[b], cnt);
@@ -754,6 +755,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 umma_commit(&bars[B_H_FULL]);
                 if (!mbar_wait(&bars[B_P_READY + st], (c >> 1) & 1, abort_flag, err)) break;
+                if (!mbar_wait(&bars[B_U_RND], c & 1, abort_flag, err)) break;
                 tc_fence_after();
                 // O2^T = U^T P^T on kind::tf32: U fp32 straight from TM_U, P fp32 (tokens 0-31 in PH, 32-63 in
                 // PL); k-step ks8 covers 8 tokens and, P being lower triangular, only columns r >= 16 (ks8 / 2)
@@ -916,7 +918,8 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int c = 0; c < nc; ++c) {
             const TcGate& gs = gates[c & 3];
             // ---- U diag f (values [32 half, 32 half + 32)) as bf16 hi/lo pairs for the h^T MMA, to TM_UF
-            // ([hi | lo], 16 columns each per half).  U itself stays fp32 in TM_U: the O2 MMA reads it as tf32.
+            // ([hi | lo], 16 columns each per half); then U itself, rounded to tf32, back into TM_U for the
+            // kind::tf32 O2 MMA.
             if (!warp_wait(&bars[B_U_FULL], c & 1, abort_flag, err)) break;
             if (!warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err)) break;
             tc_fence_after();
@@ -932,10 +935,18 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 tmem_st16u(taddr(tmem, lane_base, TM_UF + 32 * half), hi);
                 tmem_st16u(taddr(tmem, lane_base, TM_UF + 32 * half + 16), lo);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars[B_U_CONV]);
+                // U back in place rounded to tf32: the tensor core would otherwise truncate the fp32 value
+                uint32_t ur[32];
+#pragma unroll
+                for (int q = 0; q < 32; ++q) ur[q] = f2tf32(u[q]);
+                tmem_st32u(taddr(tmem, lane_base, TM_U + 32 * half), ur);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars[B_U_CONV]);
+            mbar_arrive(&bars[B_U_RND]);
             // ---- state refresh (key channels of this half)
             if (!warp_wait(&bars[B_H_FULL], c & 1, abort_flag, err)) break;
             const bool last = c + 1 == nc;
