@@ -675,7 +675,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (c >= 1 && !mbar_wait(&bars[B_S1_FREE], (c - 1) & 1, abort_flag, err)) break;
                 tc_fence_after();
                 const uint64_t d = desc_k_sw128(sbase + L::KQ + st * L::KQ_STAGE);
-#pragma unroll 1
+#pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t a = d + (kk >> 2) * 1024 + (kk & 3) * 2;
                     umma_bf16(tmem + TM_S1, a, a, id_s1, kk > 0);
@@ -687,7 +687,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc_fence_after();
                 const uint64_t da = desc_mn_sw128(sbase + L::KQ + st * L::KQ_STAGE, 16384);
                 // k-step kk (tokens s in [16 kk, 16 kk + 16)) reaches only the rows r >= 16 kk of T'
-#pragma unroll 1
+#pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16(tmem + TM_W + 16 * kk, da + kk * 128, d_tp + kk * 130, id_w - kk * n16, kk > 0);
                 umma_commit(&bars[B_W_FULL]);
@@ -698,7 +698,8 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         __syncwarp();
     } else if (warp == 2) {
         // ================================================================ serial MMAs (U^T, O^T, h^T)
-        // The k-step loops stay rolled (short code); descriptors advance by byte offset >> 4.
+        // The k-step loops are unrolled: issuing a tcgen05.mma from a rolled loop with run-time descriptor
+        // arithmetic measured ~2x slower, and these issues are on the chunk loop's critical path.
         if (lane == 0) {
             const uint32_t id_u1 = idesc_bf16(128, 64, true, false);
             const uint32_t id_u2 = idesc_bf16(128, 64, false, true);
@@ -719,7 +720,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 // U^T = V^T (T''_hi + T''_lo)^T - h^T W^T ; the first half does not need the state.  As T'' is
                 // lower triangular, k-step ks (tokens s in [16 ks, 16 ks + 16)) updates only columns r >= 16 ks.
                 const uint64_t d_t = desc_k_sw128(sbase + L::TW + st * 16384);
-#pragma unroll 1
+#pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const int ks = kk & 3;
                     umma_bf16(tmem + TM_U + 16 * ks, d_v + ks * 128, d_t + (kk >> 2) * 512 + ks * 130,
@@ -728,7 +729,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 umma_commit(&bars[B_TW_EMPTY + st]);
                 if (!mbar_wait(&bars[B_H_READY], c & 1, abort_flag, err)) break;
                 tc_fence_after();
-#pragma unroll 1
+#pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma_bf16(tmem + TM_U, d_ht + (kk >> 2) * 1024 + (kk & 3) * 2, d_wt + kk * 128, id_u2, 1);
                 umma_commit(&bars[B_U_FULL]);
@@ -737,7 +738,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (c >= 1 && !mbar_wait(&bars[B_O_FREE], (c - 1) & 1, abort_flag, err)) break;
                 tc_fence_after();
                 const uint64_t d_q = desc_k_sw128(kq + 8192);
-#pragma unroll 1
+#pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t o = (kk >> 2) * 1024 + (kk & 3) * 2;
                     umma_bf16(tmem + TM_O1, d_ht + o, d_q + o, id_o, kk > 0);
@@ -747,7 +748,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (!mbar_wait(&bars[B_HM_READY], c & 1, abort_flag, err)) break;
                 tc_fence_after();
                 const uint64_t d_k = desc_mn_sw128(kq, 16384);
-#pragma unroll 1
+#pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {  // kk < 4: hi, else lo; s-step ks covers values 16 ks .. 16 ks + 15
                     const int ks = kk & 3;
                     const uint32_t a = tmem + TM_UF + (ks >> 1) * 32 + (kk >> 2) * 16 + (ks & 1) * 8;
@@ -759,7 +760,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc_fence_after();
                 // O2^T = U^T P^T on kind::tf32: U fp32 straight from TM_U, P fp32 (tokens 0-31 in PH, 32-63 in
                 // PL); k-step ks8 covers 8 tokens and, P being lower triangular, only columns r >= 16 (ks8 / 2)
-#pragma unroll 1
+#pragma unroll
                 for (int ks8 = 0; ks8 < 8; ++ks8) {
                     const int r0 = 16 * (ks8 >> 1);
                     const uint64_t b = desc_k_sw128(sbase + ((ks8 & 4) ? L::PL : L::PH) + st * 8192) +
