@@ -466,16 +466,16 @@ struct TcSmem {
     static constexpr uint32_t KQ = 0;  // 2 stages x [K ch0-63 | Q ch0-63 | K ch64-127 | Q ch64-127], 8 KB each
     static constexpr uint32_t KQ_STAGE = 32768;
     static constexpr uint32_t V = KQ + 2 * KQ_STAGE;  // V tile: j 0-63 | j 64-127, 8 KB each (MN-major A)
-    static constexpr uint32_t TW = V + 16384;         // 2 stages x [T''_hi | T''_lo], [r][s] K-major, 8 KB each
-    static constexpr uint32_t TP = TW + 32768;        // T': [r][s] K-major, 8 KB
-    static constexpr uint32_t PH = TP + 8192;         // P hi [2]: [r][s] K-major, 8 KB each
-    static constexpr uint32_t PL = PH + 16384;        // P lo [2]
+    static constexpr uint32_t TW = V + 16384;         // [T''_hi | T''_lo], [r][s] K-major, 8 KB each
+    static constexpr uint32_t TP = TW + 16384;        // T': [r][s] K-major, 8 KB
+    static constexpr uint32_t PH = TP + 8192;         // P, tokens 0-31 [2]: [r][s] K-major fp32, 8 KB each
+    static constexpr uint32_t PL = PH + 16384;        // P, tokens 32-63 [2]
     static constexpr uint32_t WT = PL + 16384;        // -W^T: lines i (128) x 64 r, MN-major B, 16 KB
-    static constexpr uint32_t HT = WT + 16384;        // h^T bf16: [j][i] K-major, panels i 0-63 | 64-127, 16 KB each
-    static constexpr uint32_t OS = HT + 32768;        // output staging, rows 32-63: 2 x [16][128]
-    static constexpr uint32_t GATE = OS + 16384;      // 4 x TcGate
+    static constexpr uint32_t HT = WT + 16384;        // h^T bf16 [2]: [j][i] K-major, panels i 0-63 | 64-127
+    static constexpr uint32_t HT_STAGE = 32768;
+    static constexpr uint32_t GATE = HT + 2 * HT_STAGE;  // 4 x TcGate
     static constexpr uint32_t BARS = GATE + 4 * sizeof(TcGate);
-    static constexpr uint32_t N_BARS = 40;
+    static constexpr uint32_t N_BARS = 28;
     static constexpr uint32_t MISC = BARS + 8 * N_BARS;  // tmem base, abort flag
     static constexpr uint32_t END = MISC + 64;
     static constexpr uint32_t ALLOC = END + 1024;  // slack for the 1024-byte alignment of the base
@@ -486,29 +486,24 @@ static_assert(TcSmem::ALLOC <= 232448, "shared memory budget");
 enum TcBar : int {
     B_KQ_FULL = 0,     // [2] TMA K/Q landed (tx)
     B_KQ_EMPTY = 2,    // [2] serial MMAs of the stage's chunk done
-    B_V_FULL = 4,      // V landed (tx)
-    B_V_EMPTY = 5,     // U^T MMA reading V done
+    B_VT_FULL = 4,     // V, T''_hi, T''_lo landed (tx)
+    B_VT_EMPTY = 5,    // U^T MMA reading V and T'' done
     B_GATE = 6,        // [4] gate stage written
     B_S1_FULL = 10,    // S1 in TMEM
     B_S1_FREE = 11,    // P rows read S1 (64)
     B_TP_FULL = 12,    // T' landed (tx)
     B_W_FULL = 13,     // W^T in TMEM (and T' read)
     B_PREP = 14,       // [2] -W^T written (128)
-    B_P_FREE = 16,     // [2] P stage free: O^T MMA done and the output rows staged there stored
+    B_P_READY = 16,    // [2] P written (64)
     B_U_FULL = 18,     // U^T in TMEM (and -W^T no longer read)
     B_U_CONV = 19,     // U, U.f split into bf16 hi/lo in TMEM (256)
     B_H_FULL = 20,     // h^T MMA done
-    B_H_READY = 21,    // bf16 h^T staged in shared memory (256)
+    B_H_READY = 21,    // bf16 h^T of the next chunk staged in shared memory (256)
     B_O_FULL = 22,     // O^T MMAs done
     B_O_FREE = 23,     // O^T TMEM read (128)
     B_DRAIN = 24,      // [2] final commit of each MMA issuer
     B_HM_READY = 26,   // fp32 state in TMEM re-scaled by the next chunk's decay (256)
-    B_O_STAGED = 27,   // output tile staged in shared memory (128)
-    B_TW_FULL = 28,    // [2] T''_hi, T''_lo landed (tx)
-    B_TW_EMPTY = 30,   // [2] U^T MMA reading T'' done
-    B_P_READY = 32,    // [2] P written (64)
-    B_OS_FREE = 34,    // output staging rows 32-63 stored
-    B_U_RND = 35,      // U in TMEM rounded to tf32 in place, for the O2 MMA (256)
+    B_U_RND = 27,      // U in TMEM rounded to tf32 in place, for the O2 MMA (256)
 };
 
 // TMEM columns.  U^T is accumulated in fp32 at TM_U and read there, as tf32, by the O2 MMA; the state
@@ -517,14 +512,14 @@ constexpr uint32_t TM_S1 = 0, TM_W = 64, TM_U = 128, TM_UF = 192, TM_O1 = 256, T
                    TM_COLS = 512;
 
 // Warp roles (16 warps): 0 TMA producer (K, Q, V, T', T'') and gates; 1 issues S1 and W^T; 2 issues the
-// serial MMAs (U^T, O^T, h^T); 3 stores the output tiles by TMA; 4-7 (prep / output warpgroup) stage o,
-// write -W^T and, in quadrants 2-3, P; 8-11 and 12-15 (state warpgroups, one per half of U and of the key
-// channels) split U into bf16 operands, refresh the bf16 copy of h^T, re-scale the fp32 state by the next
-// chunk's decay and write hT.
+// serial MMAs (U^T, h^T, O^T); 3 idle; 4-7 (prep / output warpgroup) write -W^T, in quadrants 2-3 P, and
+// store o; 8-11 and 12-15 (state warpgroups, one per half of U and of the key channels) split U into bf16
+// operands, refresh the bf16 copy of h^T (double-buffered), re-scale the fp32 state by the next chunk's
+// decay and write hT.
 template <bool O_F32>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const FwdParams p,
+                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p,
                   const uint8_t* ws, unsigned* err) {
     using namespace sm100;
     using L = TcSmem;
@@ -573,7 +568,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int b = 0; b < (int)L::N_BARS; ++b) {
             uint32_t cnt = 1;
             if (b == B_U_CONV || b == B_U_RND || b == B_H_READY || b == B_HM_READY) cnt = 256;
-            if (b == B_PREP || b == B_PREP + 1 || b == B_O_FREE || b == B_O_STAGED) cnt = 128;
+            if (b == B_PREP || b == B_PREP + 1 || b == B_O_FREE) cnt = 128;
             if (b == B_S1_FREE || b == B_P_READY || b == B_P_READY + 1) cnt = 64;
             mbar_init(&bars[b], cnt);
         }
@@ -582,7 +577,6 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
-        prefetch_tensormap(&tm_o);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, TM_COLS);
@@ -596,7 +590,6 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     if (warp == 0) {
         // ================================================================ producer: TMA, bulk copies, gates
-        int kq_issued[2] = {0, 0}, tw_issued[2] = {0, 0}, v_issued = 0, tp_issued = 0;
         auto prefetch = [&](int c) {  // L2 prefetch of a later chunk, so the load issued later hits L2
             if (lane == 0 && c < nc) {
                 const int tok = (int)(seq_start + c * kChunk);
@@ -609,8 +602,9 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 bulk_prefetch_l2(wy_unit(c), kWyUnit);
             }
         };
-        // iteration c: T' of chunk c + 1 (once W^T of chunk c is done with it), V of chunk c + 1, T'' and
-        // K/Q (+ gates) of chunk c + 2; the iterations before 0 fill the stages
+        // iteration c: T' of chunk c + 1 (once W^T of chunk c is done with it), V and T'' of chunk c + 1 (once
+        // the U^T MMA of chunk c is), K/Q (+ gates) of chunk c + 2; the iterations before 0 fill the stages
+        int kq_issued[2] = {0, 0}, vt_issued = 0, tp_issued = 0;
         for (int c = -2; c < nc; ++c) {
             const int c1 = c + 1, c2 = c + 2;
             if (c1 >= 0 && c1 < nc) {
@@ -620,23 +614,18 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     bulk_load(sm + L::TP, wy_unit(c1), 8192, &bars[B_TP_FULL]);
                 }
                 tp_issued++;
-                if (c >= 0 && !warp_wait(&bars[B_V_EMPTY], c & 1, abort_flag, err)) break;
+                if (c >= 0 && !warp_wait(&bars[B_VT_EMPTY], c & 1, abort_flag, err)) break;
                 if (lane == 0) {
                     const int tok = (int)(seq_start + c1 * kChunk);
-                    mbar_expect_tx(&bars[B_V_FULL], 16384);
-                    tma_load_3d(sm + L::V, &tm_v, &bars[B_V_FULL], j0, h, tok);
-                    tma_load_3d(sm + L::V + 8192, &tm_v, &bars[B_V_FULL], j0 + 64, h, tok);
+                    mbar_expect_tx(&bars[B_VT_FULL], 32768);
+                    tma_load_3d(sm + L::V, &tm_v, &bars[B_VT_FULL], j0, h, tok);
+                    tma_load_3d(sm + L::V + 8192, &tm_v, &bars[B_VT_FULL], j0 + 64, h, tok);
+                    bulk_load(sm + L::TW, wy_unit(c1) + 8192, 16384, &bars[B_VT_FULL]);
                 }
-                v_issued++;
+                vt_issued++;
             }
             if (c2 < nc) {
                 const int st = c2 & 1;
-                if (c >= 0 && !warp_wait(&bars[B_TW_EMPTY + st], (c >> 1) & 1, abort_flag, err)) break;
-                if (lane == 0) {
-                    mbar_expect_tx(&bars[B_TW_FULL + st], 16384);
-                    bulk_load(sm + L::TW + st * 16384, wy_unit(c2) + 8192, 16384, &bars[B_TW_FULL + st]);
-                }
-                tw_issued[st]++;
                 if (c >= 0 && !warp_wait(&bars[B_KQ_EMPTY + st], (c >> 1) & 1, abort_flag, err)) break;
                 if (lane == 0) {
                     uint8_t* dst = sm + L::KQ + st * L::KQ_STAGE;
@@ -656,11 +645,9 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         }
         // drain: wait for every load this warp issued before the CTA may exit
-        for (int st = 0; st < 2; ++st) {
+        for (int st = 0; st < 2; ++st)
             if (kq_issued[st] > 0) drain_wait(&bars[B_KQ_FULL + st], (kq_issued[st] - 1) & 1);
-            if (tw_issued[st] > 0) drain_wait(&bars[B_TW_FULL + st], (tw_issued[st] - 1) & 1);
-        }
-        if (v_issued > 0) drain_wait(&bars[B_V_FULL], (v_issued - 1) & 1);
+        if (vt_issued > 0) drain_wait(&bars[B_VT_FULL], (vt_issued - 1) & 1);
         if (tp_issued > 0) drain_wait(&bars[B_TP_FULL], (tp_issued - 1) & 1);
     } else if (warp == 1) {
         // ================================================================ S1 = [K; Q] K^T and W^T = K^T T'^T
@@ -697,9 +684,12 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         __syncwarp();
     } else if (warp == 2) {
-        // ================================================================ serial MMAs (U^T, O^T, h^T)
+        // ================================================================ serial MMAs (U^T, h^T, O^T)
         // The k-step loops are unrolled: issuing a tcgen05.mma from a rolled loop with run-time descriptor
-        // arithmetic measured ~2x slower, and these issues are on the chunk loop's critical path.
+        // arithmetic measured ~2x slower, and these issues are on the chunk loop's critical path.  Per chunk
+        // the order is U^T (state-free half), U^T (state half), h^T, then the two O^T products: the h^T MMA
+        // goes as soon as U diag f is split, and the O^T products (which read the bf16 h^T of this chunk
+        // from its own buffer) fill the time the state warpgroups take to stage the next h^T.
         if (lane == 0) {
             const uint32_t id_u1 = idesc_bf16(128, 64, true, false);
             const uint32_t id_u2 = idesc_bf16(128, 64, false, true);
@@ -708,42 +698,31 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint32_t id_o2 = idesc_tf32(128, 64, false, false);
             const uint32_t n16 = 2u << 17;
             const uint64_t d_v = desc_mn_sw128(sbase + L::V, 8192);
-            const uint64_t d_ht = desc_k_sw128(sbase + L::HT);
+            const uint64_t d_t = desc_k_sw128(sbase + L::TW);
             const uint64_t d_wt = desc_mn_sw128(sbase + L::WT, 8192);
             for (int c = 0; c < nc; ++c) {
                 const int st = c & 1;
                 const uint32_t kq = sbase + L::KQ + st * L::KQ_STAGE;
-                if (!mbar_wait(&bars[B_PREP + st], (c >> 1) & 1, abort_flag, err)) break;
-                if (!mbar_wait(&bars[B_V_FULL], c & 1, abort_flag, err)) break;
-                if (!mbar_wait(&bars[B_TW_FULL + st], (c >> 1) & 1, abort_flag, err)) break;
+                const uint64_t d_ht = desc_k_sw128(sbase + L::HT + st * L::HT_STAGE);
+                if (!mbar_wait(&bars[B_VT_FULL], c & 1, abort_flag, err)) break;
                 tc_fence_after();
                 // U^T = V^T (T''_hi + T''_lo)^T - h^T W^T ; the first half does not need the state.  As T'' is
                 // lower triangular, k-step ks (tokens s in [16 ks, 16 ks + 16)) updates only columns r >= 16 ks.
-                const uint64_t d_t = desc_k_sw128(sbase + L::TW + st * 16384);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const int ks = kk & 3;
                     umma_bf16(tmem + TM_U + 16 * ks, d_v + ks * 128, d_t + (kk >> 2) * 512 + ks * 130,
                               id_u1 - ks * n16, kk > 0);
                 }
-                umma_commit(&bars[B_TW_EMPTY + st]);
+                umma_commit(&bars[B_VT_EMPTY]);
+                if (!mbar_wait(&bars[B_PREP + st], (c >> 1) & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[B_H_READY], c & 1, abort_flag, err)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma_bf16(tmem + TM_U, d_ht + (kk >> 2) * 1024 + (kk & 3) * 2, d_wt + kk * 128, id_u2, 1);
                 umma_commit(&bars[B_U_FULL]);
-                umma_commit(&bars[B_V_EMPTY]);
-                // O1^T = h^T Q^T (scaled by 2^G_r in the epilogue)
-                if (c >= 1 && !mbar_wait(&bars[B_O_FREE], (c - 1) & 1, abort_flag, err)) break;
-                tc_fence_after();
-                const uint64_t d_q = desc_k_sw128(kq + 8192);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t o = (kk >> 2) * 1024 + (kk & 3) * 2;
-                    umma_bf16(tmem + TM_O1, d_ht + o, d_q + o, id_o, kk > 0);
-                }
-                // h^T += (U diag f)^T K  (hi and lo halves) ;  O2^T = U^T P^T  (hi*hi + hi*lo + lo*hi)
+                // h^T += (U diag f)^T K  (hi and lo halves)
                 if (!mbar_wait(&bars[B_U_CONV], c & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[B_HM_READY], c & 1, abort_flag, err)) break;
                 tc_fence_after();
@@ -755,6 +734,15 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     umma_bf16_tmem_a(tmem + TM_H, a, d_k + ks * 128, id_h, 1);
                 }
                 umma_commit(&bars[B_H_FULL]);
+                // O1^T = h^T Q^T (scaled by 2^G_r in the epilogue)
+                if (c >= 1 && !mbar_wait(&bars[B_O_FREE], (c - 1) & 1, abort_flag, err)) break;
+                tc_fence_after();
+                const uint64_t d_q = desc_k_sw128(kq + 8192);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t o = (kk >> 2) * 1024 + (kk & 3) * 2;
+                    umma_bf16(tmem + TM_O1, d_ht + o, d_q + o, id_o, kk > 0);
+                }
                 if (!mbar_wait(&bars[B_P_READY + st], (c >> 1) & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[B_U_RND], c & 1, abort_flag, err)) break;
                 tc_fence_after();
@@ -775,46 +763,51 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         __syncwarp();
     } else if (warp == 3) {
-        // ================================================================ output stores
-        // A full chunk's o tile is staged by the prep / output warpgroup, rows 0-31 in the P buffers of its
-        // stage (free once its O^T MMAs are done), rows 32-63 in OS, and leaves by TMA; a partial chunk is
-        // written directly by that warpgroup.
-        if (lane == 0) {
-            for (int c = 0; c < nc; ++c) {
-                const int st = c & 1;
-                if (!mbar_wait(&bars[B_O_STAGED], c & 1, abort_flag, err)) break;
-                if (eos - bos - c * kChunk >= kChunk) {
-                    const int tok0 = (int)(seq_start + c * kChunk);
-                    tma_store_3d(&tm_o, sm + L::PH + st * 8192, j0, h, tok0);
-                    tma_store_3d(&tm_o, sm + L::PL + st * 8192, j0, h, tok0 + 16);
-                    tma_store_3d(&tm_o, sm + L::OS, j0, h, tok0 + 32);
-                    tma_store_3d(&tm_o, sm + L::OS + 8192, j0, h, tok0 + 48);
-                    bulk_commit();
-                    bulk_wait_read_all();
-                }
-                mbar_arrive(&bars[B_P_FREE + st]);
-                mbar_arrive(&bars[B_OS_FREE]);
-            }
-            bulk_wait_all();
-        }
-        __syncwarp();
+        // idle: its TMEM lane quadrant is served by warps 7, 11 and 15
     } else if (warp < 8) {
         // ================================================================ prep / output warpgroup
-        // Iteration k: (1) the output tile of chunk k - 2 (its O^T MMAs are done by the time chunk k - 1's
-        // U^T is), read from TMEM first so the next O^T MMAs can start, then staged for the TMA store: rows
-        // 0-31 in the P buffers of its stage, rows 32-63 in OS; a partial chunk is written directly.
-        // (2) -W^T of chunk k, line i = t, from TMEM into shared memory.  (3) The P rows of chunk k (the
-        // quadrant-2/3 warps, whose TMEM lanes hold Q K^T).  The warps run independently; a timed-out wait
-        // does not break out, the warp finishes the iteration and leaves at the top of the next.
+        // Iteration k: (1) -W^T of chunk k, line i = t, from TMEM into shared memory.  (2) The P rows of
+        // chunk k (the quadrant-2/3 warps, whose TMEM lanes hold Q K^T).  (3) The output tile of chunk k - 1:
+        // O1^T and O2^T read from TMEM (then released for the next chunk's O^T MMAs), combined and stored
+        // to global memory, one token row per store (a warp writes 32 consecutive values of the row).  The
+        // warps run independently; a timed-out wait does not break out, the warp finishes the iteration
+        // and leaves at the top of the next.
         const int t = tid - 128;  // TMEM lane: value column j of O^T / line of W^T / row of S1
         const int wid = warp & 3;
         const uint32_t lane_base = 32 * wid;
-        for (int k = 0; k < nc + 2; ++k) {
+        for (int k = 0; k <= nc; ++k) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            if (k >= 2) {
-                const int c = k - 2, st = c & 1;
+            if (k < nc) {
+                const int c = k, st = c & 1;
+                warp_wait(&bars[B_W_FULL], c & 1, abort_flag, err);
+                if (c >= 1) warp_wait(&bars[B_U_FULL], (c - 1) & 1, abort_flag, err);
+                tc_fence_after();
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    tmem_ld32(taddr(tmem, lane_base, TM_W + 32 * half), v);
+                    tmem_wait_ld();
+                    st_half_line_bf16(sm + L::WT, t, 4 * half, v, -1.f);
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                mbar_arrive(&bars[B_PREP + st]);
+                if (wid >= 2) {
+                    warp_wait(&bars[B_S1_FULL], c & 1, abort_flag, err);
+                    warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err);
+                    tc_fence_after();
+                    // rows 0-31 need columns 0-31 only: the O^T MMA never reads the blocks above the diagonal
+                    tc_row_pass<false>(taddr(tmem, lane_base, TM_S1), gates[c & 3], t - 64, 0, wid == 2 ? 31 : 63,
+                                       nullptr, sm + L::PH + st * 8192, sm + L::PL + st * 8192);
+                    fence_proxy_async();
+                    mbar_arrive(&bars[B_P_READY + st]);
+                    tc_fence_before();
+                    mbar_arrive(&bars[B_S1_FREE]);
+                }
+            }
+            if (k >= 1) {
+                const int c = k - 1;
                 warp_wait(&bars[B_O_FULL], c & 1, abort_flag, err);
-                if (c >= 1) warp_wait(&bars[B_OS_FREE], (c - 1) & 1, abort_flag, err);
                 tc_fence_after();
                 const TcGate& gs = gates[c & 3];
                 const int Lc = gs.L;
@@ -822,68 +815,28 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const size_t ostride = (size_t)H * dv;
                 size_t off = (tok0 * H + h) * (size_t)dv + j0 + t;
 #pragma unroll 1
-                for (int r32 = 0; r32 < 64; r32 += 32) {
-                    float v1[32], v2[32];
-                    tmem_ld32(taddr(tmem, lane_base, TM_O1 + r32), v1);
-                    tmem_ld32(taddr(tmem, lane_base, TM_O2 + r32), v2);
+                for (int r8 = 0; r8 < 64; r8 += 8) {
+                    float v1[8], v2[8];
+                    tmem_ld8(taddr(tmem, lane_base, TM_O1 + r8), v1);
+                    tmem_ld8(taddr(tmem, lane_base, TM_O2 + r8), v2);
                     tmem_wait_ld();
-                    if (r32 == 32) {
+                    if (r8 == 56) {
                         tc_fence_before();
                         mbar_arrive(&bars[B_O_FREE]);
                     }
-                    uint8_t* const stg0 = sm + (r32 ? L::OS : L::PH + st * 8192);
-                    uint8_t* const stg1 = sm + (r32 ? L::OS + 8192 : L::PL + st * 8192);
-                    const float4* eg4 = reinterpret_cast<const float4*>(gs.eG + r32);
+                    const float4 e0 = *reinterpret_cast<const float4*>(gs.eG + r8);
+                    const float4 e1 = *reinterpret_cast<const float4*>(gs.eG + r8 + 4);
+                    const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
-                        const float4 e = eg4[q4];
-                        const float ev[4] = {e.x, e.y, e.z, e.w};
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int q = 4 * q4 + u, r = r32 + q;
-                            const float val = p.scale * fmaf(ev[u], v1[q], v2[q]);
-                            uint8_t* stg = (q & 16) ? stg1 : stg0;
-                            if (Lc == kChunk) {  // staged for the TMA store: row r & 15 of a [16][128] box
-                                if (O_F32) reinterpret_cast<float*>(stg)[(r & 15) * kTcDV + t] = val;
-                                else reinterpret_cast<__nv_bfloat16*>(stg)[(r & 15) * kTcDV + t] = __float2bfloat16_rn(val);
-                            } else if (r < Lc) {
-                                if (O_F32) static_cast<float*>(p.o)[off] = val;
-                                else static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(val);
-                            }
-                            off += ostride;
+                    for (int q = 0; q < 8; ++q) {
+                        const float val = p.scale * fmaf(ev[q], v1[q], v2[q]);
+                        if (r8 + q < Lc) {
+                            if (O_F32) static_cast<float*>(p.o)[off] = val;
+                            else static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(val);
                         }
+                        off += ostride;
                     }
                 }
-                fence_proxy_async();
-                mbar_arrive(&bars[B_O_STAGED]);
-            }
-            if (k >= nc) continue;
-            const int c = k, st = c & 1;
-            warp_wait(&bars[B_W_FULL], c & 1, abort_flag, err);
-            if (c >= 1) warp_wait(&bars[B_U_FULL], (c - 1) & 1, abort_flag, err);
-            tc_fence_after();
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float v[32];
-                tmem_ld32(taddr(tmem, lane_base, TM_W + 32 * half), v);
-                tmem_wait_ld();
-                st_half_line_bf16(sm + L::WT, t, 4 * half, v, -1.f);
-            }
-            fence_proxy_async();
-            tc_fence_before();
-            mbar_arrive(&bars[B_PREP + st]);
-            if (wid >= 2) {
-                warp_wait(&bars[B_S1_FULL], c & 1, abort_flag, err);
-                warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err);
-                if (c >= 2) warp_wait(&bars[B_P_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err);
-                tc_fence_after();
-                // rows 0-31 need columns 0-31 only: the O^T MMA never reads the blocks above the diagonal
-                tc_row_pass<false>(taddr(tmem, lane_base, TM_S1), gates[c & 3], t - 64, 0, wid == 2 ? 31 : 63, nullptr,
-                                   sm + L::PH + st * 8192, sm + L::PL + st * 8192);
-                fence_proxy_async();
-                mbar_arrive(&bars[B_P_READY + st]);
-                tc_fence_before();
-                mbar_arrive(&bars[B_S1_FREE]);
             }
         }
     } else {
@@ -961,7 +914,8 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tmem_ld32(taddr(tmem, lane_base, TM_H + 32 * piece), v);
                 tmem_wait_ld();
                 if (!last) {
-                    st_half_line_bf16(sm + L::HT + (piece >> 1) * 16384, j, 4 * (piece & 1), v);
+                    st_half_line_bf16(sm + L::HT + ((c + 1) & 1) * L::HT_STAGE + (piece >> 1) * 16384, j,
+                                      4 * (piece & 1), v);
                 } else if (p.hT) {
                     float* hp = p.hT + state_base + (size_t)(32 * piece) * dv + j;
 #pragma unroll
@@ -1039,21 +993,6 @@ inline bool make_map(CUtensorMap* map, const void* base, int d, int H, long long
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map over the [rows, H, dv] output (fp32 or bf16), box 128 x 1 x 16 (one CTA's columns, 16 tokens),
-// no swizzle: the store source is a row-major [16][128] tile.
-inline bool make_out_map(CUtensorMap* map, void* base, int dv, int H, long long rows, bool f32) {
-    PFN_encodeTiled enc = get_encode_fn();
-    if (!enc) return false;
-    const cuuint64_t es = f32 ? 4 : 2;
-    const cuuint64_t dims[3] = {(cuuint64_t)dv, (cuuint64_t)H, (cuuint64_t)rows};
-    const cuuint64_t strides[2] = {(cuuint64_t)dv * es, (cuuint64_t)dv * H * es};
-    const cuuint32_t box[3] = {(cuuint32_t)kTcDV, 1, 16};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, void* ws, size_t ws_bytes, unsigned* err,
                             cudaStream_t stream) {
     if (gdn2) {
@@ -1065,10 +1004,10 @@ inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, void* ws,
         snprintf(t_tc_msg, sizeof(t_tc_msg), "the tcgen05 path needs %zu bytes of workspace (got %zu)", need, ws_bytes);
         return GDN_ERR_UNSUPPORTED;
     }
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv;
     const long long rows = (long long)p.B * p.T;
     if (!make_map(&mq, p.q, p.dk, p.H, rows) || !make_map(&mk, p.k, p.dk, p.H, rows) ||
-        !make_map(&mv, p.v, p.dv, p.H, rows) || !make_out_map(&mo, p.o, p.dv, p.H, rows, o_f32)) {
+        !make_map(&mv, p.v, p.dv, p.H, rows)) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "cuTensorMapEncodeTiled failed");
         return GDN_ERR_CUDA;
     }
@@ -1099,7 +1038,7 @@ inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, void* ws,
     }
     const unsigned grid = (unsigned)(p.dv / kTcDV) * p.H * p.n_seq;
     ProfScope prof_main(PK_TC_MAIN, stream);
-    kern<<<grid, kTcThreads, TcSmem::ALLOC, stream>>>(mq, mk, mv, mo, p, static_cast<const uint8_t*>(ws), err);
+    kern<<<grid, kTcThreads, TcSmem::ALLOC, stream>>>(mq, mk, mv, p, static_cast<const uint8_t*>(ws), err);
     prof_main.done();
     e = cudaGetLastError();
     if (e != cudaSuccess) {
