@@ -349,16 +349,16 @@ __device__ __forceinline__ bool tc_seq_bounds(const FwdParams& p, int n, int& ro
 // followed by 8 KB of other data: the T' and T''_hi emission areas.  T''_lo reuses the first K panel.
 struct WySmem {
     static constexpr uint32_t K0 = 0;        // K channels 0-63, [64 tokens][128 B] swizzled; then T''_lo
-    static constexpr uint32_t TP = 8192;     // T'
-    static constexpr uint32_t K1 = 16384;    // K channels 64-127
-    static constexpr uint32_t TPP = 24576;   // T''_hi
-    static constexpr uint32_t TPPL = K0;     // written by the inverse, once S1 has been computed from K
-    static constexpr uint32_t AS = 32768;    // A, then (I+A)^-1, fp32 [64][68]
+    static constexpr uint32_t K1 = 8192;     // K channels 64-127; then T'
+    static constexpr uint32_t TPP = 16384;   // T''_hi
+    static constexpr uint32_t TP = K1;       // T' and T''_lo are written by the inverse, once S1 has been
+    static constexpr uint32_t TPPL = K0;     // computed from K
+    static constexpr uint32_t AS = 24576;    // A, then (I+A)^-1, fp32 [64][68]
     static constexpr uint32_t GATE = AS + 64 * kAsLd * 4;
     static constexpr uint32_t BARS = GATE + sizeof(TcGate);  // [0] K landed, [1] S1 done
     static constexpr uint32_t MISC = BARS + 16;              // tmem base, abort flag, unit info
     static constexpr uint32_t END = MISC + 64;
-    static constexpr uint32_t ALLOC = END + 1024;  // 4 CTAs per SM
+    static constexpr uint32_t ALLOC = END + 1024;  // 5 CTAs per SM
 };
 
 // One CTA per (workspace slot, head): finds the (sequence, chunk) of its slot, builds A, inverts I + A and
@@ -422,14 +422,15 @@ __global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     if (tid == 0) {
-        // S1 = K K^T (rows 64-127 of the A operand are other data; their results are never read)
+        // S1 = K K^T (rows 64-127 of the A operand are the next 8 KB, other data; their results are never
+        // read): k-steps 0-3 read channel panel K0, 4-7 panel K1, 8 KB further
         if (mbar_wait(&bars[0], 0, abort_flag, err)) {
             tc_fence_after();
             const uint64_t d = desc_k_sw128(smem_u32(sm));
             const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll 1
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t a = d + (kk >> 2) * 1024 + (kk & 3) * 2;
+                const uint64_t a = d + (kk >> 2) * 512 + (kk & 3) * 2;
                 umma_bf16(tmem, a, a, id, kk > 0);
             }
             umma_commit(&bars[1]);
