@@ -86,7 +86,7 @@ static gdn_status check_common(const void* q, const void* k, const void* v, cons
 template <typename TIn, typename TOut, int DK, bool GDN2>
 static gdn_status launch_simt_dk(const FwdParams& p, unsigned* err, cudaStream_t stream) {
     constexpr int DVT = SimtDVT<GDN2>::value;
-    using L = SimtSmem<DK, DVT, GDN2>;
+    using L = SimtSmem<DK, DVT, GDN2, sizeof(typename SimtGate<TIn>::type) / 4>;
     auto kern = gdn_simt_fwd_kernel<TIn, TOut, DK, DVT, GDN2>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));

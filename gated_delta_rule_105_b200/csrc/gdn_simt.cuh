@@ -10,12 +10,14 @@
 // Per chunk (rows r, s < 64; zero rows pad a partial chunk, which makes them inert: k = v = 0,
 // beta = b = w = 0 and g = 0 so the padded cumulative gate stays at the last real token's value):
 //   G_r   = log2(e) * sum_{s<=r} g_s                           (GDN-2: per key channel)
-// G is accumulated and differenced in fp64: with strong decay |G| reaches ~10^3 inside a chunk, where an
-// fp32 cumsum loses ~1e-4 absolute in G_r - G_s for nearby r, s -- as much as the whole fp32 error
-// budget.  Only the (small) differences are rounded to fp32 before exp2.
+// For fp32 inputs G is accumulated and differenced in fp64: with strong decay |G| reaches ~10^3 inside a
+// chunk, where an fp32 cumsum loses ~1e-4 absolute in G_r - G_s for nearby r, s -- as much as the whole
+// fp32 error budget; only the (small) differences are rounded to fp32 before exp2.  For bf16 inputs
+// (a 2e-2 budget) the per-channel GDN-2 gate is kept in fp32, which halves its shared-memory traffic.
 //   A_rs  = beta_r (k_r . k_s) 2^(G_r - G_s)        s < r      (GDN-2: sum_i b_ri k_ri k_si 2^(G_ri - G_si))
 //   P_rs  = (q_r . k_s) 2^(G_r - G_s)               s <= r     (GDN-2: per-channel factor inside the sum)
-//   Tm    = (I + A)^-1                               forward substitution, one column per thread
+//   Tm    = (I + A)^-1                               forward substitution row by row, each row's sums
+//                                                    split over four threads per column
 //   X     = beta V - diag(beta 2^G) K h              (GDN-2: w.V - (b.2^G.K) h)
 //   U     = Tm X
 //   O     = scale [ (Q . 2^G) h + P U ]
@@ -34,13 +36,13 @@ constexpr int kSimtThreads = 256;
 template <bool GDN2> struct SimtDVT { static constexpr int value = GDN2 ? 16 : 32; };
 
 // Shared-memory map in 4-byte words.  The fp64 gate block comes first so it is 8-byte aligned.
-template <int DK, int DVT, bool GDN2>
-struct SimtSmem {
+template <int DK, int DVT, bool GDN2, int GW = 2>
+struct SimtSmem {  // GW: 4-byte words per cumulative-gate element (2: fp64, 1: fp32)
     static constexpr int LDK = DK + 1;  // padded row stride: conflict-free column walks
     static constexpr int LDT = kChunk + 1;
     static constexpr int nK = kChunk * LDK;
-    static constexpr int oGd = 0;                              // fp64 cumulative gate: GDN-2 [64][LDK], GDN [64]
-    static constexpr int oK = oGd + 2 * (GDN2 ? nK : kChunk);  // K [64][LDK]
+    static constexpr int oGd = 0;                               // cumulative gate: GDN-2 [64][LDK], GDN [64] (fp64)
+    static constexpr int oK = oGd + (GDN2 ? GW * nK : 2 * kChunk);  // K [64][LDK]
     static constexpr int oQ = oK + nK;                         // Q, then Q.2^G (GDN-2)
     static constexpr int oBK = oQ + nK;                        // GDN-2: b.K, then b.K.2^G, then K.2^(G_last-G)
     static constexpr int oV = oBK + (GDN2 ? nK : 0);           // scaled V, then X
@@ -55,16 +57,21 @@ struct SimtSmem {
     static_assert(kChunk * DVT <= kChunk * LDT, "U must fit in the space of A");
 };
 
+// Per-channel (GDN-2) cumulative-gate type: fp64 for fp32 inputs, fp32 for bf16 inputs.
+template <typename TIn> struct SimtGate { using type = double; };
+template <> struct SimtGate<__nv_bfloat16> { using type = float; };
+
 template <typename TIn, typename TOut, int DK, int DVT, bool GDN2>
 __global__ void __launch_bounds__(kSimtThreads)
 gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
-    using L = SimtSmem<DK, DVT, GDN2>;
+    using GT = typename SimtGate<TIn>::type;
+    using L = SimtSmem<DK, DVT, GDN2, sizeof(GT) / 4>;
     constexpr int LDK = L::LDK, LDT = L::LDT, NT = kSimtThreads;
     constexpr int PER = kChunk * DVT / NT;  // (row, column) outputs per thread
     static_assert(kChunk * DVT % NT == 0, "tile must divide evenly");
     extern __shared__ __align__(16) float sm[];
-    double* sG = reinterpret_cast<double*>(sm + L::oGd);  // GDN-2 [64][LDK]
-    double* sG1 = sG;                                     // GDN [64]
+    GT* sG = reinterpret_cast<GT*>(sm + L::oGd);              // GDN-2 [64][LDK]
+    double* sG1 = reinterpret_cast<double*>(sm + L::oGd);     // GDN [64]
     float* sK = sm + L::oK;
     float* sQ = sm + L::oQ;
     float* sBK = sm + L::oBK;
@@ -127,7 +134,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
             sK[r * LDK + i] = kv;
             sQ[r * LDK + i] = qv;
             if (GDN2) {
-                sG[r * LDK + i] = (double)gv;
+                sG[r * LDK + i] = (GT)gv;
                 sBK[r * LDK + i] = bv * kv;
             }
         }
@@ -153,8 +160,8 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
             for (int i = tid; i < DK; i += NT) {
                 double acc = 0.0;
                 for (int r = 0; r < kChunk; ++r) {
-                    acc += sG[r * LDK + i];
-                    sG[r * LDK + i] = acc * kLog2eD;
+                    acc += (double)sG[r * LDK + i];
+                    sG[r * LDK + i] = (GT)(acc * kLog2eD);
                 }
             }
         } else if (tid == 0) {
@@ -166,18 +173,61 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
         }
         __syncthreads();
         // ---- A (strictly lower) and P (lower incl. diagonal)
+        if (GDN2) {
+            // 2x2 tiles (rows 2R, 2R+1; columns 2S, 2S+1) on and below the diagonal, S <= R: each channel's
+            // operands are loaded once per tile instead of once per entry.  Entries above the diagonal of a
+            // diagonal tile are computed and then discarded.
+            constexpr int kTiles = (kChunk / 2) * (kChunk / 2 + 1) / 2;
+            for (int tt = tid; tt < kTiles; tt += NT) {
+                int R = (int)((sqrtf(8.f * (float)tt + 1.f) - 1.f) * 0.5f);
+                while (R * (R + 1) / 2 > tt) --R;
+                while ((R + 1) * (R + 2) / 2 <= tt) ++R;
+                const int S = tt - R * (R + 1) / 2;
+                const int r0 = 2 * R, s0 = 2 * S;
+                float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f, p00 = 0.f, p01 = 0.f, p10 = 0.f, p11 = 0.f;
+                for (int i = 0; i < DK; ++i) {
+                    const GT gr0 = sG[r0 * LDK + i], gr1 = sG[(r0 + 1) * LDK + i];
+                    const GT gs0 = sG[s0 * LDK + i], gs1 = sG[(s0 + 1) * LDK + i];
+                    const float k0 = sK[s0 * LDK + i], k1 = sK[(s0 + 1) * LDK + i];
+                    const float b0 = sBK[r0 * LDK + i], b1 = sBK[(r0 + 1) * LDK + i];
+                    const float q0 = sQ[r0 * LDK + i], q1 = sQ[(r0 + 1) * LDK + i];
+                    const float k00 = k0 * exp2f((float)(gr0 - gs0)), k01 = k1 * exp2f((float)(gr0 - gs1));
+                    const float k10 = k0 * exp2f((float)(gr1 - gs0)), k11 = k1 * exp2f((float)(gr1 - gs1));
+                    a00 = fmaf(b0, k00, a00);
+                    a01 = fmaf(b0, k01, a01);
+                    a10 = fmaf(b1, k10, a10);
+                    a11 = fmaf(b1, k11, a11);
+                    p00 = fmaf(q0, k00, p00);
+                    p01 = fmaf(q0, k01, p01);
+                    p10 = fmaf(q1, k10, p10);
+                    p11 = fmaf(q1, k11, p11);
+                }
+                const bool diag = R == S;  // then (r0, s0 + 1) is above the diagonal
+                sA[r0 * LDT + s0] = diag ? 0.f : a00;
+                sA[r0 * LDT + s0 + 1] = diag ? 0.f : a01;
+                sA[(r0 + 1) * LDT + s0] = a10;
+                sA[(r0 + 1) * LDT + s0 + 1] = diag ? 0.f : a11;
+                sP[r0 * LDT + s0] = p00;
+                sP[r0 * LDT + s0 + 1] = diag ? 0.f : p01;
+                sP[(r0 + 1) * LDT + s0] = p10;
+                sP[(r0 + 1) * LDT + s0 + 1] = p11;
+                if (!diag) {  // the mirrored tile above the diagonal is zero
+                    sA[s0 * LDT + r0] = 0.f;
+                    sA[s0 * LDT + r0 + 1] = 0.f;
+                    sA[(s0 + 1) * LDT + r0] = 0.f;
+                    sA[(s0 + 1) * LDT + r0 + 1] = 0.f;
+                    sP[s0 * LDT + r0] = 0.f;
+                    sP[s0 * LDT + r0 + 1] = 0.f;
+                    sP[(s0 + 1) * LDT + r0] = 0.f;
+                    sP[(s0 + 1) * LDT + r0 + 1] = 0.f;
+                }
+            }
+        } else {
         for (int e = tid; e < kChunk * kChunk; e += NT) {
             const int r = e / kChunk, s = e % kChunk;
             float a = 0.f, pp = 0.f;
             if (s <= r) {
-                if (GDN2) {
-                    for (int i = 0; i < DK; ++i) {
-                        const float f = exp2f((float)(sG[r * LDK + i] - sG[s * LDK + i]));
-                        const float ks = sK[s * LDK + i] * f;
-                        a = fmaf(sBK[r * LDK + i], ks, a);
-                        pp = fmaf(sQ[r * LDK + i], ks, pp);
-                    }
-                } else {
+                {
                     float dkk = 0.f, dqk = 0.f;
                     for (int i = 0; i < DK; ++i) {
                         const float ks = sK[s * LDK + i];
@@ -193,6 +243,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
             sA[r * LDT + s] = a;
             sP[r * LDT + s] = pp;
         }
+        }
         __syncthreads();
         // ---- GDN-2: fold 2^G into Q and b.K (in place); (I + A)^-1 by forward substitution
         if (GDN2) {
@@ -203,16 +254,20 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
                 sBK[r * LDK + i] *= f;
             }
         }
-        if (tid < kChunk) {
-            const int c = tid;
-            for (int r = 0; r < c; ++r) sT[r * LDT + c] = 0.f;
-            for (int r = c; r < kChunk; ++r) {
-                float t = (r == c) ? 1.f : 0.f;
-                for (int s = c; s < r; ++s) t = fmaf(-sA[r * LDT + s], sT[s * LDT + c], t);
-                sT[r * LDT + c] = t;
+        // T[r][c] = [r == c] - sum_{c <= s < r} A[r][s] T[s][c], row by row: the four threads of column c
+        // take every fourth s and add their sums by shuffles (they are adjacent lanes of one warp)
+        {
+            static_assert(NT == 4 * kChunk, "four threads per column");
+            const int c = tid >> 2, part = tid & 3;
+            for (int r = 0; r < kChunk; ++r) {
+                float acc = 0.f;
+                for (int s = c + part; s < r; s += 4) acc = fmaf(sA[r * LDT + s], sT[s * LDT + c], acc);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                if (part == 0) sT[r * LDT + c] = r < c ? 0.f : (r == c ? 1.f : -acc);
+                __syncthreads();
             }
         }
-        __syncthreads();
         // ---- X = (scaled V) - (erase-side keys . 2^G) h ;  Oi = (Q . 2^G) h  (kept in registers)
         float oi[PER];
 #pragma unroll
