@@ -71,11 +71,20 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+# Source files each timed kernel family is compiled from (its own header and what that header includes);
+# a recorded DRAM traffic figure stays valid while these are unchanged.
+KERNEL_SOURCES = {
+    "gdn_tc_wy_kernel+gdn_tc_fwd_kernel": ["gdn_common.cuh", "gdn_sm100.cuh", "gdn_tc.cuh"],
+    "gdn_simt_fwd_kernel": ["gdn_common.cuh", "gdn_simt.cuh"],
+}
+
+
+def kernel_source_hash(kernel=None):
+    """sha256[:16] over the named kernel's source files (every file under csrc/ for an unknown kernel)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_105_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in KERNEL_SOURCES.get(kernel) or sorted(os.listdir(csrc)):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -86,7 +95,7 @@ def recorded_traffic(kernel, workload):
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    src = kernel_source_hash()
+    src = kernel_source_hash(kernel)
     for line in open(path):
         parts = dict(p.split("=", 1) for p in line.split() if "=" in p)
         if parts.get("kernel") == kernel and parts.get("workload") == workload and parts.get("sources") == src:
