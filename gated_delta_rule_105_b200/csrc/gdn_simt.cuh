@@ -118,7 +118,8 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
     for (int c0 = bos; c0 < eos; c0 += kChunk) {
         const int Lc = min(kChunk, eos - c0);
         __syncthreads();  // the previous chunk is done with every buffer
-        // ---- load the chunk (zero-padded past Lc)
+        // ---- load the chunk (zero-padded past Lc); unrolled so that many global loads are in flight
+#pragma unroll 8
         for (int e = tid; e < kChunk * DK; e += NT) {
             const int r = e / DK, i = e % DK;
             float kv = 0.f, qv = 0.f, gv = 0.f, bv = 0.f;
@@ -138,6 +139,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
                 sBK[r * LDK + i] = bv * kv;
             }
         }
+#pragma unroll
         for (int e = tid; e < kChunk * DVT; e += NT) {
             const int r = e / DVT, j = e % DVT;
             float x = 0.f;
