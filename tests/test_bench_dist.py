@@ -48,3 +48,27 @@ def test_reference_arm_other_ranks_exit_without_work():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                           "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_recorded_traffic_tracks_the_timed_kernels_sources(tmp_path, monkeypatch):
+    """The committed DRAM figure is reported only while the timed kernels' own source files are unchanged:
+    a change to another kernel's file keeps it, a change to one of them drops it to None."""
+    import shutil
+    sys.path.insert(0, ROOT)
+    import bench
+    root = tmp_path / "repo"
+    shutil.copytree(os.path.join(ROOT, "gated_delta_rule_105_b200", "csrc"), root / "gated_delta_rule_105_b200" / "csrc")
+    (root / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    kernel = "gdn_tc_wy_kernel+gdn_tc_fwd_kernel"
+    line = (f"kernel={kernel} workload=w sources={bench.kernel_source_hash(kernel)} bytes_per_launch=123 "
+            f"source=x\n")
+    (root / "profiles" / "dram_traffic.txt").write_text(line)
+    assert bench.recorded_traffic(kernel, "w") == 123.0
+    assert bench.recorded_traffic(kernel, "other") is None
+    csrc = root / "gated_delta_rule_105_b200" / "csrc"
+    (csrc / "gdn_simt.cuh").write_text((csrc / "gdn_simt.cuh").read_text() + "\n// edit\n")
+    assert bench.recorded_traffic(kernel, "w") == 123.0  # not one of this kernel's files
+    (csrc / "gdn_tc.cuh").write_text((csrc / "gdn_tc.cuh").read_text() + "\n// edit\n")
+    assert bench.recorded_traffic(kernel, "w") is None
+
