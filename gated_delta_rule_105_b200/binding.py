@@ -209,8 +209,10 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, output_final_state=True
 
 def gdn_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, h0=None, output_final_state=True, cu_seqlens=None,
                           BT=64, o=None, hT=None, o_dtype=None):
-    """As :func:`gdn_chunk_fwd`, through ``gdn_chunk_fwd_noalloc``: no workspace is allocated (the library's
-    static scratch serves the tensor-core path; calls must not overlap on the device)."""
+    """As :func:`gdn_chunk_fwd`, through ``gdn_chunk_fwd_noalloc``, for callers that may not allocate device
+    memory (an engine that owns all of it, a host framework's allocator): no workspace is allocated, the
+    library's static 128 MiB scratch serves the tensor-core path, sizes that need more are refused, and calls
+    must not overlap on the device.  The outputs ``o`` and ``hT`` are still allocated here unless passed in."""
     B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype)
     _check_dev("g", g, torch.float32)
     _check_dev("beta", beta, torch.float32)

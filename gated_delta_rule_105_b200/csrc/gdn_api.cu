@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 
 #include "gdn.h"
 #include "gdn_common.cuh"
@@ -18,11 +19,19 @@ __device__ unsigned int g_err_word;
 
 static thread_local char t_msg[512];
 
-// Scratch for gdn_chunk_fwd_noalloc: reserved once per process and device when the module loads, so that
-// entry point never allocates.  Its size is GDN_STATIC_WS_BYTES (gdn.h).
+// Scratch of gdn_chunk_fwd_noalloc, for callers that must not allocate device memory.  It is part of the
+// library's device image: the CUDA runtime reserves it on a device when it loads this module there (with lazy
+// module loading, at the first launch or symbol lookup of any entry point on that device) and keeps it until
+// the process exits.  Its size is GDN_STATIC_WS_BYTES (gdn.h).
 static __device__ __align__(256) uint8_t g_static_ws[GDN_STATIC_WS_BYTES];
 static thread_local gdn_kernel t_last_kernel = GDN_KERNEL_AUTO;
 static std::atomic<int> g_kernel_choice{GDN_KERNEL_AUTO};
+
+// Device address of g_static_ws on each device.  In host code the array's name is only a host-side handle, so
+// the address is looked up once per device, with that device current, by the first no-workspace call there.
+constexpr int kMaxDevices = 64;
+static std::atomic<void*> g_static_ws_addr[kMaxDevices];
+static std::mutex g_static_ws_mu;
 
 static gdn_status fail(gdn_status st, const char* fmt, ...) {
     va_list ap;
@@ -138,6 +147,27 @@ static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, gdn_dtype o_d
     return st;
 }
 
+// The device address of the no-workspace scratch on the current device (see g_static_ws_addr).
+static gdn_status static_scratch(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GDN_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+    void* ptr = g_static_ws_addr[dev].load(std::memory_order_acquire);
+    if (!ptr) {
+        std::lock_guard<std::mutex> lock(g_static_ws_mu);
+        ptr = g_static_ws_addr[dev].load(std::memory_order_relaxed);
+        if (!ptr) {
+            e = cudaGetSymbolAddress(&ptr, g_static_ws);
+            if (e != cudaSuccess || !ptr)
+                return fail(GDN_ERR_CUDA, "static scratch address: %s", cudaGetErrorString(e));
+            g_static_ws_addr[dev].store(ptr, std::memory_order_release);
+        }
+    }
+    *out = ptr;
+    return GDN_OK;
+}
+
 }  // namespace gdn
 
 using namespace gdn;
@@ -171,10 +201,22 @@ gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, co
     gdn_status st = check_common(q, k, v, g, beta, nullptr, false, scale, h0, o, hT, B, T, H, dk, dv, BT, dt,
                                  o_dt, cu_seqlens, n_seqs, nullptr, 0, &n_seq);
     if (st != GDN_OK) return st;
-    void* ws = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&ws, g_static_ws);
-    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "static scratch: %s", cudaGetErrorString(e));
     FwdParams p{q, k, v, g, beta, nullptr, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
+    // The tensor-core path needs tc_workspace_bytes() of scratch; beyond the static array's size the call is
+    // refused (callers that can allocate use gdn_chunk_fwd with their own workspace).
+    const bool tc_path = dt == GDN_BF16 && tc_supported(p, false, o_dt == GDN_F32) &&
+                         g_kernel_choice.load() != GDN_KERNEL_SIMT && n_seq > 0;
+    if (tc_path) {
+        const size_t need = tc_workspace_bytes(B, T, H, n_seq);
+        if (need > (size_t)GDN_STATIC_WS_BYTES)
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "gdn_chunk_fwd_noalloc: these sizes need %zu bytes of scratch, the static scratch holds %zu "
+                        "(GDN_STATIC_WS_BYTES); use gdn_chunk_fwd with a caller workspace",
+                        need, (size_t)GDN_STATIC_WS_BYTES);
+    }
+    void* ws = nullptr;
+    st = static_scratch(&ws);
+    if (st != GDN_OK) return st;
     return run(p, false, dt, o_dt, ws, (size_t)GDN_STATIC_WS_BYTES, stream);
 }
 

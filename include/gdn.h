@@ -91,17 +91,34 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          const int32_t* cu_seqlens, int n_seqs,
                          void* workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Size of the scratch array compiled into the library for gdn_chunk_fwd_noalloc: 128 MiB of device memory,
- * reserved per process and device when the library's device code is loaded. */
+/* Size of the scratch array compiled into the library for gdn_chunk_fwd_noalloc: 128 MiB of device memory.  It is
+ * part of the library's device code, so the CUDA runtime reserves it on each device where it loads that code and
+ * keeps it until the process exits.  With lazy module loading (the CUDA default) that happens during the first
+ * call of ANY libgdn entry point on a device -- also in processes that never call gdn_chunk_fwd_noalloc -- and
+ * that first call can therefore fail with GDN_ERR_CUDA (out of memory) on a nearly full device. */
 #define GDN_STATIC_WS_BYTES (128u * 1024u * 1024u)
 
-/* gdn_chunk_fwd without a caller workspace and without any allocation: the tensor-core path uses the
- * library's static scratch (GDN_STATIC_WS_BYTES).  A call that needs more scratch than that (see
- * gdn_workspace_bytes) runs as gdn_chunk_fwd with a too-small workspace would: AUTO takes the SIMT kernel,
- * TC returns GDN_ERR_UNSUPPORTED.  All calls of this entry point in a process share the one scratch per
- * device, so they must not overlap on the device: issue them on one stream, or order them (events,
- * synchronisation); concurrent callers use gdn_chunk_fwd with their own workspaces.  Arguments, layouts
- * and errors are otherwise those of gdn_chunk_fwd. */
+/* gdn_chunk_fwd for callers that cannot allocate device memory.  (The pages have no counterpart to this entry
+ * point: it exists for the library's users.)  Some callers may not call cudaMalloc at all: serving engines that
+ * hand all free device memory to their own pool at start-up and forbid any later allocation; plug-ins running
+ * inside a host framework that owns the device allocator; and latency-critical loops, where cudaMalloc and
+ * cudaFree may synchronise the device and take unbounded time.  This entry point takes no workspace and
+ * allocates nothing -- no cudaMalloc, cudaFree or allocating library routine: the tensor-core path keeps its
+ * per-chunk WY factors in the library's static scratch array (GDN_STATIC_WS_BYTES, see above).  The caller still
+ * passes every input and output buffer.
+ *   Set-up: the first call on a device, with that device current, looks the scratch array's device address up
+ *   (cudaGetSymbolAddress) and caches it for later calls on that device.  Make that first call before any stream
+ *   capture, since the look-up may load the library's device code.
+ *   Limit: when the call would run the tensor-core path (bf16 inputs, dk == 128, dv a multiple of 128, kernel not
+ *   forced to SIMT) and gdn_workspace_bytes() for these sizes exceeds GDN_STATIC_WS_BYTES, the call is refused
+ *   with GDN_ERR_UNSUPPORTED (gdn_last_error() says how much it needed) and nothing is enqueued.  Calls that run
+ *   the SIMT kernel use no scratch and have no such limit.
+ *   Sharing: every call in the process uses the same array on a device, and a call leaves its contents behind
+ *   (nothing in it has to start at zero: each call writes every byte it later reads).  Calls that overlap on the
+ *   device -- issued on different streams without ordering between them -- race on the array and give undefined
+ *   results: issue them on one stream, or order them with events; concurrent callers use gdn_chunk_fwd with their
+ *   own workspaces.
+ * Arguments, layouts, results and errors are otherwise those of gdn_chunk_fwd. */
 gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                                  float scale, const float* h0, void* o, float* hT,
                                  int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt, gdn_dtype o_dt,
