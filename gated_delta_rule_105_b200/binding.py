@@ -62,6 +62,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_profile_enable.restype = i
     lib.gdn_profile_take.argtypes = [i, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
     lib.gdn_profile_take.restype = i
+    lib.gdn_debug_stall.argtypes = [i]
+    lib.gdn_debug_stall.restype = i
     _lib = lib
     return lib
 
@@ -102,6 +104,12 @@ def set_kernel(name: str) -> None:
 
 def last_kernel() -> str:
     return KERNEL_NAMES[load_library().gdn_last_kernel()]
+
+
+def debug_stall(on: bool) -> None:
+    """Diagnostic of the device time-out path (``gdn_debug_stall``): while on, tensor-core GDN calls make a
+    pipeline wait run out; ``check_error`` then raises with status GDN_ERR_TIMEOUT."""
+    _raise_on(load_library().gdn_debug_stall(1 if on else 0))
 
 
 def check_error(stream=None) -> None:

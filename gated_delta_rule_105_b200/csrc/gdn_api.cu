@@ -26,6 +26,7 @@ static thread_local char t_msg[512];
 static __device__ __align__(256) uint8_t g_static_ws[GDN_STATIC_WS_BYTES];
 static thread_local gdn_kernel t_last_kernel = GDN_KERNEL_AUTO;
 static std::atomic<int> g_kernel_choice{GDN_KERNEL_AUTO};
+static std::atomic<int> g_debug_stall{0};
 
 // Device address of g_static_ws on each device.  In host code the array's name is only a host-side handle, so
 // the address is looked up once per device, with that device current, by the first no-workspace call there.
@@ -143,7 +144,10 @@ static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, gdn_dtype o_d
         // AUTO: a configuration the tcgen05 build cannot take runs on the SIMT kernel
     }
     st = gdn2 ? launch_simt<true>(p, dt, o_dt, err, stream) : launch_simt<false>(p, dt, o_dt, err, stream);
-    if (st == GDN_OK) t_last_kernel = GDN_KERNEL_SIMT;
+    if (st == GDN_OK) {
+        t_last_kernel = GDN_KERNEL_SIMT;
+        t_msg[0] = 0;  // the refused tensor-core attempt is not a failure of this call
+    }
     return st;
 }
 
@@ -190,6 +194,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
                                  o_dt, cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
     if (st != GDN_OK) return st;
     FwdParams p{q, k, v, g, beta, nullptr, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
+    p.debug_stall = g_debug_stall.load();
     return run(p, false, dt, o_dt, workspace, ws_bytes, stream);
 }
 
@@ -202,6 +207,7 @@ gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, co
                                  o_dt, cu_seqlens, n_seqs, nullptr, 0, &n_seq);
     if (st != GDN_OK) return st;
     FwdParams p{q, k, v, g, beta, nullptr, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
+    p.debug_stall = g_debug_stall.load();
     // The tensor-core path needs tc_workspace_bytes() of scratch; beyond the static array's size the call is
     // refused (callers that can allocate use gdn_chunk_fwd with their own workspace).
     const bool tc_path = dt == GDN_BF16 && tc_supported(p, false, o_dt == GDN_F32) &&
@@ -240,6 +246,11 @@ gdn_status gdn_set_kernel(gdn_kernel kernel) {
 }
 
 gdn_kernel gdn_last_kernel(void) { return t_last_kernel; }
+
+gdn_status gdn_debug_stall(int on) {
+    g_debug_stall.store(on != 0);
+    return GDN_OK;
+}
 
 gdn_status gdn_check_error(cudaStream_t stream) {
     cudaError_t e = cudaStreamSynchronize(stream);

@@ -30,6 +30,7 @@ struct FwdParams {
     const int32_t* cu_seqlens;  // [N+1] or null
     float scale;
     int B, T, H, dk, dv, n_seq;
+    int debug_stall;  // diagnostic (gdn_debug_stall): 0 in every ordinary call
 };
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

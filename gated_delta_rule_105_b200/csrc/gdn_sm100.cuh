@@ -49,12 +49,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // every later bounded wait of the CTA then returns false at once, so all warps drain to the exit.
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 // The slow path is kept out of line: waits appear at many places and are usually satisfied by the first try.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsigned* err) {
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsigned* err,
+                                            long long limit = kWaitLimitCycles) {
     const long long t0 = clock64();
     while (true) {
         if (*abort_flag) return false;
         if (mbar_try_wait(bar, parity)) return true;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             atomicOr(err, kErrTimeout);
             return false;

@@ -476,7 +476,7 @@ struct TcSmem {
     static constexpr uint32_t HT_STAGE = 32768;
     static constexpr uint32_t GATE = HT + 2 * HT_STAGE;  // 4 x TcGate
     static constexpr uint32_t BARS = GATE + 4 * sizeof(TcGate);
-    static constexpr uint32_t N_BARS = 28;
+    static constexpr uint32_t N_BARS = 29;
     static constexpr uint32_t MISC = BARS + 8 * N_BARS;  // tmem base, abort flag
     static constexpr uint32_t END = MISC + 64;
     static constexpr uint32_t ALLOC = END + 1024;  // slack for the 1024-byte alignment of the base
@@ -505,7 +505,11 @@ enum TcBar : int {
     B_DRAIN = 24,      // [2] final commit of each MMA issuer
     B_HM_READY = 26,   // fp32 state in TMEM re-scaled by the next chunk's decay (256)
     B_U_RND = 27,      // U in TMEM rounded to tf32 in place, for the O2 MMA (256)
+    B_STALL = 28,      // diagnostic only: nothing ever arrives on it (gdn_debug_stall)
 };
+
+// Limit of the diagnostic wait on B_STALL (~1 ms): short, so the time-out path runs quickly.
+constexpr long long kStallLimitCycles = 2000000LL;
 
 // TMEM columns.  U^T is accumulated in fp32 at TM_U and read there, as tf32, by the O2 MMA; the state
 // warpgroups write U diag f as bf16 hi/lo pairs (two values per column) to TM_UF for the h^T MMA.
@@ -701,7 +705,12 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint64_t d_v = desc_mn_sw128(sbase + L::V, 8192);
             const uint64_t d_t = desc_k_sw128(sbase + L::TW);
             const uint64_t d_wt = desc_mn_sw128(sbase + L::WT, 8192);
-            for (int c = 0; c < nc; ++c) {
+            int nc_run = nc;
+            // Diagnostic: a wait on a barrier that nothing arrives on, with a short limit.  It runs out, sets
+            // the error word and the abort flag, and this warp issues no MMA; every other warp then leaves
+            // through its own bounded waits and drains what it issued.
+            if (p.debug_stall && !mbar_wait_slow(&bars[B_STALL], 0, abort_flag, err, kStallLimitCycles)) nc_run = 0;
+            for (int c = 0; c < nc_run; ++c) {
                 const int st = c & 1;
                 const uint32_t kq = sbase + L::KQ + st * L::KQ_STAGE;
                 const uint64_t d_ht = desc_k_sw128(sbase + L::HT + st * L::HT_STAGE);

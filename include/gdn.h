@@ -137,6 +137,14 @@ gdn_status gdn_set_kernel(gdn_kernel kernel);
 /* Kernel family that the most recent successful *_fwd call on this thread launched. */
 gdn_kernel gdn_last_kernel(void);
 
+/* Diagnostic of the device time-out path (no counterpart on the pages; off by default; process-wide).  While
+ * on, every later tensor-core GDN call makes one of its chunk kernel's pipeline waits wait on a barrier that
+ * nothing ever arrives on, with a ~1 ms limit.  The wait runs out, the kernel sets the device error word, its
+ * warps leave through their own bounded waits after draining every copy and tensor-core operation they issued,
+ * and the call's outputs are undefined; the call itself returns GDN_OK and gdn_check_error() then reports
+ * GDN_ERR_TIMEOUT.  Calls on the SIMT kernel are not affected.  Returns GDN_OK. */
+gdn_status gdn_debug_stall(int on);
+
 /* Synchronises `stream`, then reads and clears the device error word of the current device:
  * GDN_OK, GDN_ERR_TIMEOUT, GDN_ERR_DEVICE_ARG, or GDN_ERR_CUDA if the stream reports a CUDA error. */
 gdn_status gdn_check_error(cudaStream_t stream);

@@ -158,3 +158,28 @@ def test_workload_full_size_sampled(name, kernel, odt):
         ou, hu = unit_slices(inp, o, hT, u)
         ro, rh = ref[u]
         check(ou, hu, ro, rh, w.dtype, odt, f"{name} {kernel} o={odt} unit {u}")
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workload_full_size_every_unit(name):
+    """Every (sequence, head) unit of each workload at full size, o in q's dtype (the operation's output)."""
+    import os
+    w = WORKLOADS[name]
+    inp = generate_workload(w)
+    odt = w.dtype
+    o, hT = run_cuda(inp, w.variant, o_dtype=odt)
+    torch.cuda.synchronize()
+    n_seq = hT.shape[0]
+    units = [(n, h) for n in range(n_seq) for h in range(w.H)]
+    threads = max(1, len(os.sched_getaffinity(0)))
+    worst_o = worst_h = 0.0
+    for i in range(0, len(units), 4 * threads):
+        batch = units[i:i + 4 * threads]
+        ref = oracle_units(inp, w.variant, batch, threads=threads)
+        for u in batch:
+            ou, hu = unit_slices(inp, o, hT, u)
+            ro, rh = ref[u]
+            check(ou, hu, ro, rh, w.dtype, odt, f"{name} o={odt} unit {u}")
+            worst_o = max(worst_o, o_excess(ou, ro, w.dtype, odt))
+            worst_h = max(worst_h, relerr(hu, rh))
+    print(f"{name}: {len(units)} units, worst o {worst_o:.3f} x allowance, worst hT err {worst_h:.3g}")
