@@ -10,11 +10,11 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 
 
 def build(force: bool = False) -> str:
-    src = os.path.join(_HERE, "gdn_oracle.c")
+    srcs = [os.path.join(_HERE, f) for f in ("gdn_oracle.c", "gdn_vjp.c")]
     out = os.path.join(_HERE, "liboracle.so")
-    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+    if force or not os.path.exists(out) or os.path.getmtime(out) < max(os.path.getmtime(s) for s in srcs):
         subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC",
-                               "-o", out, src, "-lm"])
+                               "-o", out, *srcs, "-lm"])
     return out
 
 
