@@ -82,6 +82,7 @@ def load_peaks():
 # a recorded DRAM traffic figure stays valid while these are unchanged.
 KERNEL_SOURCES = {
     "gdn_tc_wy_kernel+gdn_tc_fwd_kernel": ["gdn_common.cuh", "gdn_sm100.cuh", "gdn_tc.cuh"],
+    "gdn2_tc_prep_kernel+gdn2_tc_fwd_kernel": ["gdn_common.cuh", "gdn_sm100.cuh", "gdn_tc.cuh", "gdn2_tc.cuh"],
     "gdn_simt_fwd_kernel": ["gdn_common.cuh", "gdn_simt.cuh"],
 }
 
@@ -315,7 +316,8 @@ def run_ours(args, w):
                                 device_id=torch.device("cuda", local_rank))
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    from gated_delta_rule_105_b200 import (gdn2_chunk_fwd, gdn_chunk_fwd, last_kernel, set_kernel, check_error,
+    from gated_delta_rule_105_b200 import (gdn2_chunk_fwd, gdn2_workspace_bytes, gdn_chunk_fwd, last_kernel,
+                                           set_kernel, check_error,
                                            profile_enable, profile_take, workspace_bytes)
     from gated_delta_rule_105_b200.inputs import generate
     set_kernel(args.kernel)
@@ -331,7 +333,8 @@ def run_ours(args, w):
     hT = torch.empty((n_seq, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
 
     # the tensor-core path's scratch (WY factors of every chunk), allocated once like a caller would
-    n_ws = workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, C, 0 if d["cu_seqlens"] is None else n_seq)
+    n_ws = (workspace_bytes if w.variant == "gdn" else gdn2_workspace_bytes)(
+        w.B, w.T, w.H, w.dk, w.dv, C, 0 if d["cu_seqlens"] is None else n_seq)
     wsp = torch.empty(n_ws, dtype=torch.uint8, device=dev) if (n_ws and w.dtype == "bf16") else None
 
     if w.variant == "gdn":
@@ -341,7 +344,7 @@ def run_ours(args, w):
     else:
         def step(dd, oo, hh):
             return gdn2_chunk_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["b"], dd["w"], dd["scale"], dd["h0"],
-                                  True, dd["cu_seqlens"], o=oo, hT=hh, o_dtype=o_torch)
+                                  True, dd["cu_seqlens"], o=oo, hT=hh, o_dtype=o_torch, workspace=wsp)
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -432,7 +435,8 @@ def run_ours(args, w):
     # the path's kernels: on the tensor-core path the WY kernel and then the chunk kernel run one after the
     # other on the stream, with no overlap; the roofline is taken over the whole step: the operation's
     # algorithmic bytes (o in q's dtype) against the step's device time
-    kname = {"tc": "gdn_tc_wy_kernel+gdn_tc_fwd_kernel", "simt": "gdn_simt_fwd_kernel"}.get(kernel, kernel)
+    kname = {"tc": "gdn_tc_wy_kernel+gdn_tc_fwd_kernel" if w.variant == "gdn"
+             else "gdn2_tc_prep_kernel+gdn2_tc_fwd_kernel", "simt": "gdn_simt_fwd_kernel"}.get(kernel, kernel)
     traffic = recorded_traffic(kname, w.name)
     if bound == "hbm":
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -470,6 +474,93 @@ def run_ours(args, w):
     return 0
 
 
+# ------------------------------------------------------------------------------------------ the other rows
+def run_row(args, w):
+    """Device throughput of one of the path's other kernels on the bench workload's shape (1 GPU, rank 0 prints):
+    ``decode`` -- one recurrent decode step for 64 sequences of the workload's heads (state read and written in
+    place); ``prelude`` -- short conv + SiLU + L2 norm + gates over the whole workload; ``output_gate`` -- the
+    RMSNorm x SiLU epilogue over the workload's output.  Each is HBM-bound: the roofline is its bytes per launch."""
+    import torch
+    from gated_delta_rule_105_b200 import decode_fwd, output_gate_fwd, prelude_fwd, profile_enable, profile_take
+    from gated_delta_rule_105_b200.inputs import generate, generate_prelude
+    rank, local_rank, ws = dist_env()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    if args.path == "decode":
+        N = 64
+        inp = generate(N, 1, H, dk, dv, w.dtype, w.seed, w.variant if w.variant != "gdn2" else "gdn2", 0.02)
+        d = {k: (v[:, 0].contiguous().to(dev) if isinstance(v, torch.Tensor) and k not in ("h0", "cu_seqlens")
+                 else v) for k, v in inp.items()}
+        state = inp["h0"].to(dev)
+        o = torch.empty((N, H, dv), dtype=d["q"].dtype, device=dev)
+        variant = w.variant
+
+        def step():
+            decode_fwd(d["q"], d["k"], d["v"], d["g"], d.get("beta"), state, d["scale"], o=o, b=d.get("b"),
+                       w=d.get("w"), variant=variant)
+        s = 2 if w.dtype == "bf16" else 4
+        gate_b = 8 if variant == "gdn" else 4 * (2 * dk + dv)
+        nbytes = N * H * (2 * 4 * dk * dv + s * (2 * dk + 2 * dv) + gate_b)
+        tokens, kname, workload = N, "gdn_decode_kernel", f"decode N{N} H{H} dk{dk} dv{dv} ({w.name} heads)"
+    elif args.path == "prelude":
+        inp = generate_prelude(B, T, H, dk, dv, w.dtype, w.seed)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+
+        def step():
+            prelude_fwd(d["xq"], d["xk"], d["xv"], d["wq"], d["wk"], d["wv"], d["a"], d["A_log"], d["dt_bias"], d["b"])
+        s = 2 if w.dtype == "bf16" else 4
+        nbytes = B * T * H * (2 * s * (2 * dk + dv) + 4 * 4)
+        tokens, kname, workload = B * T, "gdn_prelude_kernel", f"prelude B{B} T{T} H{H} dk{dk} dv{dv}"
+    else:
+        gen = torch.Generator().manual_seed(w.seed)
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        o_in = torch.randn((B, T, H, dv), generator=gen).to(tdt).to(dev)
+        z = torch.randn((B, T, H, dv), generator=gen).to(tdt).to(dev)
+        wt = torch.rand(dv, generator=gen).add_(0.5).to(dev)
+        y = torch.empty_like(o_in)
+
+        def step():
+            output_gate_fwd(o_in, z, wt, y=y)
+        nbytes = B * T * H * dv * 3 * o_in.element_size()
+        tokens, kname, workload = B * T, "gdn_output_gate_kernel", f"output gate B{B} T{T} H{H} dv{dv}"
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    profile_take()
+    profile_enable(True)
+    for _ in range(max(3, min(args.steps, 20))):
+        step()
+    torch.cuda.synchronize(dev)
+    profile_enable(False)
+    n_l, ms_l = profile_take()[kname]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, src = load_peaks()
+    kernel_ms = ms_l / n_l
+    gbs = nbytes / (kernel_ms * 1e-3) / 1e9
+    line = {"metric": f"{args.path} tokens/s, % of B200 HBM roofline (1 GPU)", "value": tokens / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": workload, "path": args.path},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None, "kernel": kname,
+                         "algorithmic_bytes": int(nbytes), "kernel_ms": round(kernel_ms, 5),
+                         "peak_source": src},
+            "gpu_launches": args.steps, "clocks": sampler.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -481,6 +572,8 @@ def main(argv=None):
     ap.add_argument("--o-dtype", default="bf16", choices=["f32", "bf16"],
                     help="output dtype for bf16 inputs: bf16 (q's dtype, as the operation defines o) or f32 "
                          "(its extra bytes are reported as roofline.overhead_bytes, not as algorithmic work)")
+    ap.add_argument("--path", default="chunk", choices=["chunk", "decode", "prelude", "output_gate"],
+                    help="chunk: the chunked forward (the headline); the others time that row's kernel alone")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds for the whole reference arm")
@@ -490,6 +583,8 @@ def main(argv=None):
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.path != "chunk":
+        return run_row(args, w)
     return run_ours(args, w)
 
 

@@ -40,6 +40,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, fp, i, f, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.gdn_workspace_bytes.argtypes = [i] * 7
     lib.gdn_workspace_bytes.restype = sz
+    lib.gdn2_workspace_bytes.argtypes = [i] * 7
+    lib.gdn2_workspace_bytes.restype = sz
+    lib.gdn_kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [i] * 8 + [vp, i, vp, sz, vp]
+    lib.gdn_kda_chunk_fwd.restype = i
     lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [i] * 8 + [vp, i, vp, sz, vp]
     lib.gdn_chunk_fwd.restype = i
     lib.gdn_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [i] * 8 + [vp, i, vp]
@@ -62,6 +66,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_profile_enable.restype = i
     lib.gdn_profile_take.argtypes = [i, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
     lib.gdn_profile_take.restype = i
+    for name in ("gdn_decode_fwd", "gdn_kda_decode_fwd"):
+        getattr(lib, name).argtypes = [vp, vp, vp, fp, fp, f, fp, vp] + [i] * 6 + [vp]
+        getattr(lib, name).restype = i
+    lib.gdn2_decode_fwd.argtypes = [vp, vp, vp, fp, fp, fp, f, fp, vp] + [i] * 6 + [vp]
+    lib.gdn2_decode_fwd.restype = i
+    lib.gdn_prelude_fwd.argtypes = [vp] * 11 + [fp, i, fp, fp, i, fp, fp, i, vp, vp, vp] + [i] * 5 + [i, f, vp, i, vp]
+    lib.gdn_prelude_fwd.restype = i
+    lib.gdn_output_gate_fwd.argtypes = [vp, vp, fp, vp, ctypes.c_longlong, i, i, f, vp]
+    lib.gdn_output_gate_fwd.restype = i
     lib.gdn_debug_stall.argtypes = [i]
     lib.gdn_debug_stall.restype = i
     _lib = lib
@@ -118,7 +131,9 @@ def check_error(stream=None) -> None:
     _raise_on(load_library().gdn_check_error(ctypes.c_void_p(s.cuda_stream)))
 
 
-PROFILE_KERNELS = {"gdn_simt_fwd_kernel": 0, "gdn_tc_wy_kernel": 1, "gdn_tc_fwd_kernel": 2}
+PROFILE_KERNELS = {"gdn_simt_fwd_kernel": 0, "gdn_tc_wy_kernel": 1, "gdn_tc_fwd_kernel": 2, "gdn2_tc_prep_kernel": 3,
+                   "gdn2_tc_fwd_kernel": 4, "gdn_decode_kernel": 5, "gdn_prelude_kernel": 6,
+                   "gdn_output_gate_kernel": 7}
 
 
 def profile_enable(on: bool = True) -> None:
@@ -179,13 +194,18 @@ def workspace_bytes(B, T, H, dk, dv, BT=64, n_seqs=0) -> int:
     return int(load_library().gdn_workspace_bytes(B, T, H, dk, dv, BT, n_seqs))
 
 
-def _workspace(q, B, T, H, dk, dv, BT, n_seqs, workspace):
+def gdn2_workspace_bytes(B, T, H, dk, dv, BT=64, n_seqs=0) -> int:
+    """Device workspace (bytes) the tensor-core path of ``gdn2_chunk_fwd`` / ``gdn_kda_chunk_fwd`` can use."""
+    return int(load_library().gdn2_workspace_bytes(B, T, H, dk, dv, BT, n_seqs))
+
+
+def _workspace(q, B, T, H, dk, dv, BT, n_seqs, workspace, gdn2=False):
     if workspace is not None:
         _check_dev("workspace", workspace, torch.uint8)
         return workspace
     if q.dtype != torch.bfloat16:
         return None
-    nbytes = workspace_bytes(B, T, H, dk, dv, BT, n_seqs)
+    nbytes = (gdn2_workspace_bytes if gdn2 else workspace_bytes)(B, T, H, dk, dv, BT, n_seqs)
     return torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes > 0 else None
 
 
@@ -237,10 +257,11 @@ def gdn_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, h0=None, output_final_st
 
 
 def gdn2_chunk_fwd(q, k, v, g, b, w, scale=None, h0=None, output_final_state=True, cu_seqlens=None, BT=64,
-                   o=None, hT=None, o_dtype=None):
+                   o=None, hT=None, o_dtype=None, workspace=None):
     """Gated Delta Rule-2 forward through ``gdn2_chunk_fwd`` of the C ABI.
 
     g (per-channel log-decay) and b (erase gate) are [B,T,H,dk] fp32, w (write gate) is [B,T,H,dv] fp32.
+    ``workspace`` (uint8, at least :func:`gdn2_workspace_bytes`) is allocated per call when not given.
     """
     B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype)
     for name, t, shape in (("g", g, (B, T, H, dk)), ("b", b, (B, T, H, dk)), ("w", w, (B, T, H, dv))):
@@ -249,10 +270,33 @@ def gdn2_chunk_fwd(q, k, v, g, b, w, scale=None, h0=None, output_final_state=Tru
             raise ValueError(f"{name} must be {list(shape)}")
     scale = dk ** -0.5 if scale is None else float(scale)
     stream = torch.cuda.current_stream(q.device).cuda_stream
+    n_seqs = 0 if cu_seqlens is None else n_seq
+    ws = _workspace(q, B, T, H, dk, dv, BT, n_seqs, workspace, gdn2=True)
     st = load_library().gdn2_chunk_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), scale, _ptr(h0), _ptr(o), _ptr(hT),
         B, T, H, dk, dv, BT, _dtype_code(q), _dtype_code(o), _ptr(cu_seqlens),
-        0 if cu_seqlens is None else n_seq, None, 0, ctypes.c_void_p(stream))
+        n_seqs, _ptr(ws), 0 if ws is None else ws.numel(), ctypes.c_void_p(stream))
+    _raise_on(st)
+    return o, hT
+
+
+def gdn_kda_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, output_final_state=True, cu_seqlens=None, BT=64,
+                      o=None, hT=None, o_dtype=None, workspace=None):
+    """KDA forward through ``gdn_kda_chunk_fwd``: per-channel log-decay g [B,T,H,dk] fp32 and one scalar
+    beta [B,T,H] fp32 as both the erase and the write gate (GDN-2 with b = w = beta)."""
+    B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype)
+    for name, t, shape in (("g", g, (B, T, H, dk)), ("beta", beta, (B, T, H))):
+        _check_dev(name, t, torch.float32)
+        if t.shape != shape:
+            raise ValueError(f"{name} must be {list(shape)}")
+    scale = dk ** -0.5 if scale is None else float(scale)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    n_seqs = 0 if cu_seqlens is None else n_seq
+    ws = _workspace(q, B, T, H, dk, dv, BT, n_seqs, workspace, gdn2=True)
+    st = load_library().gdn_kda_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(o), _ptr(hT),
+        B, T, H, dk, dv, BT, _dtype_code(q), _dtype_code(o), _ptr(cu_seqlens),
+        n_seqs, _ptr(ws), 0 if ws is None else ws.numel(), ctypes.c_void_p(stream))
     _raise_on(st)
     return o, hT
 
@@ -261,3 +305,102 @@ def chunk_gated_delta_rule(q, k, v, g, beta, scale=None, initial_state=None, out
                            cu_seqlens=None):
     """The token mixer call by the name the pages use; same as :func:`gdn_chunk_fwd`."""
     return gdn_chunk_fwd(q, k, v, g, beta, scale, initial_state, output_final_state, cu_seqlens)
+
+
+def decode_fwd(q, k, v, g, beta, state, scale=None, o=None, o_dtype=None, b=None, w=None, variant="gdn"):
+    """One recurrent decode step (``gdn_decode_fwd`` / ``gdn2_decode_fwd`` / ``gdn_kda_decode_fwd``).
+
+    q, k [N,H,dk] and v [N,H,dv] (fp32 or bf16); ``state`` [N,H,dk,dv] fp32 is updated in place.  GDN: g, beta
+    [N,H]; KDA: g [N,H,dk], beta [N,H]; GDN-2: g, b [N,H,dk], w [N,H,dv] (pass beta=None).  Returns o [N,H,dv].
+    """
+    _check_dev("q", q)
+    dt = q.dtype
+    o_dtype = dt if o_dtype is None else o_dtype
+    _check_dev("k", k, dt)
+    _check_dev("v", v, dt)
+    _check_dev("state", state, torch.float32)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:2] != (N, H) or state.shape != (N, H, dk, dv):
+        raise ValueError("q, k [N,H,dk], v [N,H,dv] and state [N,H,dk,dv] must agree")
+    gate_shapes = {"gdn": {"g": (N, H), "beta": (N, H)}, "kda": {"g": (N, H, dk), "beta": (N, H)},
+                   "gdn2": {"g": (N, H, dk), "b": (N, H, dk), "w": (N, H, dv)}}[variant]
+    gates = {"g": g, "beta": beta, "b": b, "w": w}
+    for name, shape in gate_shapes.items():
+        _check_dev(name, gates[name], torch.float32)
+        if gates[name] is None or gates[name].shape != shape:
+            raise ValueError(f"{name} must be {list(shape)}")
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=o_dtype, device=q.device)
+    _check_dev("o", o, o_dtype)
+    scale = dk ** -0.5 if scale is None else float(scale)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(q.device).cuda_stream)
+    lib = load_library()
+    tail = (scale, _ptr(state), _ptr(o), N, H, dk, dv, _dtype_code(q), _dtype_code(o), stream)
+    if variant == "gdn2":
+        st = lib.gdn2_decode_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), *tail)
+    else:
+        fn = lib.gdn_decode_fwd if variant == "gdn" else lib.gdn_kda_decode_fwd
+        st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), *tail)
+    _raise_on(st)
+    return o
+
+
+def prelude_fwd(xq, xk, xv, wq, wk, wv, a, A_log, dt_bias, b, c=None, conv_state=None, conv_state_out=None,
+                cu_seqlens=None, l2_eps=1e-6):
+    """The mixer's prelude through ``gdn_prelude_fwd`` (one launch): causal 4-tap conv + SiLU of xq, xk [B,T,H,dk]
+    and xv [B,T,H,dv] (taps wq, wk [H*dk, 4], wv [H*dv, 4], fp32), L2 norm of q and k, and the gates
+    g = -exp(A_log) softplus(a + dt_bias) (a [B,T,H] or [B,T,H,G]), beta = sigmoid(b), optional w = sigmoid(c).
+    ``conv_state`` [N, 2 H dk + H dv, 3] fp32 is the cache before each sequence (None: zeros);
+    ``conv_state_out`` (may be ``conv_state`` itself when T == 1) receives the cache after it.
+    Returns a dict with q, k, v, g, beta (, w) and conv_state_out."""
+    _check_dev("xq", xq)
+    dt = xq.dtype
+    for name, t in (("xk", xk), ("xv", xv)):
+        _check_dev(name, t, dt)
+    for name, t in (("wq", wq), ("wk", wk), ("wv", wv), ("a", a), ("A_log", A_log), ("dt_bias", dt_bias), ("b", b),
+                    ("c", c), ("conv_state", conv_state), ("conv_state_out", conv_state_out)):
+        _check_dev(name, t, torch.float32)
+    B, T, H, dk = xq.shape
+    dv = xv.shape[-1]
+    if cu_seqlens is not None:
+        _check_dev("cu_seqlens", cu_seqlens, torch.int32)
+    n_seq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    q = torch.empty_like(xq)
+    k = torch.empty_like(xk)
+    v = torch.empty_like(xv)
+    g = torch.empty_like(a)
+    beta = torch.empty_like(b)
+    w = None if c is None else torch.empty_like(c)
+    gw = 1 if a.dim() == 3 else a.shape[-1]
+    bw = 1 if b.dim() == 3 else b.shape[-1]
+    cw = 0 if c is None else (1 if c.dim() == 3 else c.shape[-1])
+    stream = ctypes.c_void_p(torch.cuda.current_stream(xq.device).cuda_stream)
+    st = load_library().gdn_prelude_fwd(
+        _ptr(xq), _ptr(xk), _ptr(xv), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(conv_state), _ptr(conv_state_out), _ptr(a),
+        _ptr(A_log), _ptr(dt_bias), _ptr(g), gw, _ptr(b), _ptr(beta), bw, _ptr(c), _ptr(w), cw, _ptr(q), _ptr(k),
+        _ptr(v), B, T, H, dk, dv, _dtype_code(xq), float(l2_eps), _ptr(cu_seqlens),
+        0 if cu_seqlens is None else n_seq, stream)
+    _raise_on(st)
+    out = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "conv_state_out": conv_state_out}
+    if w is not None:
+        out["w"] = w
+    return out
+
+
+def output_gate_fwd(o, z, weight, eps=1e-5, y=None):
+    """The mixer's epilogue through ``gdn_output_gate_fwd``: y = o / sqrt(mean(o^2) + eps) * weight * silu(z) over the
+    last axis (dv) of o, z [..., dv] (fp32 or bf16, same dtype); weight [dv] fp32."""
+    _check_dev("o", o)
+    _check_dev("z", z, o.dtype)
+    _check_dev("weight", weight, torch.float32)
+    if z.shape != o.shape or weight.shape != (o.shape[-1],):
+        raise ValueError("o and z must have one shape and weight [dv]")
+    y = torch.empty_like(o) if y is None else y
+    _check_dev("y", y, o.dtype)
+    dv = o.shape[-1]
+    stream = ctypes.c_void_p(torch.cuda.current_stream(o.device).cuda_stream)
+    st = load_library().gdn_output_gate_fwd(_ptr(o), _ptr(z), _ptr(weight), _ptr(y), o.numel() // dv, dv,
+                                            _dtype_code(o), float(eps), stream)
+    _raise_on(st)
+    return y

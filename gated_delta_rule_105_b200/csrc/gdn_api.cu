@@ -1,5 +1,6 @@
 // libgdn C ABI: host-side argument checks, kernel selection and launches.  Every kernel of the library
 // is included here so that they share one device error word without relocatable device code.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -11,6 +12,9 @@
 #include "gdn_prof.cuh"
 #include "gdn_simt.cuh"
 #include "gdn_tc.cuh"
+#include "gdn2_tc.cuh"
+#include "gdn_decode.cuh"
+#include "gdn_prelude.cuh"
 #include "gdn_tc_selftest.cuh"
 
 namespace gdn {
@@ -125,7 +129,7 @@ static gdn_status launch_simt(const FwdParams& p, gdn_dtype dt, gdn_dtype o_dt, 
 static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, gdn_dtype o_dt, void* ws, size_t ws_bytes,
                       cudaStream_t stream) {
     const int choice = g_kernel_choice.load();
-    const bool tc_ok = dt == GDN_BF16 && tc_supported(p, gdn2, o_dt == GDN_F32);
+    const bool tc_ok = dt == GDN_BF16 && (gdn2 ? tc2_supported(p) : tc_supported(p));
     if (choice == GDN_KERNEL_TC && !tc_ok)
         return fail(GDN_ERR_UNSUPPORTED, "the tcgen05 kernel needs bf16 inputs and a supported shape");
     gdn_status st;
@@ -134,7 +138,8 @@ static gdn_status run(const FwdParams& p, bool gdn2, gdn_dtype dt, gdn_dtype o_d
     if (p.n_seq == 0 || p.H == 0) return GDN_OK;
     const bool use_tc = tc_ok && choice != GDN_KERNEL_SIMT;
     if (use_tc) {
-        st = launch_tc(p, gdn2, o_dt == GDN_F32, ws, ws_bytes, err, stream);
+        st = gdn2 ? launch_tc2(p, o_dt == GDN_F32, ws, ws_bytes, err, stream)
+                  : launch_tc(p, o_dt == GDN_F32, ws, ws_bytes, err, stream);
         if (st == GDN_OK) {
             t_last_kernel = GDN_KERNEL_TC;
             return st;
@@ -172,6 +177,69 @@ static gdn_status static_scratch(void** out) {
     return GDN_OK;
 }
 
+// ---- decode step
+static gdn_status check_decode(const void* q, const void* k, const void* v, const float* g, const float* gate,
+                               const float* w, int gates, float scale, const float* state, const void* o, int N, int H,
+                               int dk, int dv, gdn_dtype dt, gdn_dtype o_dt) {
+    t_msg[0] = 0;
+    if (N < 1 || H < 1) return fail(GDN_ERR_INVALID_ARG, "need N >= 1, H >= 1 (got %d, %d)", N, H);
+    if (!q || !k || !v || !g || !gate || !state || !o || (gates == DEC_GDN2 && !w))
+        return fail(GDN_ERR_INVALID_ARG, "a required pointer is NULL");
+    const void* ptrs[] = {q, k, v, g, gate, w, state, o};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return fail(GDN_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", ptr);
+    if (dk != 64 && dk != 128) return fail(GDN_ERR_UNSUPPORTED, "dk must be 64 or 128 (got %d)", dk);
+    if (dv < 64 || dv > 256 || dv % 64 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "dv must be a multiple of 64 in [64, 256] (got %d)", dv);
+    if (dt != GDN_F32 && dt != GDN_BF16) return fail(GDN_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
+    if (o_dt != GDN_F32 && o_dt != dt)
+        return fail(GDN_ERR_UNSUPPORTED, "o_dt must be GDN_F32 or the input dtype (got %d)", (int)o_dt);
+    if (!std::isfinite(scale)) return fail(GDN_ERR_INVALID_ARG, "scale is not finite");
+    if ((long long)N * H > 0x7fffffffLL) return fail(GDN_ERR_INVALID_ARG, "N * H too large");
+    return GDN_OK;
+}
+
+template <typename TIn, typename TOut>
+static gdn_status launch_decode_io(const DecodeParams& p, cudaStream_t stream) {
+    auto kern = p.dk == 64 ? gdn_decode_kernel<TIn, TOut, 64> : gdn_decode_kernel<TIn, TOut, 128>;
+    ProfScope prof(PK_DECODE, stream);
+    kern<<<(unsigned)((long long)p.N * p.H), p.dv, 0, stream>>>(p);
+    prof.done();
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "decode kernel launch: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+static gdn_status decode(const DecodeParams& p, gdn_dtype dt, gdn_dtype o_dt, cudaStream_t stream) {
+    if (dt == GDN_F32) return launch_decode_io<float, float>(p, stream);
+    if (o_dt == GDN_F32) return launch_decode_io<__nv_bfloat16, float>(p, stream);
+    return launch_decode_io<__nv_bfloat16, __nv_bfloat16>(p, stream);
+}
+
+template <typename TIO>
+static gdn_status launch_prelude(const PreludeParams& p, cudaStream_t stream) {
+    const long long rows = (long long)p.B * p.T;
+    const long long tiles = rows > 0 ? (rows + kPreTokens - 1) / kPreTokens : 1;
+    if (tiles > 0x7fffffffLL) return fail(GDN_ERR_INVALID_ARG, "too many tokens for one launch");
+    ProfScope prof(PK_PRELUDE, stream);
+    gdn_prelude_kernel<TIO><<<dim3((unsigned)tiles, p.H, 4), kPreThreads, 0, stream>>>(p);
+    prof.done();
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "prelude kernel launch: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+template <typename TIO>
+static gdn_status launch_out_gate(const OutGateParams& p, cudaStream_t stream) {
+    const long long blocks = std::min<long long>((p.rows + 7) / 8, 148LL * 16);
+    ProfScope prof(PK_OUT_GATE, stream);
+    gdn_output_gate_kernel<TIO><<<(unsigned)std::max<long long>(blocks, 1), 256, 0, stream>>>(p);
+    prof.done();
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "output gate kernel launch: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
 }  // namespace gdn
 
 using namespace gdn;
@@ -183,6 +251,13 @@ size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_se
     if (B < 1 || T < 1 || H < 1 || BT != kChunk || dk != kTcDK || dv < kTcDV || dv % kTcDV != 0 || n_seqs < 0)
         return 0;
     return tc_workspace_bytes(B, T, H, n_seqs);
+}
+
+size_t gdn2_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs) {
+    // the tcgen05 GDN-2 / KDA path keeps one 80.5 KB unit per chunk and head; the SIMT path needs nothing
+    if (B < 1 || T < 1 || H < 1 || BT != kChunk || dk != kTcDK || dv < kTcDV || dv % kTcDV != 0 || n_seqs < 0)
+        return 0;
+    return tc2_workspace_bytes(B, T, H, n_seqs);
 }
 
 gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -210,7 +285,7 @@ gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, co
     p.debug_stall = g_debug_stall.load();
     // The tensor-core path needs tc_workspace_bytes() of scratch; beyond the static array's size the call is
     // refused (callers that can allocate use gdn_chunk_fwd with their own workspace).
-    const bool tc_path = dt == GDN_BF16 && tc_supported(p, false, o_dt == GDN_F32) &&
+    const bool tc_path = dt == GDN_BF16 && tc_supported(p) &&
                          g_kernel_choice.load() != GDN_KERNEL_SIMT && n_seq > 0;
     if (tc_path) {
         const size_t need = tc_workspace_bytes(B, T, H, n_seq);
@@ -236,6 +311,97 @@ gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const flo
     if (st != GDN_OK) return st;
     FwdParams p{q, k, v, g, b, w, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
     return run(p, true, dt, o_dt, workspace, ws_bytes, stream);
+}
+
+gdn_status gdn_kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             float scale, const float* h0, void* o, float* hT, int B, int T, int H, int dk, int dv,
+                             int BT, gdn_dtype dt, gdn_dtype o_dt, const int32_t* cu_seqlens, int n_seqs,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    int n_seq = 0;
+    gdn_status st = check_common(q, k, v, g, beta, nullptr, false, scale, h0, o, hT, B, T, H, dk, dv, BT, dt, o_dt,
+                                 cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
+    if (st != GDN_OK) return st;
+    FwdParams p{q, k, v, g, beta, nullptr, h0, o, hT, cu_seqlens, scale, B, T, H, dk, dv, n_seq};
+    p.kda = 1;
+    return run(p, true, dt, o_dt, workspace, ws_bytes, stream);
+}
+
+gdn_status gdn_decode_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta, float scale,
+                          float* state, void* o, int N, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt,
+                          cudaStream_t stream) {
+    gdn_status st = check_decode(q, k, v, g, beta, nullptr, DEC_GDN, scale, state, o, N, H, dk, dv, dt, o_dt);
+    if (st != GDN_OK) return st;
+    return decode(DecodeParams{q, k, v, g, beta, nullptr, state, o, scale, N, H, dk, dv, DEC_GDN}, dt, o_dt, stream);
+}
+
+gdn_status gdn2_decode_fwd(const void* q, const void* k, const void* v, const float* g, const float* b, const float* w,
+                           float scale, float* state, void* o, int N, int H, int dk, int dv, gdn_dtype dt,
+                           gdn_dtype o_dt, cudaStream_t stream) {
+    gdn_status st = check_decode(q, k, v, g, b, w, DEC_GDN2, scale, state, o, N, H, dk, dv, dt, o_dt);
+    if (st != GDN_OK) return st;
+    return decode(DecodeParams{q, k, v, g, b, w, state, o, scale, N, H, dk, dv, DEC_GDN2}, dt, o_dt, stream);
+}
+
+gdn_status gdn_kda_decode_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                              float scale, float* state, void* o, int N, int H, int dk, int dv, gdn_dtype dt,
+                              gdn_dtype o_dt, cudaStream_t stream) {
+    gdn_status st = check_decode(q, k, v, g, beta, nullptr, DEC_KDA, scale, state, o, N, H, dk, dv, dt, o_dt);
+    if (st != GDN_OK) return st;
+    return decode(DecodeParams{q, k, v, g, beta, nullptr, state, o, scale, N, H, dk, dv, DEC_KDA}, dt, o_dt, stream);
+}
+
+gdn_status gdn_prelude_fwd(const void* xq, const void* xk, const void* xv, const float* wq, const float* wk,
+                           const float* wv, const float* conv_in, float* conv_out, const float* a, const float* A_log,
+                           const float* dt_bias, float* g, int g_width, const float* b, float* beta, int b_width,
+                           const float* c, float* w_gate, int c_width, void* q, void* k, void* v, int B, int T, int H,
+                           int dk, int dv, gdn_dtype dt, float l2_eps, const int32_t* cu_seqlens, int n_seqs,
+                           cudaStream_t stream) {
+    t_msg[0] = 0;
+    if (B < 1 || H < 1 || T < 0) return fail(GDN_ERR_INVALID_ARG, "need B >= 1, H >= 1, T >= 0 (got %d, %d, %d)", B, H, T);
+    if (T > 0 && (!xq || !xk || !xv || !wq || !wk || !wv || !a || !A_log || !dt_bias || !g || !b || !beta || !q ||
+                  !k || !v))
+        return fail(GDN_ERR_INVALID_ARG, "a required pointer is NULL");
+    if ((c == nullptr) != (w_gate == nullptr)) return fail(GDN_ERR_INVALID_ARG, "c and w_gate go together");
+    const void* ptrs[] = {xq, xk, xv, wq, wk, wv, conv_in, conv_out, a, g, b, beta, c, w_gate, q, k, v, cu_seqlens};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return fail(GDN_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", ptr);
+    if (dk != 64 && dk != 128) return fail(GDN_ERR_UNSUPPORTED, "dk must be 64 or 128 (got %d)", dk);
+    if (dv < 64 || dv > 256 || dv % 64 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "dv must be a multiple of 64 in [64, 256] (got %d)", dv);
+    if (g_width < 1 || b_width < 1 || (c && c_width < 1) || g_width > 256 || b_width > 256 || c_width > 256)
+        return fail(GDN_ERR_INVALID_ARG, "gate widths must be in [1, 256]");
+    if (dt != GDN_F32 && dt != GDN_BF16) return fail(GDN_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
+    if (!(l2_eps >= 0.f) || !std::isfinite(l2_eps)) return fail(GDN_ERR_INVALID_ARG, "l2_eps must be >= 0");
+    int n_seq = B;
+    if (cu_seqlens) {
+        if (B != 1) return fail(GDN_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (got %d)", B);
+        if (n_seqs < 1 || n_seqs > 65535) return fail(GDN_ERR_INVALID_ARG, "n_seqs must be in [1, 65535]");
+        n_seq = n_seqs;
+    } else if (n_seqs != 0 && n_seqs != B) {
+        return fail(GDN_ERR_INVALID_ARG, "without cu_seqlens n_seqs must be 0 or B (got %d)", n_seqs);
+    }
+    if (conv_in && conv_in == conv_out && (cu_seqlens || T != 1))
+        return fail(GDN_ERR_INVALID_ARG, "conv_in and conv_out may be one buffer only for single-token steps (T == 1)");
+    PreludeParams p{{xq, xk, xv}, {wq, wk, wv}, conv_in, conv_out, {q, k, v}, a, A_log, dt_bias, g, b, beta, c,
+                    w_gate, cu_seqlens, l2_eps, B, T, H, dk, dv, g_width, b_width, c ? c_width : 0, n_seq};
+    return dt == GDN_F32 ? launch_prelude<float>(p, stream) : launch_prelude<__nv_bfloat16>(p, stream);
+}
+
+gdn_status gdn_output_gate_fwd(const void* o, const void* z, const float* weight, void* y, long long rows, int dv,
+                               gdn_dtype dt, float eps, cudaStream_t stream) {
+    t_msg[0] = 0;
+    if (rows < 0) return fail(GDN_ERR_INVALID_ARG, "rows must be >= 0");
+    if (rows == 0) return GDN_OK;
+    if (!o || !z || !weight || !y) return fail(GDN_ERR_INVALID_ARG, "a required pointer is NULL");
+    const void* ptrs[] = {o, z, weight, y};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return fail(GDN_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", ptr);
+    if (dv < 64 || dv > 256 || dv % 64 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "dv must be a multiple of 64 in [64, 256] (got %d)", dv);
+    if (dt != GDN_F32 && dt != GDN_BF16) return fail(GDN_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(GDN_ERR_INVALID_ARG, "eps must be >= 0");
+    OutGateParams p{o, z, weight, y, rows, dv, eps};
+    return dt == GDN_F32 ? launch_out_gate<float>(p, stream) : launch_out_gate<__nv_bfloat16>(p, stream);
 }
 
 gdn_status gdn_set_kernel(gdn_kernel kernel) {

@@ -31,6 +31,7 @@ struct FwdParams {
     float scale;
     int B, T, H, dk, dv, n_seq;
     int debug_stall;  // diagnostic (gdn_debug_stall): 0 in every ordinary call
+    int kda;          // GDN-2 entry as KDA: beta [B,T,H] is both the erase and the write gate; w unused
 };
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

@@ -129,7 +129,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
                 qv = to_f32(q[tok * DK + i]);
                 if (GDN2) {
                     gv = p.g[tok * DK + i];
-                    bv = p.beta[tok * DK + i];
+                    bv = p.kda ? p.beta[tok] : p.beta[tok * DK + i];
                 }
             }
             sK[r * LDK + i] = kv;
@@ -146,7 +146,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
             if (r < Lc) {
                 const size_t tok = ((size_t)row * T + c0 + r) * H + h;
                 const float vv = to_f32(v[tok * dv + j0 + j]);
-                x = GDN2 ? p.w[tok * dv + j0 + j] * vv : p.beta[tok] * vv;
+                x = (GDN2 && !p.kda ? p.w[tok * dv + j0 + j] : p.beta[tok]) * vv;
             }
             sV[e] = x;
         }

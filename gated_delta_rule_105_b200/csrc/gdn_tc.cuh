@@ -204,35 +204,66 @@ __device__ __forceinline__ void store16(float* S, int r0, int c0, bool tr, int l
     }
 }
 
-// Where the blocks of T go once final: T' = T diag(beta 2^G) as bf16, and T'' = T diag(beta) as a bf16 hi + lo
-// pair, each [r][s] K-major with 128-byte swizzle.  Only the blocks on and below the diagonal are written;
-// the MMAs that read these operands skip the zero blocks above it.
+// Where the blocks of T go once final.  An emitter receives elements of T itself: elem(r, s, x) one element,
+// pair(r, s, x0, x1) the elements (r, s) and (r, s + 1), s even.  Every output is [r][s] K-major with 128-byte
+// swizzle; only the blocks on and below the diagonal are written (the MMAs that read these operands skip the
+// zero blocks above it).
+// GDN: T' = T diag(beta 2^G) as bf16, and T'' = T diag(beta) as a bf16 hi + lo pair.
 struct TEmit {
     uint8_t* tp;
     uint8_t* tpp;
     uint8_t* tppl;
     const float* beta;
     const float* eG;
+    __device__ __forceinline__ void elem(int r, int s, float t) const {
+        using namespace sm100;
+        const float x = t * beta[s];
+        const uint32_t off = sw128(r, s >> 3) + (s & 7) * 2;
+        const __nv_bfloat16 xh = __float2bfloat16_rn(x);
+        *reinterpret_cast<__nv_bfloat16*>(tp + off) = __float2bfloat16_rn(x * eG[s]);
+        *reinterpret_cast<__nv_bfloat16*>(tpp + off) = xh;
+        *reinterpret_cast<__nv_bfloat16*>(tppl + off) = __float2bfloat16_rn(x - __bfloat162float(xh));
+    }
+    __device__ __forceinline__ void pair(int r, int s, float t0, float t1) const {
+        using namespace sm100;
+        const float x0 = t0 * beta[s], x1 = t1 * beta[s + 1];
+        const uint32_t off = sw128(r, s >> 3) + (s & 7) * 2;
+        uint32_t hi, lo;
+        split_pack_bf16(x0, x1, hi, lo);
+        *reinterpret_cast<uint32_t*>(tp + off) = pack_bf16(x0 * eG[s], x1 * eG[s + 1]);
+        *reinterpret_cast<uint32_t*>(tpp + off) = hi;
+        *reinterpret_cast<uint32_t*>(tppl + off) = lo;
+    }
+};
+// GDN-2: T itself as a bf16 hi + lo pair (the gates do not factor out of T).
+struct TEmitPlain {
+    uint8_t* th;
+    uint8_t* tl;
+    __device__ __forceinline__ void elem(int r, int s, float x) const {
+        using namespace sm100;
+        const uint32_t off = sw128(r, s >> 3) + (s & 7) * 2;
+        const __nv_bfloat16 xh = __float2bfloat16_rn(x);
+        *reinterpret_cast<__nv_bfloat16*>(th + off) = xh;
+        *reinterpret_cast<__nv_bfloat16*>(tl + off) = __float2bfloat16_rn(x - __bfloat162float(xh));
+    }
+    __device__ __forceinline__ void pair(int r, int s, float x0, float x1) const {
+        using namespace sm100;
+        const uint32_t off = sw128(r, s >> 3) + (s & 7) * 2;
+        uint32_t hi, lo;
+        split_pack_bf16(x0, x1, hi, lo);
+        *reinterpret_cast<uint32_t*>(th + off) = hi;
+        *reinterpret_cast<uint32_t*>(tl + off) = lo;
+    }
 };
 // Emits sgn * acc, the final 16x16 block (r0, c0) of T held as an mma.sync accumulator.
-__device__ __forceinline__ void emit16(const TEmit& em, int r0, int c0, int lane, const float (&acc)[2][4], float sgn) {
-    using namespace sm100;
+template <class Emit>
+__device__ __forceinline__ void emit16(const Emit& em, int r0, int c0, int lane, const float (&acc)[2][4], float sgn) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh) {
         const int s = c0 + 8 * nh + 2 * t;
-        const float b0 = sgn * em.beta[s], b1 = sgn * em.beta[s + 1];
-        const float e0 = em.eG[s], e1 = em.eG[s + 1];
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const float x0 = acc[nh][2 * hr] * b0, x1 = acc[nh][2 * hr + 1] * b1;
-            const uint32_t off = sw128(r0 + g + 8 * hr, s >> 3) + (s & 7) * 2;
-            uint32_t hi, lo;
-            split_pack_bf16(x0, x1, hi, lo);
-            *reinterpret_cast<uint32_t*>(em.tp + off) = pack_bf16(x0 * e0, x1 * e1);
-            *reinterpret_cast<uint32_t*>(em.tpp + off) = hi;
-            *reinterpret_cast<uint32_t*>(em.tppl + off) = lo;
-        }
+        for (int hr = 0; hr < 2; ++hr) em.pair(r0 + g + 8 * hr, s, sgn * acc[nh][2 * hr], sgn * acc[nh][2 * hr + 1]);
     }
 }
 
@@ -245,7 +276,8 @@ __device__ __forceinline__ void emit16(const TEmit& em, int r0, int c0, int lane
 // (q, p).  Each block product runs on tf32 MMAs, at most two per warp per step.  The lower off-diagonal
 // blocks of A are left intact.  The code is unrolled: it is one chain of dependent shared-memory loads and
 // MMAs, which only unrolling lets the compiler overlap.
-__device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane, uint32_t bar_id, const TEmit& em) {
+template <class Emit>
+__device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane, uint32_t bar_id, const Emit& em) {
     using namespace sm100;
     {
         const int b0 = 16 * wid, c = lane & 15;
@@ -264,16 +296,8 @@ __device__ __forceinline__ void invert_unit_lower64(float* S, int wid, int lane,
         }
         // emit column c of T_ii: lanes 0-15 rows 0-7, lanes 16-31 rows 8-15
         const int s = b0 + c, hr = lane >> 4;
-        const float bs = em.beta[s], es = em.eG[s];
 #pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-            const float x = (hr ? t[8 + rr] : t[rr]) * bs;
-            const uint32_t off = sw128(b0 + 8 * hr + rr, s >> 3) + (s & 7) * 2;
-            const __nv_bfloat16 xh = __float2bfloat16_rn(x);
-            *reinterpret_cast<__nv_bfloat16*>(em.tp + off) = __float2bfloat16_rn(x * es);
-            *reinterpret_cast<__nv_bfloat16*>(em.tpp + off) = xh;
-            *reinterpret_cast<__nv_bfloat16*>(em.tppl + off) = __float2bfloat16_rn(x - __bfloat162float(xh));
-        }
+        for (int rr = 0; rr < 8; ++rr) em.elem(b0 + 8 * hr + rr, s, hr ? t[8 + rr] : t[rr]);
     }
     named_bar_sync(bar_id, 128);
     // T_10 (warp 0) and T_32 (warp 1): X = A_ij T_jj, then T_ij = -T_ii X
@@ -343,6 +367,31 @@ __device__ __forceinline__ bool tc_seq_bounds(const FwdParams& p, int n, int& ro
     return true;
 }
 
+// The (sequence, chunk) that workspace slot `slot` belongs to: the unit's first global token index
+// (row * T + bos + 64 c) goes to *tok0 and its valid rows to *Lc, which stays 0 for a slot no chunk uses.
+__device__ __forceinline__ void wy_unit_of_slot(const FwdParams& p, long long slot, int* tok0, int* Lc,
+                                                unsigned* err) {
+    // the sequence n whose slot range holds `slot`: largest n with wy_slot(n, start_n, 0) <= slot
+    int lo = 0, hi = p.n_seq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        const long long st0 = p.cu_seqlens ? (long long)p.cu_seqlens[mid] : (long long)mid * p.T;
+        if (wy_slot(mid, st0, 0) <= slot) lo = mid;
+        else hi = mid - 1;
+    }
+    int row, bos, eos, c = 0;
+    *Lc = 0;
+    if (tc_seq_bounds(p, lo, row, bos, eos, err)) {
+        const long long start = (long long)row * p.T + bos;
+        const long long cc = slot - wy_slot(lo, start, 0);
+        if (cc >= 0 && cc * kChunk < eos - bos) {
+            c = (int)cc;
+            *Lc = min(kChunk, eos - bos - c * kChunk);
+        }
+        *tok0 = (int)(start + (long long)c * kChunk);
+    }
+}
+
 // ------------------------------------------------------------------------------------------ the WY kernel
 // Shared-memory map (bytes from a 1024-aligned base).  The S1 MMA reads a 128-row A operand per 64-channel
 // panel (rows 0-63: the K tile; rows 64-127: whatever follows it, results unused), so each K panel is
@@ -380,24 +429,8 @@ __global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_cons
     const int h = blockIdx.x % p.H;
 
     if (tid == 0) {
-        // the sequence n whose slot range holds `slot`: largest n with wy_slot(n, start_n, 0) <= slot
-        int lo = 0, hi = p.n_seq - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            const long long st0 = p.cu_seqlens ? (long long)p.cu_seqlens[mid] : (long long)mid * p.T;
-            if (wy_slot(mid, st0, 0) <= slot) lo = mid;
-            else hi = mid - 1;
-        }
-        int row, bos, eos, Lc = 0, c = 0;
-        if (tc_seq_bounds(p, lo, row, bos, eos, err)) {
-            const long long start = (long long)row * p.T + bos;
-            const long long cc = slot - wy_slot(lo, start, 0);
-            if (cc >= 0 && cc * kChunk < eos - bos) {
-                c = (int)cc;
-                Lc = min(kChunk, eos - bos - c * kChunk);
-            }
-            info[1] = (int)(start + (long long)c * kChunk);
-        }
+        int Lc = 0;
+        wy_unit_of_slot(p, slot, &info[1], &Lc, err);
         info[2] = Lc;
         if (Lc > 0) {
             mbar_init(&bars[0], 1);
@@ -963,9 +996,7 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 }
 
 // ------------------------------------------------------------------------------------------ host side
-inline bool tc_supported(const FwdParams& p, bool gdn2, bool /*o_f32*/) {
-    return !gdn2 && p.dk == kTcDK && p.dv % kTcDV == 0 && p.T > 0;
-}
+inline bool tc_supported(const FwdParams& p) { return p.dk == kTcDK && p.dv % kTcDV == 0 && p.T > 0; }
 // Workspace bytes the tcgen05 path needs (the WY kernel's output).
 inline size_t tc_workspace_bytes(int B, int T, int H, int n_seqs) {
     return (size_t)wy_slots(B, T, n_seqs) * (size_t)H * kWyUnit;
@@ -1003,12 +1034,8 @@ inline bool make_map(CUtensorMap* map, const void* base, int d, int H, long long
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-inline gdn_status launch_tc(const FwdParams& p, bool gdn2, bool o_f32, void* ws, size_t ws_bytes, unsigned* err,
+inline gdn_status launch_tc(const FwdParams& p, bool o_f32, void* ws, size_t ws_bytes, unsigned* err,
                             cudaStream_t stream) {
-    if (gdn2) {
-        snprintf(t_tc_msg, sizeof(t_tc_msg), "GDN-2 has no tcgen05 kernel yet");
-        return GDN_ERR_UNSUPPORTED;
-    }
     const size_t need = tc_workspace_bytes(p.B, p.T, p.H, p.n_seq);
     if (!ws || ws_bytes < need) {
         snprintf(t_tc_msg, sizeof(t_tc_msg), "the tcgen05 path needs %zu bytes of workspace (got %zu)", need, ws_bytes);

@@ -89,7 +89,8 @@ def generate(B, T, H, dk, dv, dtype="bf16", seed=0, variant="gdn", h0_std=0.0, n
     """Draw one input set.  Returns a dict of CPU torch tensors plus ``scale`` and ``cu_seqlens``.
 
     q,k [B,T,H,dk] and v [B,T,H,dv] in ``dtype``; GDN: g, beta [B,T,H] fp32; GDN-2: g, b [B,T,H,dk]
-    and w [B,T,H,dv] fp32; h0 [n_seq,H,dk,dv] fp32 or None; cu_seqlens int32 [n_seq+1] or None.
+    and w [B,T,H,dv] fp32; KDA: g [B,T,H,dk] and beta [B,T,H] fp32; h0 [n_seq,H,dk,dv] fp32 or None;
+    cu_seqlens int32 [n_seq+1] or None.
     """
     rng = np.random.Generator(np.random.PCG64(seed))
     fdt = np.float64 if dtype == "f32" else np.float32
@@ -121,6 +122,12 @@ def generate(B, T, H, dk, dv, dtype="bf16", seed=0, variant="gdn", h0_std=0.0, n
         out["g"] = torch.from_numpy(g.astype(np.float32))
         out["b"] = torch.from_numpy(b.astype(np.float32))
         out["w"] = torch.from_numpy(w.astype(np.float32))
+    elif variant == "kda":  # per-channel decay as GDN-2, one scalar beta per token as GDN
+        gn = normal((B, T, H, dk)).astype(np.float64)
+        g = -A[None, None, :, None] * _softplus(gn + dt_bias[None, None, :, None])
+        beta = _sigmoid(normal((B, T, H)).astype(np.float64))
+        out["g"] = torch.from_numpy(g.astype(np.float32))
+        out["beta"] = torch.from_numpy(beta.astype(np.float32))
     else:
         raise ValueError(variant)
     if n_seqs > 0 and cu_seqlens is None:
@@ -142,3 +149,38 @@ def generate(B, T, H, dk, dv, dtype="bf16", seed=0, variant="gdn", h0_std=0.0, n
 
 def generate_workload(w: Workload):
     return generate(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.seed, w.variant, w.h0_std, w.n_seqs, w.len_range)
+
+
+def generate_prelude(B, T, H, dk, dv, dtype="bf16", seed=0, gate_width=1, write_gate=False, conv_state=False,
+                     n_seqs=0, cu_seqlens=None, len_range=(1, 64)):
+    """Inputs of the mixer's prelude (projection outputs, conv taps, gate pre-activations, cache), seeded.
+
+    xq, xk [B,T,H,dk] and xv [B,T,H,dv] ~ N(0,1) in ``dtype``; taps wq, wk [H*dk,4], wv [H*dv,4] ~ N(0, 0.5^2);
+    a [B,T,H(,gate_width)], b [B,T,H(,gate_width)] ~ N(0,1); c [B,T,H,dv] ~ N(0,1) when ``write_gate``;
+    A_log = log U(1,16) and dt_bias ~ N(0, 0.1^2) per head; conv_state [N, 2 H dk + H dv, 3] ~ N(0,1) if asked.
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    A_log = np.log(rng.uniform(1.0, 16.0, size=H)).astype(np.float32)
+    dt_bias = rng.normal(0.0, 0.1, size=H).astype(np.float32)
+    tdt = _torch_dtype(dtype)
+
+    def t(x, dt=torch.float32):
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dt)
+
+    out = {"xq": t(rng.standard_normal((B, T, H, dk)), tdt), "xk": t(rng.standard_normal((B, T, H, dk)), tdt),
+           "xv": t(rng.standard_normal((B, T, H, dv)), tdt),
+           "wq": t(rng.normal(0, 0.5, (H * dk, 4))), "wk": t(rng.normal(0, 0.5, (H * dk, 4))),
+           "wv": t(rng.normal(0, 0.5, (H * dv, 4))),
+           "A_log": t(A_log), "dt_bias": t(dt_bias)}
+    gshape = (B, T, H) if gate_width == 1 else (B, T, H, gate_width)
+    out["a"] = t(rng.standard_normal(gshape))
+    out["b"] = t(rng.standard_normal(gshape))
+    out["c"] = t(rng.standard_normal((B, T, H, dv))) if write_gate else None
+    if n_seqs > 0 and cu_seqlens is None:
+        assert B == 1
+        lens = draw_lengths(rng, n_seqs, T, *len_range)
+        cu_seqlens = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    out["cu_seqlens"] = None if cu_seqlens is None else torch.as_tensor(np.asarray(cu_seqlens, dtype=np.int32))
+    n_seq = B if cu_seqlens is None else len(cu_seqlens) - 1
+    out["conv_state"] = t(rng.standard_normal((n_seq, 2 * H * dk + H * dv, 3))) if conv_state else None
+    return out

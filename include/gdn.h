@@ -16,8 +16,14 @@
  *                   Definition: NVIDIA Gated DeltaNet-2 article (7minutos.es), section "Regla-2 del Delta
  *                   cerrado: dos puertas en lugar de una"; chunk size C = 64 from section "Entrenamiento
  *                   fragmentado".
+ *   gdn_kda_chunk_fwd  KDA (Kimi Delta Attention): GDN-2 with a per-channel decay and one scalar write strength
+ *                   beta_t used as both the erase gate (b_t = beta_t on every key channel) and the write gate
+ *                   (w_t = beta_t on every value column):
+ *                     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,  o_t = scale S_t^T q_t.
+ *                   Definition: the Gated DeltaNet-2 article, section "Regla-2 del Delta cerrado" (when the two
+ *                   gates collapse to the same scalar the rule is KDA exactly).
  *   The read-out o_t and scale = dk^-1/2 are not printed on the pages; o_t = scale S_t^T q_t is the adopted
- *   reading (the same for both operations).
+ *   reading (the same for every operation).
  *
  * Layouts (row-major, contiguous, all device pointers):
  *   q, k        [B, T, H, dk]   dtype `dt` (GDN_F32 or GDN_BF16)
@@ -26,6 +32,7 @@
  *                               rounding (half an ulp, 2^-9 relative, per element) on top of the kernel's error.
  *   GDN:   g, beta  [B, T, H]        fp32; g is the natural-log decay (g <= 0 expected), beta the write strength
  *   GDN-2: g, b     [B, T, H, dk]    fp32 per-channel log-decay and erase gate;  w [B, T, H, dv] fp32 write gate
+ *   KDA:   g [B, T, H, dk] fp32 per-channel log-decay;  beta [B, T, H] fp32
  *   h0, hT      [N, H, dk, dv]  fp32, N = B, or n_seqs with cu_seqlens.  h0 == NULL means zeros;
  *                               hT == NULL means the final state is not written.
  *   cu_seqlens  int32 [n_seqs + 1] or NULL.  With cu_seqlens, B must be 1 and the T tokens of the single
@@ -43,7 +50,9 @@
  * (24 KB per chunk slot and head; slots = ceil(B T / 64) + number of sequences).  The workspace is scratch:
  * its contents are undefined before and after a call, and it must not be shared by calls in flight at the
  * same time.  With a smaller (or NULL) workspace, AUTO runs the SIMT kernel and TC returns
- * GDN_ERR_UNSUPPORTED.
+ * GDN_ERR_UNSUPPORTED.  The GDN-2 and KDA tensor-core path (same shape rule) keeps, per chunk slot and head, an
+ * 80.5 KB unit of state-independent operands (T, W, P and the gate-scaled q and k of the chunk) and needs
+ * gdn2_workspace_bytes() instead.
  *
  * Errors
  *   Arguments are checked on the host before anything is enqueued; a failed check returns
@@ -83,6 +92,10 @@ typedef enum { GDN_KERNEL_AUTO = 0, GDN_KERNEL_SIMT = 1, GDN_KERNEL_TC = 2 } gdn
 /* Bytes of caller-provided device workspace the tensor-core path needs for these sizes (see Workspace
  * above); 0 when only the SIMT kernel can take them (then pass NULL, 0).  n_seqs as for the *_fwd calls. */
 size_t gdn_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs);
+
+/* Bytes of workspace the GDN-2 / KDA tensor-core path needs (see Workspace above); 0 when only the SIMT kernel can
+ * take these sizes. */
+size_t gdn2_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs);
 
 /* Gated delta rule forward; see the header comment for the definition, layouts and errors. */
 gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -131,6 +144,62 @@ gdn_status gdn2_chunk_fwd(const void* q, const void* k, const void* v, const flo
                           const int32_t* cu_seqlens, int n_seqs,
                           void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* KDA forward (GDN-2 with b = w = beta); g is [B,T,H,dk] and beta [B,T,H], both fp32.  Workspace as for
+ * gdn2_chunk_fwd (gdn2_workspace_bytes); arguments, layouts and errors otherwise those of gdn_chunk_fwd. */
+gdn_status gdn_kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             float scale, const float* h0, void* o, float* hT,
+                             int B, int T, int H, int dk, int dv, int BT, gdn_dtype dt, gdn_dtype o_dt,
+                             const int32_t* cu_seqlens, int n_seqs,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Recurrent decode step: one new token for each of N sequences, the state updated in place.  Per (sequence n,
+ * head h) it is one step of the token recurrence (the GatedDeltaNet walkthrough's reference loop, section "Delta
+ * Rule: predict first, then correct"; GDN-2 and KDA as in the Gated DeltaNet-2 article, section "Regla-2 del Delta
+ * cerrado"; decoding with constant memory is the point of the fixed-size state, the article's opening paragraph):
+ *   S <- Diag(exp(g)) S;  u = z - S^T e;  S <- S + k u^T;  o = scale S^T q
+ * with e = beta k, z = beta v (GDN; KDA with a per-channel g), or e = b . k, z = w . v (GDN-2).
+ * Layouts (device, row-major): q, k [N, H, dk] and v [N, H, dv] in `dt`; o [N, H, dv] in `o_dt` (fp32 or `dt`);
+ * state [N, H, dk, dv] fp32, read and overwritten (it is h0 on entry and hT on return).  GDN: g, beta [N, H];
+ * GDN-2: g, b [N, H, dk] and w [N, H, dv]; KDA: g [N, H, dk] and beta [N, H]; all gates fp32.  dk in {64, 128},
+ * dv a multiple of 64 in [64, 256], N >= 1, H >= 1, pointers 16-byte aligned.  Asynchronous on `stream`; the
+ * caller owns every buffer; nothing is allocated.  Errors as for gdn_chunk_fwd (host checks before any launch). */
+gdn_status gdn_decode_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta, float scale,
+                          float* state, void* o, int N, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt,
+                          cudaStream_t stream);
+gdn_status gdn2_decode_fwd(const void* q, const void* k, const void* v, const float* g, const float* b, const float* w,
+                           float scale, float* state, void* o, int N, int H, int dk, int dv, gdn_dtype dt,
+                           gdn_dtype o_dt, cudaStream_t stream);
+gdn_status gdn_kda_decode_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                              float scale, float* state, void* o, int N, int H, int dk, int dv, gdn_dtype dt,
+                              gdn_dtype o_dt, cudaStream_t stream);
+
+/* The mixer's prelude, one launch (GatedDeltaNet walkthrough, sections "Short convolution" and "Gating"; Gated
+ * DeltaNet-2 article, section "Diseno de bloques y modelo hibrido"):
+ *   q = l2norm(silu(conv4(xq))), k = l2norm(silu(conv4(xk))), v = silu(conv4(xv)),
+ *   g = -exp(A_log[h]) * softplus(a + dt_bias[h]),  beta = sigmoid(b),  w_gate = sigmoid(c) (optional),
+ * where conv4 is a depthwise causal convolution per channel, y[t] = w[0] x[t-3] + w[1] x[t-2] + w[2] x[t-1] + w[3] x[t]
+ * (no bias), inputs before a sequence start taken from conv_in (or 0), and l2norm(x) = x / sqrt(sum x^2 + l2_eps) over
+ * each head's channels.  Layouts (device, row-major): xq, xk, q, k [B, T, H, dk] and xv, v [B, T, H, dv] in `dt`;
+ * taps wq, wk [H*dk][4], wv [H*dv][4] fp32; conv_in / conv_out [N][2*H*dk + H*dv][3] fp32 (channels of q, then k, then
+ * v; the three inputs before / at the end of each sequence, oldest first; NULL conv_in means zeros, NULL conv_out
+ * means not written; one buffer for both only when T == 1 and cu_seqlens is NULL, the decode step); a, g [B, T, H,
+ * g_width], b, beta [B, T, H, b_width], c, w_gate [B, T, H, c_width] (c and w_gate both NULL or both given), A_log,
+ * dt_bias [H], all fp32.  cu_seqlens as for gdn_chunk_fwd (sequence starts also restart the convolution).  dk in
+ * {64, 128}, dv a multiple of 64 in [64, 256], widths in [1, 256].  Asynchronous, no allocation; host checks as for
+ * gdn_chunk_fwd. */
+gdn_status gdn_prelude_fwd(const void* xq, const void* xk, const void* xv, const float* wq, const float* wk,
+                           const float* wv, const float* conv_in, float* conv_out, const float* a, const float* A_log,
+                           const float* dt_bias, float* g, int g_width, const float* b, float* beta, int b_width,
+                           const float* c, float* w_gate, int c_width, void* q, void* k, void* v, int B, int T, int H,
+                           int dk, int dv, gdn_dtype dt, float l2_eps, const int32_t* cu_seqlens, int n_seqs,
+                           cudaStream_t stream);
+
+/* The mixer's epilogue (the walkthrough's fused RMSNorm with a Swish gate, data-flow step 5): over each of `rows`
+ * rows of dv channels, y = o / sqrt(mean(o^2) + eps) * weight * silu(z).  o, z, y [rows][dv] in `dt` (device);
+ * weight [dv] fp32, shared by every row.  dv a multiple of 64 in [64, 256].  Asynchronous, no allocation. */
+gdn_status gdn_output_gate_fwd(const void* o, const void* z, const float* weight, void* y, long long rows, int dv,
+                               gdn_dtype dt, float eps, cudaStream_t stream);
+
 /* Selects the kernel family for later calls from any thread (process-wide; default AUTO). */
 gdn_status gdn_set_kernel(gdn_kernel kernel);
 
@@ -166,9 +235,11 @@ const char* gdn_last_error(void);
 gdn_status gdn_debug_umma_selftest(const float* A, const float* B, float* D, int mode, cudaStream_t stream);
 
 /* Per-kernel device timing, a measurement aid (off by default; process-wide).  While enabled, every kernel
- * launch made by gdn_chunk_fwd / gdn2_chunk_fwd is bracketed by two CUDA events recorded on its stream.
+ * launch made by the *_fwd calls is bracketed by two CUDA events recorded on its stream.
  * gdn_profile_take(kernel, &launches, &total_ms) waits for the recorded events of one kernel -- 0: SIMT
- * kernel, 1: tensor-core WY kernel, 2: tensor-core chunk kernel -- returns how many launches they cover and
+ * kernel, 1: tensor-core WY kernel, 2: tensor-core chunk kernel, 3: GDN-2 / KDA prep kernel, 4: GDN-2 / KDA
+ * chunk kernel, 5: decode kernel, 6: prelude kernel, 7: output gate kernel -- returns how many launches they
+ * cover and
  * their summed device time in milliseconds, and forgets them.  Errors: GDN_ERR_INVALID_ARG for an unknown
  * kernel id or NULL outputs, GDN_ERR_CUDA if an event failed. */
 gdn_status gdn_profile_enable(int on);

@@ -46,12 +46,15 @@ def to_dev(inp, device="cuda"):
 
 def run_cuda(inp, variant, output_final_state=True, o_dtype="f32"):
     """Run the C ABI through the binding on device copies of ``inp``; returns (o, hT) on the device."""
-    from gated_delta_rule_105_b200 import gdn2_chunk_fwd, gdn_chunk_fwd
+    from gated_delta_rule_105_b200 import gdn2_chunk_fwd, gdn_chunk_fwd, gdn_kda_chunk_fwd
     d = to_dev(inp)
     odt = {"f32": torch.float32, "bf16": torch.bfloat16}[o_dtype]
     if variant == "gdn":
         return gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"],
                              output_final_state, d["cu_seqlens"], o_dtype=odt)
+    if variant == "kda":
+        return gdn_kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"],
+                                 output_final_state, d["cu_seqlens"], o_dtype=odt)
     return gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["scale"], d["h0"],
                           output_final_state, d["cu_seqlens"], o_dtype=odt)
 
@@ -65,10 +68,21 @@ def seq_spans(inp):
     return [(0, cu[n], cu[n + 1]) for n in range(len(cu) - 1)]
 
 
+def kda_gates(inp):
+    """KDA as GDN-2: the scalar beta broadcast to the erase gate b [..,dk] and the write gate w [..,dv]."""
+    beta = f64(inp["beta"])[..., None]
+    dk, dv = inp["q"].shape[-1], inp["v"].shape[-1]
+    return np.repeat(beta, dk, axis=-1), np.repeat(beta, dv, axis=-1)
+
+
 def run_oracle(inp, variant, threads=8):
     """Whole-input fp64 oracle run (small inputs)."""
     import oracle
     cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].numpy()
+    if variant == "kda":
+        b, w = kda_gates(inp)
+        return oracle.gdn2_fwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]), b, w, inp["scale"],
+                               f64(inp["h0"]), cu_seqlens=cu, threads=threads)
     if variant == "gdn":
         return oracle.gdn_fwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]), f64(inp["beta"]),
                               inp["scale"], f64(inp["h0"]), cu_seqlens=cu, threads=threads)
@@ -96,6 +110,11 @@ def oracle_units(inp, variant, units, threads=8):
         if variant == "gdn":
             o, hT = oracle.gdn_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]), sl(inp["beta"]),
                                    inp["scale"], h0)
+        elif variant == "kda":
+            bt = sl(inp["beta"])[..., None]
+            dk, dv = inp["q"].shape[-1], inp["v"].shape[-1]
+            o, hT = oracle.gdn2_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]),
+                                    np.repeat(bt, dk, axis=-1), np.repeat(bt, dv, axis=-1), inp["scale"], h0)
         else:
             o, hT = oracle.gdn2_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]), sl(inp["b"]),
                                     sl(inp["w"]), inp["scale"], h0)

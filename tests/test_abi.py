@@ -28,7 +28,9 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["gdn_chunk_fwd", "gdn2_chunk_fwd", "gdn_workspace_bytes", "gdn_check_error", "gdn_status_string",
               "gdn_last_error", "gdn_set_kernel", "gdn_last_kernel", "gdn_debug_umma_selftest",
-              "gdn_chunk_fwd_noalloc", "gdn_profile_enable", "gdn_profile_take"]:
+              "gdn_chunk_fwd_noalloc", "gdn_profile_enable", "gdn_profile_take", "gdn2_workspace_bytes",
+              "gdn_kda_chunk_fwd", "gdn_debug_stall", "gdn_decode_fwd", "gdn2_decode_fwd",
+              "gdn_kda_decode_fwd", "gdn_prelude_fwd", "gdn_output_gate_fwd"]:
         assert n in names
 
 
@@ -85,6 +87,42 @@ def test_host_checks_gdn2(lib, kw, status):
     assert call2(lib, **kw) == status
 
 
+def call_kda(lib, **kw):
+    args = dict(q=A, k=A, v=A, g=A, beta=A, B=1, T=64, H=1, dk=128, dv=128, BT=64, dt=1)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    return lib.gdn_kda_chunk_fwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]), vp(args["beta"]),
+                                 0.125, None, vp(A), None, args["B"], args["T"], args["H"], args["dk"], args["dv"],
+                                 args["BT"], args["dt"], 0, None, 0, None, 0, None)
+
+
+@pytest.mark.parametrize("kw,status", [(dict(beta=None), 1), (dict(g=None), 1), (dict(beta=A + 4), 1),
+                                       (dict(dk=32), 2), (dict(BT=16), 2)])
+def test_host_checks_kda(lib, kw, status):
+    assert call_kda(lib, **kw) == status
+    assert lib.gdn_last_error().decode() != ""
+
+
+def call_decode(lib, name="gdn_decode_fwd", **kw):
+    args = dict(q=A, k=A, v=A, g=A, beta=A, state=A, o=A, N=2, H=1, dk=128, dv=128, dt=1, odt=0)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    head = [vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]), vp(args["beta"])]
+    if name == "gdn2_decode_fwd":
+        head.append(vp(A))
+    return getattr(lib, name)(*head, ctypes.c_float(0.125), vp(args["state"]), vp(args["o"]), args["N"], args["H"],
+                              args["dk"], args["dv"], args["dt"], args["odt"], None)
+
+
+@pytest.mark.parametrize("name", ["gdn_decode_fwd", "gdn2_decode_fwd", "gdn_kda_decode_fwd"])
+@pytest.mark.parametrize("kw,status", [(dict(state=None), 1), (dict(state=A + 4), 1), (dict(q=None), 1),
+                                       (dict(N=0), 1), (dict(dk=96), 2), (dict(dv=320), 2), (dict(dv=96), 2),
+                                       (dict(dt=0, odt=1), 2)])
+def test_host_checks_decode(lib, name, kw, status):
+    assert call_decode(lib, name, **kw) == status
+    assert lib.gdn_last_error().decode() != ""
+
+
 def test_status_strings_and_kernel_choice(lib):
     for s in range(6):
         assert lib.gdn_status_string(s).decode() not in ("", "unknown status")
@@ -96,6 +134,10 @@ def test_status_strings_and_kernel_choice(lib):
     assert lib.gdn_workspace_bytes(1, 100, 2, 128, 128, 64, 0) == (2 + 1) * 2 * 24576
     assert lib.gdn_workspace_bytes(4, 4096, 16, 64, 64, 64, 0) == 0  # shapes only the SIMT kernel takes
     assert lib.gdn_workspace_bytes(4, 0, 16, 128, 256, 64, 0) == 0
+    # GDN-2 / KDA: one 82432-byte unit (T hi/lo, -W^T, P, Q', K~, Lambda) per chunk slot and head
+    assert lib.gdn2_workspace_bytes(4, 4096, 16, 128, 128, 64, 0) == (256 + 4) * 16 * 82432
+    assert lib.gdn2_workspace_bytes(1, 100, 2, 128, 256, 64, 0) == (2 + 1) * 2 * 82432
+    assert lib.gdn2_workspace_bytes(4, 4096, 16, 64, 64, 64, 0) == 0
 
 
 def test_binding_refuses_cpu_tensors(lib):

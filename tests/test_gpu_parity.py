@@ -31,8 +31,8 @@ def use_kernel(name):
 
 
 def tc_takes(variant, dk, dv):
-    """Shapes the tcgen05 kernel handles; others are covered by the SIMT kernel."""
-    return variant == "gdn" and dk == 128 and dv % 128 == 0
+    """Shapes the tcgen05 kernels handle (GDN, GDN-2 and KDA alike); others are covered by the SIMT kernel."""
+    return dk == 128 and dv % 128 == 0
 
 
 def _np(x):
@@ -54,7 +54,7 @@ def check(o, hT, ref_o, ref_hT, dtype, odt, what=""):
 SHAPES = [(T, 128, 128) for T in (1, 63, 64, 65, 130, 257)] + [(130, 64, 64), (130, 128, 256), (97, 64, 192)]
 
 
-@pytest.mark.parametrize("variant", ["gdn", "gdn2"])
+@pytest.mark.parametrize("variant", ["gdn", "gdn2", "kda"])
 @pytest.mark.parametrize("dtype,kernel,odt", CASES)
 @pytest.mark.parametrize("T,dk,dv", SHAPES)
 def test_small_shapes(variant, dtype, kernel, odt, T, dk, dv):
@@ -68,7 +68,7 @@ def test_small_shapes(variant, dtype, kernel, odt, T, dk, dv):
     check(o, hT, ro, rh, dtype, odt, f"{variant} {dtype}->{odt} {kernel} T={T} dk={dk} dv={dv}")
 
 
-@pytest.mark.parametrize("variant", ["gdn", "gdn2"])
+@pytest.mark.parametrize("variant", ["gdn", "gdn2", "kda"])
 @pytest.mark.parametrize("dtype,kernel,odt", CASES)
 def test_varlen_with_empty_and_ragged_sequences(variant, dtype, kernel, odt):
     if kernel == "tc" and not tc_takes(variant, 128, 128):
@@ -120,6 +120,36 @@ def test_deterministic_bits(kernel):
     use_kernel(kernel)
     o1, h1 = run_cuda(inp, "gdn")
     o2, h2 = run_cuda(inp, "gdn")
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+@pytest.mark.parametrize("kernel", ["simt", "tc"])
+def test_gdn2_deterministic_bits_and_split_continuation(kernel):
+    inp = generate(2, 300, 2, 128, 128, "bf16", seed=23, variant="gdn2", h0_std=0.02)
+    use_kernel(kernel)
+    o, hT = run_cuda(inp, "gdn2")
+    o2, h2 = run_cuda(inp, "gdn2")
+    assert torch.equal(o, o2) and torch.equal(hT, h2)
+    t0 = 128
+    per_token = ("q", "k", "v", "g", "b", "w")
+    a = {k: (v[:, :t0].contiguous() if k in per_token else v) for k, v in inp.items()}
+    b = {k: (v[:, t0:].contiguous() if k in per_token else v) for k, v in inp.items()}
+    oa, ha = run_cuda(a, "gdn2")
+    b["h0"] = ha.cpu()
+    ob, hb = run_cuda(b, "gdn2")
+    assert relerr(f64(torch.cat([oa, ob], 1)), f64(o)) < 1e-2 and relerr(f64(hb), f64(hT)) < 1e-2
+
+
+@pytest.mark.parametrize("kernel", ["simt", "tc"])
+def test_kda_entry_equals_gdn2_with_broadcast_gates(kernel):
+    """gdn_kda_chunk_fwd is gdn2_chunk_fwd with b = w = beta: the same kernels on the same numbers, bit for bit."""
+    inp = generate(1, 200, 2, 128, 128, "bf16", seed=29, variant="kda", h0_std=0.05)
+    use_kernel(kernel)
+    o1, h1 = run_cuda(inp, "kda")
+    g2 = dict(inp)
+    g2["b"] = inp["beta"][..., None].expand(-1, -1, -1, 128).contiguous()
+    g2["w"] = inp["beta"][..., None].expand(-1, -1, -1, 128).contiguous()
+    o2, h2 = run_cuda(g2, "gdn2")
     assert torch.equal(o1, o2) and torch.equal(h1, h2)
 
 
