@@ -75,6 +75,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_prelude_fwd.restype = i
     lib.gdn_output_gate_fwd.argtypes = [vp, vp, fp, vp, ctypes.c_longlong, i, i, f, vp]
     lib.gdn_output_gate_fwd.restype = i
+    lib.gdn_bwd_workspace_bytes.argtypes = [i] * 7
+    lib.gdn_bwd_workspace_bytes.restype = sz
+    lib.gdn_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [fp] * 6 + [i] * 6 + [i, vp, i, vp, sz, vp]
+    lib.gdn_chunk_bwd.restype = i
     lib.gdn_debug_stall.argtypes = [i]
     lib.gdn_debug_stall.restype = i
     _lib = lib
@@ -133,7 +137,7 @@ def check_error(stream=None) -> None:
 
 PROFILE_KERNELS = {"gdn_simt_fwd_kernel": 0, "gdn_tc_wy_kernel": 1, "gdn_tc_fwd_kernel": 2, "gdn2_tc_prep_kernel": 3,
                    "gdn2_tc_fwd_kernel": 4, "gdn_decode_kernel": 5, "gdn_prelude_kernel": 6,
-                   "gdn_output_gate_kernel": 7}
+                   "gdn_output_gate_kernel": 7, "gdn_bwd_kernels": 8}
 
 
 def profile_enable(on: bool = True) -> None:
@@ -404,3 +408,45 @@ def output_gate_fwd(o, z, weight, eps=1e-5, y=None):
                                             _dtype_code(o), float(eps), stream)
     _raise_on(st)
     return y
+
+
+def bwd_workspace_bytes(B, T, H, dk, dv, BT=64, n_seqs=0) -> int:
+    """Device workspace (bytes) ``gdn_chunk_bwd`` needs: two fp32 states per chunk slot and head."""
+    return int(load_library().gdn_bwd_workspace_bytes(B, T, H, dk, dv, BT, n_seqs))
+
+
+def gdn_chunk_bwd(q, k, v, g, beta, d_o, scale=None, h0=None, dhT=None, cu_seqlens=None, BT=64, workspace=None,
+                  want_dh0=True):
+    """Backward pass of :func:`gdn_chunk_fwd` through ``gdn_chunk_bwd``: the gradients of <d_o, o> + <dhT, hT>.
+
+    d_o [B,T,H,dv] in q's dtype; dhT [N,H,dk,dv] fp32 or None.  Returns a dict of fp32 tensors dq, dk, dv, dg,
+    dbeta and (when ``want_dh0``) dh0.
+    """
+    _check_dev("q", q)
+    dt = q.dtype
+    for name, t in (("k", k), ("v", v), ("d_o", d_o)):
+        _check_dev(name, t, dt)
+    for name, t in (("g", g), ("beta", beta), ("h0", h0), ("dhT", dhT)):
+        _check_dev(name, t, torch.float32)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        _check_dev("cu_seqlens", cu_seqlens, torch.int32)
+    n_seq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    n_seqs = 0 if cu_seqlens is None else n_seq
+    f32 = dict(dtype=torch.float32, device=q.device)
+    out = {"dq": torch.empty((B, T, H, dk), **f32), "dk": torch.empty((B, T, H, dk), **f32),
+           "dv": torch.empty((B, T, H, dv), **f32), "dg": torch.empty((B, T, H), **f32),
+           "dbeta": torch.empty((B, T, H), **f32),
+           "dh0": torch.empty((n_seq, H, dk, dv), **f32) if want_dh0 else None}
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(B, T, H, dk, dv, BT, n_seqs), dtype=torch.uint8, device=q.device)
+    _check_dev("workspace", workspace, torch.uint8)
+    scale = dk ** -0.5 if scale is None else float(scale)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(q.device).cuda_stream)
+    st = load_library().gdn_chunk_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(d_o), _ptr(dhT), _ptr(out["dq"]),
+        _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dh0"]), B, T, H, dk, dv,
+        BT, _dtype_code(q), _ptr(cu_seqlens), n_seqs, _ptr(workspace), workspace.numel(), stream)
+    _raise_on(st)
+    return out

@@ -158,12 +158,6 @@ gdn2_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto qk_off = [](int r, int i) -> uint32_t {
         return (uint32_t)(i >> 6) * 8192u + sm100::sw128(r, (i & 63) >> 3) + (i & 7) * 2;
     };
-    auto ldq = [&](int r, int i) {
-        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(stg + G2Unit::QP + qk_off(r, i)));
-    };
-    auto ldk = [&](int r, int i) {
-        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(stg + G2Unit::KT + qk_off(r, i)));
-    };
     if (p.kda && tid < 64) sBeta[tid] = tid < Lc ? p.beta[(size_t)(tok0 + tid) * H + h] : 0.f;
     for (int e = tid; e < 64 * kAsLd; e += kG2Threads) sA[e] = 0.f;
     const bool landed = mbar_wait(bar, 0, abort_flag, err);
@@ -491,12 +485,16 @@ enum G2Bar : int {
     G_H_FULL = 14,    // h^T MMA done (and K~ read)
     G_H_READY = 15,   // bf16 h^T of the next chunk staged (256)
     G_HM_READY = 16,  // fp32 state re-scaled by the next chunk's decay (256)
-    G_O_FULL = 17,    // O^T MMAs done (and Q', P read)
-    G_O_FREE = 18,    // O^T TMEM read (128)
-    G_DRAIN = 19,     // final commit of the MMA issuer
+    G_O_FULL = 17,    // [2] O^T MMAs of a chunk done (and Q', P read), per O buffer
+    G_O_FREE = 19,    // [2] O^T buffer read by the output warps (128)
+    G_DRAIN = 21,     // final commit of the MMA issuer
 };
 
-constexpr uint32_t T2_U = 0, T2_UF = 64, T2_O1 = 128, T2_O2 = 192, T2_H = 256, T2_COLS = 512;
+// TMEM columns.  The O^T accumulators are double-buffered by chunk parity: the next chunk's O^T MMAs do not wait
+// for the output warps to read the previous chunk's.
+constexpr uint32_t T2_U = 0, T2_UF = 64, T2_H = 256, T2_COLS = 512;
+__device__ __forceinline__ uint32_t t2_o1(int c) { return (c & 1) ? 384u : 128u; }
+__device__ __forceinline__ uint32_t t2_o2(int c) { return (c & 1) ? 448u : 192u; }
 
 // One CTA per (sequence n, head h, block of 128 value columns).  Warp roles: 0 loads (TMA of V, bulk copies of
 // the workspace units); 2 issues every MMA; 4-7 form w . V and store o; 8-15 (two state warpgroups) split U,
@@ -550,7 +548,7 @@ gdn2_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
         for (int b = 0; b < (int)L::N_BARS; ++b) {
             uint32_t cnt = 1;
             if (b == G_U_CONV || b == G_U_RND || b == G_H_READY || b == G_HM_READY) cnt = 256;
-            if (b == G_VW_FULL || b == G_O_FREE) cnt = 128;
+            if (b == G_VW_FULL || b == G_O_FREE || b == G_O_FREE + 1) cnt = 128;
             mbar_init(&bars[b], cnt);
         }
         *abort_flag = 0;
@@ -605,7 +603,7 @@ gdn2_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
                 bulk_load(sm + L::KT, u + G2Unit::KT, 16384, &bars[G_KT_FULL]);
             }
             n_kt++;
-            if (c >= 0 && !warp_wait(&bars[G_O_FULL], c & 1, abort_flag, err)) break;
+            if (c >= 0 && !warp_wait(&bars[G_O_FULL + (c & 1)], (c >> 1) & 1, abort_flag, err)) break;
             if (lane == 0) {
                 mbar_expect_tx(&bars[G_QP_FULL], 16384);
                 bulk_load(sm + L::QP, u + G2Unit::QP, 16384, &bars[G_QP_FULL]);
@@ -682,13 +680,13 @@ gdn2_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
                     umma_bf16_tmem_a(tmem + T2_H, a, d_kt + ks * 128, id_h, 1);
                 }
                 umma_commit(&bars[G_H_FULL]);
-                // O1^T = h^T Q'^T
-                if (c >= 1 && !mbar_wait(&bars[G_O_FREE], (c - 1) & 1, abort_flag, err)) break;
+                // O1^T = h^T Q'^T, into the O buffer of this chunk's parity (read out two chunks ago)
+                if (c >= 2 && !mbar_wait(&bars[G_O_FREE + st], ((c - 2) >> 1) & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[G_QP_FULL], c & 1, abort_flag, err)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_bf16(tmem + T2_O1, d_ht + (kk >> 2) * 1024 + (kk & 3) * 2,
+                    umma_bf16(tmem + t2_o1(c), d_ht + (kk >> 2) * 1024 + (kk & 3) * 2,
                               d_qp + (kk >> 2) * 512 + (kk & 3) * 2, id_o, kk > 0);
                 // O2^T = U^T P^T on kind::tf32 (P lower triangular: k-step ks8 of 8 tokens reaches r >= 16 (ks8/2))
                 if (!mbar_wait(&bars[G_P_FULL], c & 1, abort_flag, err)) break;
@@ -699,9 +697,9 @@ gdn2_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
                     const int r0 = 16 * (ks8 >> 1);
                     const uint64_t b = desc_k_sw128(sbase + L::P + ((ks8 & 4) ? 8192 : 0)) +
                                        ((r0 * 128 + (ks8 & 3) * 32) >> 4);
-                    umma_tf32_tmem_a(tmem + T2_O2 + r0, tmem + T2_U + 8 * ks8, b, id_o2 - (r0 >> 4) * n16, ks8 > 0);
+                    umma_tf32_tmem_a(tmem + t2_o2(c) + r0, tmem + T2_U + 8 * ks8, b, id_o2 - (r0 >> 4) * n16, ks8 > 0);
                 }
-                umma_commit(&bars[G_O_FULL]);
+                umma_commit(&bars[G_O_FULL + st]);
             }
             umma_commit(&bars[G_DRAIN]);
             drain_wait(&bars[G_DRAIN], 0);
@@ -768,19 +766,19 @@ gdn2_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
             if (k >= 1) {
                 const int c = k - 1;
                 const int Lc = min(kChunk, eos - bos - c * kChunk);
-                warp_wait(&bars[G_O_FULL], c & 1, abort_flag, err);
+                warp_wait(&bars[G_O_FULL + (c & 1)], (c >> 1) & 1, abort_flag, err);
                 tc_fence_after();
                 const size_t tok0 = (size_t)(seq_start + (long long)c * kChunk);
                 size_t off = (tok0 * H + h) * (size_t)dv + j0 + t;
 #pragma unroll 1
                 for (int r8 = 0; r8 < 64; r8 += 8) {
                     float v1[8], v2[8];
-                    tmem_ld8(taddr(tmem, lane_base, T2_O1 + r8), v1);
-                    tmem_ld8(taddr(tmem, lane_base, T2_O2 + r8), v2);
+                    tmem_ld8(taddr(tmem, lane_base, t2_o1(c) + r8), v1);
+                    tmem_ld8(taddr(tmem, lane_base, t2_o2(c) + r8), v2);
                     tmem_wait_ld();
                     if (r8 == 56) {
                         tc_fence_before();
-                        mbar_arrive(&bars[G_O_FREE]);
+                        mbar_arrive(&bars[G_O_FREE + (c & 1)]);
                     }
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {

@@ -15,6 +15,7 @@
 #include "gdn2_tc.cuh"
 #include "gdn_decode.cuh"
 #include "gdn_prelude.cuh"
+#include "gdn_bwd.cuh"
 #include "gdn_tc_selftest.cuh"
 
 namespace gdn {
@@ -203,7 +204,7 @@ template <typename TIn, typename TOut>
 static gdn_status launch_decode_io(const DecodeParams& p, cudaStream_t stream) {
     auto kern = p.dk == 64 ? gdn_decode_kernel<TIn, TOut, 64> : gdn_decode_kernel<TIn, TOut, 128>;
     ProfScope prof(PK_DECODE, stream);
-    kern<<<(unsigned)((long long)p.N * p.H), p.dv, 0, stream>>>(p);
+    kern<<<(unsigned)((long long)p.N * p.H), p.dv / 4 * kDecRowGroups, 0, stream>>>(p);
     prof.done();
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "decode kernel launch: %s", cudaGetErrorString(e));
@@ -221,8 +222,12 @@ static gdn_status launch_prelude(const PreludeParams& p, cudaStream_t stream) {
     const long long rows = (long long)p.B * p.T;
     const long long tiles = rows > 0 ? (rows + kPreTokens - 1) / kPreTokens : 1;
     if (tiles > 0x7fffffffLL) return fail(GDN_ERR_INVALID_ARG, "too many tokens for one launch");
+    const size_t smem = prelude_smem_bytes(std::max(p.dk, p.dv));
+    cudaError_t e0 = cudaFuncSetAttribute(gdn_prelude_kernel<TIO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)smem);
+    if (e0 != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e0));
     ProfScope prof(PK_PRELUDE, stream);
-    gdn_prelude_kernel<TIO><<<dim3((unsigned)tiles, p.H, 4), kPreThreads, 0, stream>>>(p);
+    gdn_prelude_kernel<TIO><<<dim3((unsigned)tiles, p.H, 3), kPreThreads, smem, stream>>>(p);
     prof.done();
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "prelude kernel launch: %s", cudaGetErrorString(e));
@@ -237,6 +242,37 @@ static gdn_status launch_out_gate(const OutGateParams& p, cudaStream_t stream) {
     prof.done();
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "output gate kernel launch: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+// ---- backward
+inline size_t bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int n_seqs) {
+    return 2 * (size_t)wy_slots(B, T, n_seqs) * H * (size_t)dk * dv * sizeof(float);
+}
+
+template <typename TIn, int DK>
+static gdn_status launch_bwd_dk(const FwdParams& fp, const BwdParams& bp, unsigned* err, cudaStream_t stream) {
+    // (1) the state at every chunk start, from the SIMT forward (no o written)
+    gdn_status st = launch_simt_dk<TIn, float, DK, false>(fp, err, stream);
+    if (st != GDN_OK) return st;
+    ProfScope prof(PK_BWD, stream);
+    // (2) the state cotangent, chunk by chunk backwards
+    auto kdh = gdn_bwd_dh_kernel<TIn, DK>;
+    cudaError_t e = cudaFuncSetAttribute(kdh, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwDhSmem<DK>::bytes);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    kdh<<<dim3(bp.vdim / BwDhSmem<DK>::DVT, bp.H, bp.n_seq), kBwThreads, BwDhSmem<DK>::bytes, stream>>>(bp, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward state kernel: %s", cudaGetErrorString(e));
+    // (3) every input gradient, all chunks at once
+    const long long grid = wy_slots(bp.B, bp.T, bp.n_seq) * bp.H;
+    if (grid > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "too many chunks for one launch");
+    auto kc = gdn_bwd_chunk_kernel<TIn, DK>;
+    e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwChunkSmem<DK>::bytes);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    if (grid > 0) kc<<<(unsigned)grid, kBwThreads, BwChunkSmem<DK>::bytes, stream>>>(bp, err);
+    prof.done();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward chunk kernel: %s", cudaGetErrorString(e));
     return GDN_OK;
 }
 
@@ -402,6 +438,45 @@ gdn_status gdn_output_gate_fwd(const void* o, const void* z, const float* weight
     if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(GDN_ERR_INVALID_ARG, "eps must be >= 0");
     OutGateParams p{o, z, weight, y, rows, dv, eps};
     return dt == GDN_F32 ? launch_out_gate<float>(p, stream) : launch_out_gate<__nv_bfloat16>(p, stream);
+}
+
+size_t gdn_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs) {
+    if (B < 1 || T < 0 || H < 1 || BT != kChunk || (dk != 64 && dk != 128) || dv < 64 || dv > 256 || dv % 64 != 0 ||
+        n_seqs < 0)
+        return 0;
+    return bwd_workspace_bytes(B, T, H, dk, dv, n_seqs);
+}
+
+gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta, float scale,
+                         const float* h0, const void* d_o, const float* dhT, float* dq, float* dk, float* dv,
+                         float* dg, float* dbeta, float* dh0, int B, int T, int H, int dk_, int dv_, int BT,
+                         gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs, void* workspace, size_t ws_bytes,
+                         cudaStream_t stream) {
+    int n_seq = 0;
+    gdn_status st = check_common(q, k, v, g, beta, nullptr, false, scale, h0, d_o, dhT, B, T, H, dk_, dv_, BT, dt, dt,
+                                 cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
+    if (st != GDN_OK) return st;
+    if (T > 0 && (!dq || !dk || !dv || !dg || !dbeta))
+        return fail(GDN_ERR_INVALID_ARG, "a gradient output (dq, dk, dv, dg, dbeta) is NULL");
+    const void* outs[] = {dq, dk, dv, dg, dbeta, dh0};
+    for (const void* ptr : outs)
+        if (ptr && !aligned16(ptr)) return fail(GDN_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", ptr);
+    const size_t need = bwd_workspace_bytes(B, T, H, dk_, dv_, cu_seqlens ? n_seq : 0);
+    if (!workspace || ws_bytes < need)
+        return fail(GDN_ERR_INVALID_ARG, "the backward pass needs %zu bytes of workspace (got %zu)", need, ws_bytes);
+    gdn_status es;
+    unsigned* err = err_word_ptr(&es);
+    if (!err) return es;
+    float* hc = static_cast<float*>(workspace);
+    float* dhc = hc + need / 2 / sizeof(float);
+    FwdParams fp{q, k, v, g, beta, nullptr, h0, nullptr, nullptr, cu_seqlens, scale, B, T, H, dk_, dv_, n_seq};
+    fp.h_chunks = hc;
+    BwdParams bp{q, k, v, g, beta, d_o, dhT, hc, dhc, dq, dk, dv, dg, dbeta, dh0, cu_seqlens, scale,
+                 B, T, H, dk_, dv_, n_seq};
+    if (dt == GDN_F32)
+        return dk_ == 64 ? launch_bwd_dk<float, 64>(fp, bp, err, stream) : launch_bwd_dk<float, 128>(fp, bp, err, stream);
+    return dk_ == 64 ? launch_bwd_dk<__nv_bfloat16, 64>(fp, bp, err, stream)
+                     : launch_bwd_dk<__nv_bfloat16, 128>(fp, bp, err, stream);
 }
 
 gdn_status gdn_set_kernel(gdn_kernel kernel) {

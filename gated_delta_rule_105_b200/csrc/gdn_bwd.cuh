@@ -1,0 +1,552 @@
+// Backward pass (reverse mode) of the chunked gated delta rule, GDN (scalar gates): fp32 on CUDA cores.
+//
+// The forward per chunk of C = 64 tokens (the WY form of the SIMT forward kernel; GatedDeltaNet data-flow
+// walkthrough, yfxerp.com/news/367755, section "Chunked parallelism", which also names the full backward --
+// gradients of q, k, v, beta and g), with Gamma_rs = 2^(G_r - G_s), F = 2^G, f = 2^(G_last - G), gamma = 2^(G_last):
+//   A = strict_lower(diag(beta) (K K^T) . Gamma),  T = (I + A)^-1,  P = lower((Q K^T) . Gamma)
+//   X = diag(beta) V - diag(beta F) K h,  U = T X
+//   O = scale (diag(F) Q h + P U),  h' = gamma h + (diag(f) K)^T U
+// Given the cotangents dO of the output and dh' of the chunk's end state:
+//   dU = scale P^T dO + diag(f) K dh'      dX = T^T dU
+//   dh = scale (diag(F) Q)^T dO + gamma dh' - K^T diag(beta F) dX       (the state recurrence, chunk to chunk)
+//   dT = dU X^T  ->  dA = -T^T dT T^T (strictly lower part),   dP = scale dO U^T (lower part)
+// and from A, P, X, F, f, gamma to q, k, v, beta and the chunk-local cumulative gate; dg is the reverse cumulative
+// sum of the gate's gradient inside the chunk.
+//
+// Three kernels: (1) the SIMT forward kernel, asked to write the state at every chunk start (FwdParams::h_chunks);
+// (2) gdn_bwd_dh_kernel walks each sequence's chunks backwards with the state cotangent dh in shared memory (one
+// CTA per (sequence, head, 32 value columns), the value columns of dh never mix) and writes dh' of every chunk;
+// (3) gdn_bwd_chunk_kernel forms every input gradient of one (chunk, head), all chunks at once, walking the value
+// columns in tiles of 16 and keeping the key-side sums in registers.
+#pragma once
+
+#include "gdn_common.cuh"
+
+namespace gdn {
+
+constexpr int kBwThreads = 256;
+
+struct BwdParams {
+    const void* q;            // [B,T,H,dk]   (dtype TIn)
+    const void* k;
+    const void* v;            // [B,T,H,dv]
+    const float* g;           // [B,T,H]
+    const float* beta;        // [B,T,H]
+    const void* dout;         // dO [B,T,H,dv] (dtype TIn)
+    const float* dhT;         // [N,H,dk,dv] or null
+    const float* h_chunks;    // [slot][H][dk][dv]: the state at each chunk's start (from the forward)
+    float* dh_chunks;         // [slot][H][dk][dv]: the cotangent of the state at each chunk's end
+    float* dq;                // [B,T,H,dk] fp32
+    float* dk;
+    float* dv;                // [B,T,H,dv] fp32
+    float* dg;                // [B,T,H] fp32
+    float* dbeta;             // [B,T,H] fp32
+    float* dh0;               // [N,H,dk,dv] fp32 or null
+    const int32_t* cu_seqlens;
+    float scale;
+    int B, T, H, kdim, vdim, n_seq;
+};
+
+// Shared per-chunk quantities of the backward kernels (pointers into shared memory).
+template <int DK>
+struct BwChunk {
+    static constexpr int LDK = DK + 1, LDT = kChunk + 1;
+    float* K;      // [64][LDK]
+    float* Q;      // [64][LDK]
+    float* Gm;     // Gamma [64][LDT], 0 above the diagonal
+    float* T;      // (I + A)^-1 [64][LDT]
+    float* P;      // [64][LDT], 0 above the diagonal
+    float* A;      // scratch [64][LDT] (A while inverting)
+    double* G;     // [64] log2(e) * chunk-local cumsum of g
+    float* beta;   // [64]
+    float* F;      // [64] 2^G
+    float* f;      // [64] 2^(G_last - G)
+    float* gamma;  // [1]
+};
+
+// Loads one chunk (rows past Lc zero: k = q = beta = g = 0) and forms G, F, f, gamma, Gamma, P and T.
+template <typename TIn, int DK>
+__device__ void bw_chunk_prep(const BwChunk<DK>& c, const BwdParams& p, size_t tok0, int h, int Lc) {
+    constexpr int LDK = BwChunk<DK>::LDK, LDT = BwChunk<DK>::LDT, NT = kBwThreads;
+    const int tid = threadIdx.x, H = p.H;
+    const TIn* q = static_cast<const TIn*>(p.q);
+    const TIn* k = static_cast<const TIn*>(p.k);
+    __syncthreads();  // the previous user of these buffers is done
+    for (int e = tid; e < kChunk * DK; e += NT) {
+        const int r = e / DK, i = e % DK;
+        float kv = 0.f, qv = 0.f;
+        if (r < Lc) {
+            const size_t idx = ((tok0 + r) * H + h) * DK + i;
+            kv = to_f32(k[idx]);
+            qv = to_f32(q[idx]);
+        }
+        c.K[r * LDK + i] = kv;
+        c.Q[r * LDK + i] = qv;
+    }
+    if (tid < kChunk) {
+        const bool ok = tid < Lc;
+        c.beta[tid] = ok ? p.beta[(tok0 + tid) * H + h] : 0.f;
+        c.G[tid] = ok ? (double)p.g[(tok0 + tid) * H + h] : 0.0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double acc = 0.0;
+        for (int r = 0; r < kChunk; ++r) {
+            acc += c.G[r];
+            c.G[r] = acc * kLog2eD;
+        }
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        c.F[tid] = exp2f((float)c.G[tid]);
+        c.f[tid] = exp2f((float)(c.G[kChunk - 1] - c.G[tid]));
+        if (tid == 0) c.gamma[0] = exp2f((float)c.G[kChunk - 1]);
+    }
+    for (int e = tid; e < kChunk * kChunk; e += NT) {
+        const int r = e / kChunk, s = e % kChunk;
+        float gm = 0.f, a = 0.f, pp = 0.f;
+        if (s <= r) {
+            float kk = 0.f, qk = 0.f;
+            for (int i = 0; i < DK; ++i) {
+                const float ks = c.K[s * LDK + i];
+                kk = fmaf(c.K[r * LDK + i], ks, kk);
+                qk = fmaf(c.Q[r * LDK + i], ks, qk);
+            }
+            gm = exp2f((float)(c.G[r] - c.G[s]));
+            a = s < r ? c.beta[r] * gm * kk : 0.f;
+            pp = gm * qk;
+        }
+        c.Gm[r * LDT + s] = gm;
+        c.A[r * LDT + s] = a;
+        c.P[r * LDT + s] = pp;
+    }
+    __syncthreads();
+    // T = (I + A)^-1 row by row, four threads per column (adjacent lanes) splitting each row's sum
+    {
+        const int col = tid >> 2, part = tid & 3;
+        for (int r = 0; r < kChunk; ++r) {
+            float acc = 0.f;
+            for (int s = col + part; s < r; s += 4) acc = fmaf(c.A[r * LDT + s], c.T[s * LDT + col], acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (part == 0) c.T[r * LDT + col] = r < col ? 0.f : (r == col ? 1.f : -acc);
+            __syncthreads();
+        }
+    }
+}
+
+// Sequence bounds (row, first token, end) of sequence n; false (and the error word) for a bad cu_seqlens entry.
+__device__ __forceinline__ bool bw_seq_bounds(const BwdParams& p, int n, int& row, int& bos, int& eos, unsigned* err) {
+    if (p.cu_seqlens) {
+        row = 0;
+        bos = p.cu_seqlens[n];
+        eos = p.cu_seqlens[n + 1];
+        if (bos < 0 || eos < bos || eos > p.T) {
+            if (threadIdx.x == 0) atomicOr(err, kErrSeqlens);
+            return false;
+        }
+    } else {
+        row = n;
+        bos = 0;
+        eos = p.T;
+    }
+    return true;
+}
+
+template <int DK>
+struct BwDhSmem {  // 4-byte words
+    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 32, LDV = DVT + 1;
+    static constexpr int oK = 0, oQ = oK + kChunk * LDK, oGm = oQ + kChunk * LDK, oT = oGm + kChunk * LDT;
+    static constexpr int oP = oT + kChunk * LDT, oA = oP + kChunk * LDT;
+    static constexpr int oG = oA + kChunk * LDT;  // double [64]
+    static constexpr int oBeta = oG + 2 * kChunk, oF = oBeta + kChunk, of = oF + kChunk, oGam = of + kChunk;
+    static constexpr int oDh = oGam + 4;          // dh [DK][LDV]
+    static constexpr int oDo = oDh + DK * LDV;    // dO [64][LDV]
+    static constexpr int oDu = oDo + kChunk * LDV;
+    static constexpr int oDx = oDu + kChunk * LDV;
+    static constexpr int total = oDx + kChunk * LDV;
+    static constexpr size_t bytes = sizeof(float) * (size_t)total;
+};
+
+// (2) One CTA per (sequence, head, 32 value columns): the state cotangent, walked from the last chunk to the first.
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams p, unsigned* err) {
+    using L = BwDhSmem<DK>;
+    constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBwThreads;
+    extern __shared__ __align__(16) float bsm[];
+    const BwChunk<DK> c{bsm + L::oK, bsm + L::oQ, bsm + L::oGm, bsm + L::oT, bsm + L::oP, bsm + L::oA,
+                        reinterpret_cast<double*>(bsm + L::oG), bsm + L::oBeta, bsm + L::oF, bsm + L::of,
+                        bsm + L::oGam};
+    float* sDh = bsm + L::oDh;
+    float* sDo = bsm + L::oDo;
+    float* sDu = bsm + L::oDu;
+    float* sDx = bsm + L::oDx;
+    const int tid = threadIdx.x, j0 = blockIdx.x * DVT, h = blockIdx.y, n = blockIdx.z;
+    const int H = p.H, dv = p.vdim;
+    int row, bos, eos;
+    if (!bw_seq_bounds(p, n, row, bos, eos, err)) return;
+    const long long start = (long long)row * p.T + bos;
+    const size_t state_base = ((size_t)n * H + h) * DK * (size_t)dv + j0;
+    for (int e = tid; e < DK * DVT; e += NT) {
+        const int i = e / DVT, j = e % DVT;
+        sDh[i * LDV + j] = p.dhT ? p.dhT[state_base + (size_t)i * dv + j] : 0.f;
+    }
+    const TIn* dout = static_cast<const TIn*>(p.dout);
+    const int nc = (eos - bos + kChunk - 1) / kChunk;
+    for (int ci = nc - 1; ci >= 0; --ci) {
+        const int Lc = min(kChunk, eos - bos - ci * kChunk);
+        const size_t tok0 = (size_t)(start + (long long)ci * kChunk);
+        bw_chunk_prep<TIn, DK>(c, p, tok0, h, Lc);
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int r = e / DVT, j = e % DVT;
+            sDo[r * LDV + j] = r < Lc ? to_f32(dout[((tok0 + r) * H + h) * dv + j0 + j]) : 0.f;
+        }
+        // dh' of this chunk (its end state's cotangent) for the gradient kernel
+        float* dh_out = p.dh_chunks + ((size_t)wy_slot(n, start, ci) * H + h) * DK * (size_t)dv + j0;
+        for (int e = tid; e < DK * DVT; e += NT) {
+            const int i = e / DVT, j = e % DVT;
+            dh_out[(size_t)i * dv + j] = sDh[i * LDV + j];
+        }
+        __syncthreads();
+        // dU = scale P^T dO + diag(f) K dh'
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int s = e / DVT, j = e % DVT;
+            float acc = 0.f;
+            for (int r = s; r < kChunk; ++r) acc = fmaf(c.P[r * LDT + s], sDo[r * LDV + j], acc);
+            float kd = 0.f;
+            for (int i = 0; i < DK; ++i) kd = fmaf(c.K[s * LDK + i], sDh[i * LDV + j], kd);
+            sDu[s * LDV + j] = p.scale * acc + c.f[s] * kd;
+        }
+        __syncthreads();
+        // dX = T^T dU
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int s = e / DVT, j = e % DVT;
+            float acc = 0.f;
+            for (int r = s; r < kChunk; ++r) acc = fmaf(c.T[r * LDT + s], sDu[r * LDV + j], acc);
+            sDx[s * LDV + j] = acc;
+        }
+        __syncthreads();
+        // dh = scale (diag(F) Q)^T dO + gamma dh' - K^T diag(beta F) dX
+        float nd[DK * DVT / NT];
+        const float gam = c.gamma[0];
+#pragma unroll
+        for (int m = 0; m < DK * DVT / NT; ++m) {
+            const int e = tid + m * NT, i = e / DVT, j = e % DVT;
+            float a = 0.f;
+            for (int r = 0; r < kChunk; ++r) {
+                a = fmaf(p.scale * c.F[r] * c.Q[r * LDK + i], sDo[r * LDV + j], a);
+                a = fmaf(-c.beta[r] * c.F[r] * c.K[r * LDK + i], sDx[r * LDV + j], a);
+            }
+            nd[m] = a + gam * sDh[i * LDV + j];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < DK * DVT / NT; ++m) {
+            const int e = tid + m * NT;
+            sDh[(e / DVT) * LDV + e % DVT] = nd[m];
+        }
+    }
+    __syncthreads();
+    if (p.dh0)
+        for (int e = tid; e < DK * DVT; e += NT) {
+            const int i = e / DVT, j = e % DVT;
+            p.dh0[state_base + (size_t)i * dv + j] = sDh[i * LDV + j];
+        }
+}
+
+template <int DK>
+struct BwChunkSmem {  // 4-byte words
+    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 16, LDV = DVT + 1;
+    static constexpr int oK = 0, oQ = oK + kChunk * LDK, oGm = oQ + kChunk * LDK, oT = oGm + kChunk * LDT;
+    static constexpr int oP = oT + kChunk * LDT, oA = oP + kChunk * LDT;  // A, then dT
+    static constexpr int odP = oA + kChunk * LDT;
+    static constexpr int oG = odP + kChunk * LDT;  // double [64]
+    static constexpr int oBeta = oG + 2 * kChunk, oF = oBeta + kChunk, of = oF + kChunk, oGam = of + kChunk;
+    static constexpr int odBeta = oGam + 4, odF = odBeta + kChunk, odf = odF + kChunk, odGn = odf + kChunk;
+    static constexpr int odGam = odGn + kChunk;
+    static constexpr int oH = odGam + 4;          // h tile [DK][LDV]
+    static constexpr int oDH = oH + DK * LDV;     // dh' tile [DK][LDV]
+    static constexpr int oV = oDH + DK * LDV;     // [64][LDV] tiles: V, dO, Kh, Qh, Kdh, X, U, dU, dX
+    static constexpr int oDO = oV + kChunk * LDV, oKh = oDO + kChunk * LDV, oQh = oKh + kChunk * LDV;
+    static constexpr int oKd = oQh + kChunk * LDV, oX = oKd + kChunk * LDV, oU = oX + kChunk * LDV;
+    static constexpr int oDU = oU + kChunk * LDV, oDX = oDU + kChunk * LDV;
+    static constexpr int total = oDX + kChunk * LDV;
+    static constexpr size_t bytes = sizeof(float) * (size_t)total;
+};
+
+// (3) One CTA per (chunk slot, head): every input gradient of the chunk.
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdParams p, unsigned* err) {
+    using L = BwChunkSmem<DK>;
+    constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBwThreads;
+    constexpr int ACC = DK / 4;  // key channels per thread in the register sums (row tid / 4)
+    extern __shared__ __align__(16) float bsm[];
+    const BwChunk<DK> c{bsm + L::oK, bsm + L::oQ, bsm + L::oGm, bsm + L::oT, bsm + L::oP, bsm + L::oA,
+                        reinterpret_cast<double*>(bsm + L::oG), bsm + L::oBeta, bsm + L::oF, bsm + L::of,
+                        bsm + L::oGam};
+    float* sdT = bsm + L::oA;
+    float* sdP = bsm + L::odP;
+    float* sdBeta = bsm + L::odBeta;
+    float* sdF = bsm + L::odF;
+    float* sdf = bsm + L::odf;
+    float* sdGn = bsm + L::odGn;
+    float* sdGam = bsm + L::odGam;
+    float* sH = bsm + L::oH;
+    float* sDH = bsm + L::oDH;
+    float* sV = bsm + L::oV;
+    float* sDO = bsm + L::oDO;
+    float* sKh = bsm + L::oKh;
+    float* sQh = bsm + L::oQh;
+    float* sKd = bsm + L::oKd;
+    float* sX = bsm + L::oX;
+    float* sU = bsm + L::oU;
+    float* sDU = bsm + L::oDU;
+    float* sDX = bsm + L::oDX;
+    __shared__ int info[4];
+    const int tid = threadIdx.x, H = p.H, dv = p.vdim;
+    const long long slot = blockIdx.x / H;
+    const int h = blockIdx.x % H;
+    if (tid == 0) {
+        // the (sequence, chunk) of this slot: largest n with wy_slot(n, start_n, 0) <= slot
+        int lo = 0, hi = p.n_seq - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            const long long st0 = p.cu_seqlens ? (long long)p.cu_seqlens[mid] : (long long)mid * p.T;
+            if (wy_slot(mid, st0, 0) <= slot) lo = mid;
+            else hi = mid - 1;
+        }
+        int row, bos, eos, Lc = 0;
+        if (bw_seq_bounds(p, lo, row, bos, eos, err)) {
+            const long long start = (long long)row * p.T + bos;
+            const long long cc = slot - wy_slot(lo, start, 0);
+            if (cc >= 0 && cc * kChunk < eos - bos) {
+                Lc = min(kChunk, (int)(eos - bos - cc * kChunk));
+                info[0] = (int)(start + cc * kChunk);
+            }
+        }
+        info[1] = Lc;
+    }
+    __syncthreads();
+    const int Lc = info[1];
+    if (Lc == 0) return;
+    const size_t tok0 = (size_t)info[0];
+    const TIn* vin = static_cast<const TIn*>(p.v);
+    const TIn* dout = static_cast<const TIn*>(p.dout);
+    const float* hc = p.h_chunks + ((size_t)slot * H + h) * DK * (size_t)dv;
+    const float* dhc = p.dh_chunks + ((size_t)slot * H + h) * DK * (size_t)dv;
+
+    bw_chunk_prep<TIn, DK>(c, p, tok0, h, Lc);
+    for (int e = tid; e < kChunk * LDT; e += NT) {
+        sdT[e] = 0.f;
+        sdP[e] = 0.f;
+    }
+    if (tid < kChunk) sdBeta[tid] = sdF[tid] = sdf[tid] = 0.f;
+    if (tid == 0) sdGam[0] = 0.f;
+    const int ar = tid >> 2, ai = tid & 3;  // register sums: row ar, channels ai + 4 m
+    float aQ[ACC], aK[ACC];
+#pragma unroll
+    for (int m = 0; m < ACC; ++m) aQ[m] = aK[m] = 0.f;
+    float dgam = 0.f;
+
+    for (int j0 = 0; j0 < dv; j0 += DVT) {
+        __syncthreads();  // the previous tile is done
+        for (int e = tid; e < DK * DVT; e += NT) {
+            const int i = e / DVT, j = e % DVT;
+            sH[i * LDV + j] = hc[(size_t)i * dv + j0 + j];
+            sDH[i * LDV + j] = dhc[(size_t)i * dv + j0 + j];
+        }
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int r = e / DVT, j = e % DVT;
+            const bool ok = r < Lc;
+            const size_t idx = ((tok0 + r) * H + h) * dv + j0 + j;
+            sV[r * LDV + j] = ok ? to_f32(vin[idx]) : 0.f;
+            sDO[r * LDV + j] = ok ? to_f32(dout[idx]) : 0.f;
+        }
+        __syncthreads();
+        // K h, Q h, K dh' ; X = beta V - beta F (K h)
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int r = e / DVT, j = e % DVT;
+            float kh = 0.f, qh = 0.f, kd = 0.f;
+            for (int i = 0; i < DK; ++i) {
+                const float hv = sH[i * LDV + j], dh = sDH[i * LDV + j];
+                kh = fmaf(c.K[r * LDK + i], hv, kh);
+                qh = fmaf(c.Q[r * LDK + i], hv, qh);
+                kd = fmaf(c.K[r * LDK + i], dh, kd);
+            }
+            sKh[r * LDV + j] = kh;
+            sQh[r * LDV + j] = qh;
+            sKd[r * LDV + j] = kd;
+            sX[r * LDV + j] = c.beta[r] * (sV[r * LDV + j] - c.F[r] * kh);
+        }
+        __syncthreads();
+        // U = T X ; dU = scale P^T dO + diag(f) K dh'
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int r = e / DVT, j = e % DVT;
+            float u = 0.f, du = 0.f;
+            for (int s = 0; s <= r; ++s) u = fmaf(c.T[r * LDT + s], sX[s * LDV + j], u);
+            for (int t = r; t < kChunk; ++t) du = fmaf(c.P[t * LDT + r], sDO[t * LDV + j], du);
+            sU[r * LDV + j] = u;
+            sDU[r * LDV + j] = p.scale * du + c.f[r] * sKd[r * LDV + j];
+        }
+        __syncthreads();
+        // dX = T^T dU ; dv = beta dX
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int s = e / DVT, j = e % DVT;
+            float acc = 0.f;
+            for (int r = s; r < kChunk; ++r) acc = fmaf(c.T[r * LDT + s], sDU[r * LDV + j], acc);
+            sDX[s * LDV + j] = acc;
+            if (s < Lc) p.dv[((tok0 + s) * H + h) * dv + j0 + j] = c.beta[s] * acc;
+        }
+        __syncthreads();
+        // dT += dU X^T, dP += scale dO U^T (lower parts)
+        for (int e = tid; e < kChunk * kChunk; e += NT) {
+            const int r = e / kChunk, s = e % kChunk;
+            if (s > r) continue;
+            float t = 0.f, pp = 0.f;
+#pragma unroll
+            for (int j = 0; j < DVT; ++j) {
+                t = fmaf(sDU[r * LDV + j], sX[s * LDV + j], t);
+                pp = fmaf(sDO[r * LDV + j], sU[s * LDV + j], pp);
+            }
+            sdT[r * LDT + s] += t;
+            sdP[r * LDT + s] += p.scale * pp;
+        }
+        // per-row sums: dbeta, dF, df
+        if (tid < kChunk) {
+            const int r = tid;
+            float db = 0.f, dF = 0.f, df = 0.f;
+#pragma unroll
+            for (int j = 0; j < DVT; ++j) {
+                const float dx = sDX[r * LDV + j], kh = sKh[r * LDV + j];
+                db = fmaf(dx, sV[r * LDV + j] - c.F[r] * kh, db);
+                dF = fmaf(-c.beta[r] * dx, kh, dF);
+                dF = fmaf(p.scale * sDO[r * LDV + j], sQh[r * LDV + j], dF);
+                df = fmaf(sU[r * LDV + j], sKd[r * LDV + j], df);
+            }
+            sdBeta[r] += db;
+            sdF[r] += dF;
+            sdf[r] += df;
+        }
+        // dgamma: <h, dh'> over the tile
+        for (int e = tid; e < DK * DVT; e += NT) {
+            const int i = e / DVT, j = e % DVT;
+            dgam = fmaf(sH[i * LDV + j], sDH[i * LDV + j], dgam);
+        }
+        // register sums: dQ += scale F_r dO h^T ; dK += f_r U dh'^T - beta_r F_r dX h^T
+        {
+            const float sF = p.scale * c.F[ar], fr = c.f[ar], bF = -c.beta[ar] * c.F[ar];
+#pragma unroll
+            for (int m = 0; m < ACC; ++m) {
+                const int i = ai + 4 * m;
+                float q1 = 0.f, k1 = 0.f, k2 = 0.f;
+#pragma unroll
+                for (int j = 0; j < DVT; ++j) {
+                    const float hv = sH[i * LDV + j];
+                    q1 = fmaf(sDO[ar * LDV + j], hv, q1);
+                    k1 = fmaf(sU[ar * LDV + j], sDH[i * LDV + j], k1);
+                    k2 = fmaf(sDX[ar * LDV + j], hv, k2);
+                }
+                aQ[m] = fmaf(sF, q1, aQ[m]);
+                aK[m] = fmaf(fr, k1, fmaf(bF, k2, aK[m]));
+            }
+        }
+    }
+    // dgamma over the CTA
+    for (int o = 16; o > 0; o >>= 1) dgam += __shfl_xor_sync(0xffffffffu, dgam, o);
+    __syncthreads();
+    if ((tid & 31) == 0) atomicAdd(sdGam, dgam);
+    // dA = -T^T dT T^T on the strictly lower part (dT's diagonal and upper part do not reach A)
+    float* sM = sV;  // [64][LDT] scratch over the tile buffers (V, dO, Kh, Qh ... are no longer needed)
+    static_assert(kChunk * (kChunk + 1) <= 9 * kChunk * (16 + 1), "scratch fits the tile buffers");
+    __syncthreads();
+    for (int e = tid; e < kChunk * kChunk; e += NT) {  // M = dT T^T, dT strictly lower
+        const int r = e / kChunk, s = e % kChunk;
+        float m = 0.f;
+        const int tmax = min(r - 1, s);
+        for (int t = 0; t <= tmax; ++t) m = fmaf(sdT[r * LDT + t], c.T[s * LDT + t], m);
+        sM[r * LDT + s] = m;
+    }
+    __syncthreads();
+    float* sdA = c.A;  // A is no longer needed
+    for (int e = tid; e < kChunk * kChunk; e += NT) {
+        const int r = e / kChunk, s = e % kChunk;
+        float a = 0.f;
+        if (s < r)
+            for (int t = r; t < kChunk; ++t) a = fmaf(c.T[t * LDT + r], sM[t * LDT + s], a);
+        sdA[r * LDT + s] = -a;
+    }
+    __syncthreads();
+    // through A and P to K, Q, beta and Gamma: dKK = dA beta_r Gamma, dQK = dP Gamma; W = dGamma . Gamma
+    float* sW = sM;
+    for (int e = tid; e < kChunk * kChunk; e += NT) {
+        const int r = e / kChunk, s = e % kChunk;
+        float dkk = 0.f, dqk = 0.f, w = 0.f;
+        if (s <= r) {
+            float kk = 0.f, qk = 0.f;
+            for (int i = 0; i < DK; ++i) {
+                const float ks = c.K[s * LDK + i];
+                kk = fmaf(c.K[r * LDK + i], ks, kk);
+                qk = fmaf(c.Q[r * LDK + i], ks, qk);
+            }
+            const float gm = c.Gm[r * LDT + s], da = sdA[r * LDT + s], dp = sdP[r * LDT + s];
+            if (s < r) {
+                dkk = da * c.beta[r] * gm;
+                atomicAdd(&sdBeta[r], da * gm * kk);
+            }
+            dqk = dp * gm;
+            w = (da * c.beta[r] * kk + dp * qk) * gm;
+        }
+        sdT[r * LDT + s] = dkk;  // dT holds dKK from here on
+        sdP[r * LDT + s] = dqk;  // dP holds dQK
+        sW[r * LDT + s] = w;
+    }
+    __syncthreads();
+    // gradient of the natural-log cumulative gate Gn (Gamma_rs = exp(Gn_r - Gn_s), F = exp(Gn), f = exp(Gn_L - Gn),
+    // gamma = exp(Gn_L), L the chunk's last row 63: padded rows add nothing)
+    if (tid < kChunk) {
+        const int r = tid;
+        float d = c.F[r] * sdF[r] - c.f[r] * sdf[r];
+        for (int s = 0; s <= r; ++s) d += sW[r * LDT + s];
+        for (int t = r; t < kChunk; ++t) d -= sW[t * LDT + r];
+        if (r == kChunk - 1) {
+            float fs = 0.f;
+            for (int s = 0; s < kChunk; ++s) fs = fmaf(c.f[s], sdf[s], fs);
+            d += fs + c.gamma[0] * sdGam[0];
+        }
+        sdGn[r] = d;
+    }
+    // dQ += dQK K ; dK += dQK^T Q + dKK^T K + dKK K   (register sums of row ar)
+#pragma unroll
+    for (int m = 0; m < ACC; ++m) {
+        const int i = ai + 4 * m;
+        float qa = 0.f, ka = 0.f;
+        for (int s = 0; s <= ar; ++s) {
+            qa = fmaf(sdP[ar * LDT + s], c.K[s * LDK + i], qa);
+            ka = fmaf(sdT[ar * LDT + s], c.K[s * LDK + i], ka);
+        }
+        for (int r = ar; r < kChunk; ++r) {
+            ka = fmaf(sdP[r * LDT + ar], c.Q[r * LDK + i], ka);
+            ka = fmaf(sdT[r * LDT + ar], c.K[r * LDK + i], ka);
+        }
+        aQ[m] += qa;
+        aK[m] += ka;
+    }
+    __syncthreads();
+    if (ar < Lc) {
+#pragma unroll
+        for (int m = 0; m < ACC; ++m) {
+            const size_t idx = ((tok0 + ar) * H + h) * DK + ai + 4 * m;
+            p.dq[idx] = aQ[m];
+            p.dk[idx] = aK[m];
+        }
+    }
+    if (tid < Lc) {
+        const int t = tid;
+        float dg = 0.f;
+        for (int r = t; r < kChunk; ++r) dg += sdGn[r];
+        p.dg[(tok0 + t) * H + h] = dg;
+        p.dbeta[(tok0 + t) * H + h] = sdBeta[t];
+    }
+}
+
+}  // namespace gdn

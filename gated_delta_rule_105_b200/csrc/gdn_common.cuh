@@ -32,7 +32,16 @@ struct FwdParams {
     int B, T, H, dk, dv, n_seq;
     int debug_stall;  // diagnostic (gdn_debug_stall): 0 in every ordinary call
     int kda;          // GDN-2 entry as KDA: beta [B,T,H] is both the erase and the write gate; w unused
+    float* h_chunks;  // SIMT kernel, backward pass only: the state at every chunk start [slot][H][dk][dv], or null
 };
+
+// Chunk slot of chunk c of sequence n that starts at global token offset `start` (row * T + bos):
+// n + floor((start + 64 c) / 64).  Slots of different chunks never coincide, and all are below
+// ceil(B T / 64) + (number of sequences).
+__host__ __device__ inline long long wy_slot(int n, long long start, int c) { return n + (start >> 6) + c; }
+inline long long wy_slots(int B, int T, int n_seqs) {
+    return ((long long)B * T + kChunk - 1) / kChunk + (n_seqs > B ? n_seqs : B);
+}
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -10,7 +10,7 @@
 // Delta cerrado", whose opening paragraph names decoding with constant memory as the point of the fixed-size
 // state).  It is bound by the state's bytes: 8 dk dv bytes per (sequence, head), moved once.
 //
-// One CTA per (sequence, head), DV threads: thread t owns 4 consecutive value columns (float4) of one quarter of
+// One CTA per (sequence, head), dv threads: thread t owns 4 consecutive value columns (float4) of one quarter of
 // the key rows, kept in registers between the read and the write; the two sums over i meet in shared memory.
 #pragma once
 
@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(256) gdn_decode_kernel(const DecodeParams p) {
     constexpr int RPT = DK / kDecRowGroups;  // key rows per thread
     __shared__ float sq[DK], sk[DK], se[DK], sa[DK];
     __shared__ float sz[256];
-    __shared__ __align__(16) float red[2][kDecRowGroups][256];
+    __shared__ __align__(16) float red[2][kDecRowGroups][256];  // 16 KB
     const int dv = p.dv, cg_n = dv / 4;
     const int tid = threadIdx.x, cgp = tid % cg_n, rg = tid / cg_n;
     const size_t nh = blockIdx.x;  // n * H + h

@@ -14,7 +14,7 @@ namespace gdn {
 
 enum ProfKernel : int {
     PK_SIMT = 0, PK_TC_WY = 1, PK_TC_MAIN = 2, PK_TC2_PREP = 3, PK_TC2_MAIN = 4, PK_DECODE = 5, PK_PRELUDE = 6,
-    PK_OUT_GATE = 7, PK_COUNT = 8
+    PK_OUT_GATE = 7, PK_BWD = 8, PK_COUNT = 9
 };
 
 struct ProfState {

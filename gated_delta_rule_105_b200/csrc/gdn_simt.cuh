@@ -118,6 +118,11 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
     for (int c0 = bos; c0 < eos; c0 += kChunk) {
         const int Lc = min(kChunk, eos - c0);
         __syncthreads();  // the previous chunk is done with every buffer
+        if (p.h_chunks) {  // the state at this chunk's start, for the backward pass
+            float* hc = p.h_chunks + ((size_t)wy_slot(n, (long long)row * T + bos, (c0 - bos) / kChunk) * H + h) *
+                                         DK * (size_t)dv + j0;
+            for (int e = tid; e < DK * DVT; e += NT) hc[(size_t)(e / DVT) * dv + e % DVT] = sH[e];
+        }
         // ---- load the chunk (zero-padded past Lc); unrolled so that many global loads are in flight
 #pragma unroll 8
         for (int e = tid; e < kChunk * DK; e += NT) {
@@ -322,7 +327,7 @@ gdn_simt_fwd_kernel(FwdParams p, unsigned* err) {
             const int r = e / DVT, j = e % DVT;
             float acc = oi[m];
             for (int s = 0; s <= r; ++s) acc = fmaf(sP[r * LDT + s], sU[s * DVT + j], acc);
-            if (r < Lc) {
+            if (o && r < Lc) {  // o is null when only the chunk states are wanted (backward pass)
                 const size_t tok = ((size_t)row * T + c0 + r) * H + h;
                 o[tok * dv + j0 + j] = from_f32<TOut>(p.scale * acc);
             }

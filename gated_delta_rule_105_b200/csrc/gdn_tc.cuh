@@ -53,13 +53,6 @@ struct TcGate {  // one chunk's gate data
 };
 static_assert(sizeof(TcGate) % 16 == 0, "gate stage size");
 
-// Workspace slot of chunk c of a sequence that starts at global token offset `start` (row * T + bos) and
-// is sequence number n: n + floor((start + 64 c) / 64).  Slots of different chunks never coincide, and
-// all are below ceil(B T / 64) + (number of sequences).
-__host__ __device__ inline long long wy_slot(int n, long long start, int c) { return n + (start >> 6) + c; }
-inline long long wy_slots(int B, int T, int n_seqs) {
-    return ((long long)B * T + kChunk - 1) / kChunk + (n_seqs > B ? n_seqs : B);
-}
 
 // One chunk's gates, by one warp (lane l: tokens 2l, 2l+1).  tok0 = global token index of row 0.
 __device__ __forceinline__ void tc_make_gates(TcGate& gs, const FwdParams& p, size_t tok0, int Lc, int h, int lane) {

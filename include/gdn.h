@@ -200,6 +200,23 @@ gdn_status gdn_prelude_fwd(const void* xq, const void* xk, const void* xv, const
 gdn_status gdn_output_gate_fwd(const void* o, const void* z, const float* weight, void* y, long long rows, int dv,
                                gdn_dtype dt, float eps, cudaStream_t stream);
 
+/* Backward pass (reverse mode) of gdn_chunk_fwd: given the cotangents d_o of o and dhT of the final state, the
+ * gradients of <d_o, o> + <dhT, hT> with respect to q, k, v, g, beta and h0.  (The walkthrough's section "Chunked
+ * parallelism" names this full backward for q, k, v, beta and g.)  It runs the chunk recurrence backwards through
+ * the WY form: the forward states at every chunk start are recomputed into the workspace, the state cotangent is
+ * carried from the last chunk to the first, and every chunk's input gradients are then formed in parallel.
+ * Arithmetic is fp32 on CUDA cores for both input dtypes.
+ * Layouts: q, k, v, d_o as for gdn_chunk_fwd (d_o [B,T,H,dv] in `dt`); g, beta [B,T,H] fp32; h0, dhT
+ * [N,H,dk,dv] fp32 or NULL (zeros); outputs dq, dk [B,T,H,dk], dv [B,T,H,dv], dg, dbeta [B,T,H] and dh0
+ * [N,H,dk,dv] (NULL: not written), all fp32, overwritten.  Workspace: gdn_bwd_workspace_bytes() bytes (two fp32
+ * states per chunk slot and head), required.  Shapes, cu_seqlens and errors as for gdn_chunk_fwd. */
+size_t gdn_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs);
+gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta, float scale,
+                         const float* h0, const void* d_o, const float* dhT, float* dq, float* dk, float* dv,
+                         float* dg, float* dbeta, float* dh0, int B, int T, int H, int dk_, int dv_, int BT,
+                         gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs, void* workspace, size_t ws_bytes,
+                         cudaStream_t stream);
+
 /* Selects the kernel family for later calls from any thread (process-wide; default AUTO). */
 gdn_status gdn_set_kernel(gdn_kernel kernel);
 
@@ -238,8 +255,8 @@ gdn_status gdn_debug_umma_selftest(const float* A, const float* B, float* D, int
  * launch made by the *_fwd calls is bracketed by two CUDA events recorded on its stream.
  * gdn_profile_take(kernel, &launches, &total_ms) waits for the recorded events of one kernel -- 0: SIMT
  * kernel, 1: tensor-core WY kernel, 2: tensor-core chunk kernel, 3: GDN-2 / KDA prep kernel, 4: GDN-2 / KDA
- * chunk kernel, 5: decode kernel, 6: prelude kernel, 7: output gate kernel -- returns how many launches they
- * cover and
+ * chunk kernel, 5: decode kernel, 6: prelude kernel, 7: output gate kernel, 8: the backward's two kernels
+ * (its forward recompute counts as 0) -- returns how many launches they cover and
  * their summed device time in milliseconds, and forgets them.  Errors: GDN_ERR_INVALID_ARG for an unknown
  * kernel id or NULL outputs, GDN_ERR_CUDA if an event failed. */
 gdn_status gdn_profile_enable(int on);

@@ -30,7 +30,8 @@ def test_header_declares_the_entry_points():
               "gdn_last_error", "gdn_set_kernel", "gdn_last_kernel", "gdn_debug_umma_selftest",
               "gdn_chunk_fwd_noalloc", "gdn_profile_enable", "gdn_profile_take", "gdn2_workspace_bytes",
               "gdn_kda_chunk_fwd", "gdn_debug_stall", "gdn_decode_fwd", "gdn2_decode_fwd",
-              "gdn_kda_decode_fwd", "gdn_prelude_fwd", "gdn_output_gate_fwd"]:
+              "gdn_kda_decode_fwd", "gdn_prelude_fwd", "gdn_output_gate_fwd", "gdn_bwd_workspace_bytes",
+              "gdn_chunk_bwd"]:
         assert n in names
 
 

@@ -11,7 +11,7 @@ from gated_delta_rule_105_b200.inputs import generate
 def test_profile_take_rejects_bad_ids(oracle_lib):
     lib = bd.load_library()
     n, ms = ctypes.c_int(7), ctypes.c_double(1.0)
-    assert lib.gdn_profile_take(8, ctypes.byref(n), ctypes.byref(ms)) == 1
+    assert lib.gdn_profile_take(9, ctypes.byref(n), ctypes.byref(ms)) == 1
     assert lib.gdn_profile_take(-1, ctypes.byref(n), ctypes.byref(ms)) == 1
     assert lib.gdn_profile_take(0, None, ctypes.byref(ms)) == 1
     # nothing recorded: zero launches, no device work
