@@ -479,8 +479,8 @@ def run_row(args, w):
     """Device throughput of one of the path's other kernels on the bench workload's shape (1 GPU, rank 0 prints):
     ``decode`` -- one recurrent decode step for 64 sequences of the workload's heads (state read and written in
     place); ``prelude`` -- short conv + SiLU + L2 norm + gates over the whole workload; ``output_gate`` -- the
-    RMSNorm x SiLU epilogue over the workload's output; ``bwd`` -- the backward pass of the workload (GDN).  Each is
-    reported against the HBM roofline of its bytes per launch."""
+    RMSNorm x SiLU epilogue over the workload's output; ``bwd`` -- the backward pass of the workload (GDN or
+    GDN-2).  Each is reported against the HBM roofline of its bytes per launch."""
     import torch
     from gated_delta_rule_105_b200 import decode_fwd, output_gate_fwd, prelude_fwd, profile_enable, profile_take
     from gated_delta_rule_105_b200.inputs import generate, generate_prelude
@@ -514,22 +514,32 @@ def run_row(args, w):
         nbytes = B * T * H * (2 * s * (2 * dk + dv) + 4 * 4)
         tokens, kname, workload = B * T, "gdn_prelude_kernel", f"prelude B{B} T{T} H{H} dk{dk} dv{dv}"
     elif args.path == "bwd":
-        from gated_delta_rule_105_b200 import bwd_workspace_bytes, gdn_chunk_bwd
-        inp = generate(B, T, H, dk, dv, w.dtype, w.seed, "gdn", w.h0_std or 0.02, w.n_seqs, w.len_range)
+        from gated_delta_rule_105_b200 import (bwd_workspace_bytes, gdn2_bwd_workspace_bytes, gdn2_chunk_bwd,
+                                               gdn_chunk_bwd)
+        gdn2 = w.variant == "gdn2"
+        inp = generate(B, T, H, dk, dv, w.dtype, w.seed, w.variant, w.h0_std or 0.02, w.n_seqs, w.len_range)
         d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
         gen = torch.Generator().manual_seed(w.seed + 1)
         d_o = torch.randn((B, T, H, dv), generator=gen).to(d["q"].dtype).to(dev)
         n_seq = d["h0"].shape[0]
         dhT = torch.randn((n_seq, H, dk, dv), generator=gen).mul_(0.5).to(dev)
-        n_ws = bwd_workspace_bytes(B, T, H, dk, dv, C, 0 if d["cu_seqlens"] is None else n_seq)
+        n_ws = (gdn2_bwd_workspace_bytes if gdn2 else bwd_workspace_bytes)(
+            B, T, H, dk, dv, C, 0 if d["cu_seqlens"] is None else n_seq)
         wsp = torch.empty(n_ws, dtype=torch.uint8, device=dev)
 
         def step():
-            gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d_o, d["scale"], d["h0"], dhT, d["cu_seqlens"],
-                          workspace=wsp)
+            if gdn2:
+                gdn2_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d_o, d["scale"], d["h0"], dhT,
+                               d["cu_seqlens"], workspace=wsp)
+            else:
+                gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d_o, d["scale"], d["h0"], dhT,
+                              d["cu_seqlens"], workspace=wsp)
         s = 2 if w.dtype == "bf16" else 4
-        # read q, k, v, d_o, g, beta, h0, dhT; write dq, dk, dv (fp32), dg, dbeta, dh0
-        nbytes = B * T * H * (s * (2 * dk + 2 * dv) + 8 + 4 * (2 * dk + dv) + 8) + 3 * n_seq * H * dk * dv * 4
+        if gdn2:  # read q, k, v, d_o, g, b, w, h0, dhT; write dq, dk, dg, db, dv, dw (fp32), dh0
+            nbytes = B * T * H * (s * (2 * dk + 2 * dv) + 4 * (2 * dk + dv) + 4 * (4 * dk + 2 * dv))
+        else:  # read q, k, v, d_o, g, beta, h0, dhT; write dq, dk, dv (fp32), dg, dbeta, dh0
+            nbytes = B * T * H * (s * (2 * dk + 2 * dv) + 8 + 4 * (2 * dk + dv) + 8)
+        nbytes += 3 * n_seq * H * dk * dv * 4
         tokens, kname, workload = B * T, "gdn_bwd_kernels", f"backward {w.name}"
     else:
         gen = torch.Generator().manual_seed(w.seed)

@@ -79,6 +79,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_bwd_workspace_bytes.restype = sz
     lib.gdn_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [fp] * 6 + [i] * 6 + [i, vp, i, vp, sz, vp]
     lib.gdn_chunk_bwd.restype = i
+    lib.gdn2_bwd_workspace_bytes.argtypes = [i] * 7
+    lib.gdn2_bwd_workspace_bytes.restype = sz
+    lib.gdn2_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, f, fp, vp, fp] + [fp] * 7 + [i] * 6 + [i, vp, i, vp, sz, vp]
+    lib.gdn2_chunk_bwd.restype = i
+    lib.gdn_kda_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp] + [fp] * 6 + [i] * 6 + [i, vp, i, vp, sz, vp]
+    lib.gdn_kda_chunk_bwd.restype = i
     lib.gdn_debug_stall.argtypes = [i]
     lib.gdn_debug_stall.restype = i
     _lib = lib
@@ -243,7 +249,7 @@ def gdn_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, h0=None, output_final_st
                           BT=64, o=None, hT=None, o_dtype=None):
     """As :func:`gdn_chunk_fwd`, through ``gdn_chunk_fwd_noalloc``, for callers that may not allocate device
     memory (an engine that owns all of it, a host framework's allocator): no workspace is allocated, the
-    library's static 128 MiB scratch serves the tensor-core path, sizes that need more are refused, and calls
+    library's static 256 MiB scratch serves the tensor-core path, sizes that need more are refused, and calls
     must not overlap on the device.  The outputs ``o`` and ``hT`` are still allocated here unless passed in."""
     B, T, H, dk, dv, n_seq, o, hT = _prep(q, k, v, h0, cu_seqlens, o, hT, output_final_state, o_dtype)
     _check_dev("g", g, torch.float32)
@@ -450,3 +456,67 @@ def gdn_chunk_bwd(q, k, v, g, beta, d_o, scale=None, h0=None, dhT=None, cu_seqle
         BT, _dtype_code(q), _ptr(cu_seqlens), n_seqs, _ptr(workspace), workspace.numel(), stream)
     _raise_on(st)
     return out
+
+
+def gdn2_bwd_workspace_bytes(B, T, H, dk, dv, BT=64, n_seqs=0) -> int:
+    """Device workspace (bytes) ``gdn2_chunk_bwd`` and ``gdn_kda_chunk_bwd`` need: two fp32 states and the fp32
+    T and P of every chunk slot and head."""
+    return int(load_library().gdn2_bwd_workspace_bytes(B, T, H, dk, dv, BT, n_seqs))
+
+
+def _bwd2(kda, q, k, v, g, b, w, d_o, scale, h0, dhT, cu_seqlens, BT, workspace, want_dh0):
+    _check_dev("q", q)
+    dt = q.dtype
+    for name, t in (("k", k), ("v", v), ("d_o", d_o)):
+        _check_dev(name, t, dt)
+    for name, t in (("g", g), ("b" if not kda else "beta", b), ("w", w), ("h0", h0), ("dhT", dhT)):
+        _check_dev(name, t, torch.float32)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        _check_dev("cu_seqlens", cu_seqlens, torch.int32)
+    n_seq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    n_seqs = 0 if cu_seqlens is None else n_seq
+    f32 = dict(dtype=torch.float32, device=q.device)
+    out = {"dq": torch.empty((B, T, H, dk), **f32), "dk": torch.empty((B, T, H, dk), **f32),
+           "dv": torch.empty((B, T, H, dv), **f32), "dg": torch.empty((B, T, H, dk), **f32)}
+    if kda:
+        out["dbeta"] = torch.empty((B, T, H), **f32)
+    else:
+        out["db"] = torch.empty((B, T, H, dk), **f32)
+        out["dw"] = torch.empty((B, T, H, dv), **f32)
+    out["dh0"] = torch.empty((n_seq, H, dk, dv), **f32) if want_dh0 else None
+    if workspace is None:
+        workspace = torch.empty(gdn2_bwd_workspace_bytes(B, T, H, dk, dv, BT, n_seqs), dtype=torch.uint8,
+                                device=q.device)
+    _check_dev("workspace", workspace, torch.uint8)
+    scale = dk ** -0.5 if scale is None else float(scale)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(q.device).cuda_stream)
+    lib = load_library()
+    tail = (B, T, H, dk, dv, BT, _dtype_code(q), _ptr(cu_seqlens), n_seqs, _ptr(workspace), workspace.numel(), stream)
+    if kda:
+        st = lib.gdn_kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), scale, _ptr(h0), _ptr(d_o), _ptr(dhT),
+                                   _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                                   _ptr(out["dbeta"]), _ptr(out["dh0"]), *tail)
+    else:
+        st = lib.gdn2_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), scale, _ptr(h0), _ptr(d_o),
+                                _ptr(dhT), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                                _ptr(out["db"]), _ptr(out["dw"]), _ptr(out["dh0"]), *tail)
+    _raise_on(st)
+    return out
+
+
+def gdn2_chunk_bwd(q, k, v, g, b, w, d_o, scale=None, h0=None, dhT=None, cu_seqlens=None, BT=64, workspace=None,
+                   want_dh0=True):
+    """Backward pass of :func:`gdn2_chunk_fwd` through ``gdn2_chunk_bwd``: the gradients of <d_o, o> + <dhT, hT>.
+
+    g, b [B,T,H,dk] and w [B,T,H,dv] fp32; d_o in q's dtype.  Returns fp32 dq, dk, dv, dg, db, dw and dh0.
+    """
+    return _bwd2(False, q, k, v, g, b, w, d_o, scale, h0, dhT, cu_seqlens, BT, workspace, want_dh0)
+
+
+def gdn_kda_chunk_bwd(q, k, v, g, beta, d_o, scale=None, h0=None, dhT=None, cu_seqlens=None, BT=64, workspace=None,
+                      want_dh0=True):
+    """Backward pass of :func:`gdn_kda_chunk_fwd` through ``gdn_kda_chunk_bwd``.  g [B,T,H,dk] and beta [B,T,H]
+    fp32.  Returns fp32 dq, dk, dv, dg [B,T,H,dk], dbeta [B,T,H] and dh0."""
+    return _bwd2(True, q, k, v, g, beta, None, d_o, scale, h0, dhT, cu_seqlens, BT, workspace, want_dh0)

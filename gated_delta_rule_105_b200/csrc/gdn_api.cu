@@ -16,6 +16,7 @@
 #include "gdn_decode.cuh"
 #include "gdn_prelude.cuh"
 #include "gdn_bwd.cuh"
+#include "gdn2_bwd.cuh"
 #include "gdn_tc_selftest.cuh"
 
 namespace gdn {
@@ -276,6 +277,84 @@ static gdn_status launch_bwd_dk(const FwdParams& fp, const BwdParams& bp, unsign
     return GDN_OK;
 }
 
+// ---- backward of GDN-2 and KDA
+inline size_t bwd2_tp_bytes(int B, int T, int H, int n_seqs) {
+    return (size_t)wy_slots(B, T, n_seqs) * H * 2 * kChunk * kChunk * sizeof(float);
+}
+inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv, int n_seqs) {
+    return bwd_workspace_bytes(B, T, H, dk, dv, n_seqs) + bwd2_tp_bytes(B, T, H, n_seqs);
+}
+
+template <typename TIn, int DK>
+static gdn_status launch_bwd2_dk(const FwdParams& fp, const Bwd2Params& bp, unsigned* err, cudaStream_t stream) {
+    // (1) the state at every chunk start, from the SIMT forward (no o written)
+    gdn_status st = launch_simt_dk<TIn, float, DK, true>(fp, err, stream);
+    if (st != GDN_OK) return st;
+    const long long grid = wy_slots(bp.B, bp.T, bp.n_seq) * bp.H;
+    if (grid > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "too many chunks for one launch");
+    ProfScope prof(PK_BWD, stream);
+    // (2) T and P of every chunk
+    auto kp = gdn2_bwd_prep_kernel<TIn, DK>;
+    cudaError_t e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Bw2PrepSmem<DK>::bytes);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    if (grid > 0) kp<<<(unsigned)grid, kBw2Threads, Bw2PrepSmem<DK>::bytes, stream>>>(bp, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward prep kernel: %s", cudaGetErrorString(e));
+    // (3) the state cotangent, chunk by chunk backwards
+    auto kdh = gdn2_bwd_dh_kernel<TIn, DK>;
+    e = cudaFuncSetAttribute(kdh, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Bw2DhSmem<DK>::bytes);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    kdh<<<dim3(bp.vdim / Bw2DhSmem<DK>::DVT, bp.H, bp.n_seq), kBw2Threads, Bw2DhSmem<DK>::bytes, stream>>>(bp, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward state kernel: %s", cudaGetErrorString(e));
+    // (4) every input gradient, all chunks at once
+    auto kc = gdn2_bwd_chunk_kernel<TIn, DK>;
+    e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Bw2ChunkSmem<DK>::bytes);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    if (grid > 0) kc<<<(unsigned)grid, kBw2Threads, Bw2ChunkSmem<DK>::bytes, stream>>>(bp, err);
+    prof.done();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward chunk kernel: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+// Shared body of gdn2_chunk_bwd and gdn_kda_chunk_bwd (kda: b is beta [B,T,H], w and dw unused).
+static gdn_status chunk_bwd2(const void* q, const void* k, const void* v, const float* g, const float* b,
+                             const float* w, bool kda, float scale, const float* h0, const void* d_o, const float* dhT,
+                             float* dq, float* dk, float* dv, float* dg, float* db, float* dw, float* dh0, int B, int T,
+                             int H, int dk_, int dv_, int BT, gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    int n_seq = 0;
+    gdn_status st = check_common(q, k, v, g, b, w, !kda, scale, h0, d_o, dhT, B, T, H, dk_, dv_, BT, dt, dt,
+                                 cu_seqlens, n_seqs, workspace, ws_bytes, &n_seq);
+    if (st != GDN_OK) return st;
+    if (T > 0 && (!dq || !dk || !dv || !dg || !db || (!kda && !dw)))
+        return fail(GDN_ERR_INVALID_ARG, "a gradient output (dq, dk, dv, dg, %s) is NULL", kda ? "dbeta" : "db, dw");
+    const void* outs[] = {dq, dk, dv, dg, db, dw, dh0};
+    for (const void* ptr : outs)
+        if (ptr && !aligned16(ptr)) return fail(GDN_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", ptr);
+    const int ns = cu_seqlens ? n_seq : 0;
+    const size_t need = bwd2_workspace_bytes(B, T, H, dk_, dv_, ns);
+    if (!workspace || ws_bytes < need)
+        return fail(GDN_ERR_INVALID_ARG, "the backward pass needs %zu bytes of workspace (got %zu)", need, ws_bytes);
+    gdn_status es;
+    unsigned* err = err_word_ptr(&es);
+    if (!err) return es;
+    const size_t states = bwd_workspace_bytes(B, T, H, dk_, dv_, ns) / sizeof(float);
+    float* hc = static_cast<float*>(workspace);
+    float* dhc = hc + states / 2;
+    float* tp = hc + states;
+    FwdParams fp{q, k, v, g, b, kda ? nullptr : w, h0, nullptr, nullptr, cu_seqlens, scale, B, T, H, dk_, dv_, n_seq};
+    fp.kda = kda ? 1 : 0;
+    fp.h_chunks = hc;
+    Bwd2Params bp{q, k, v, g, b, kda ? nullptr : w, d_o, dhT, hc, dhc, tp, dq, dk, dv, dg, db, kda ? nullptr : dw,
+                  dh0, cu_seqlens, scale, B, T, H, dk_, dv_, n_seq, kda ? 1 : 0};
+    if (dt == GDN_F32)
+        return dk_ == 64 ? launch_bwd2_dk<float, 64>(fp, bp, err, stream) : launch_bwd2_dk<float, 128>(fp, bp, err, stream);
+    return dk_ == 64 ? launch_bwd2_dk<__nv_bfloat16, 64>(fp, bp, err, stream)
+                     : launch_bwd2_dk<__nv_bfloat16, 128>(fp, bp, err, stream);
+}
+
 }  // namespace gdn
 
 using namespace gdn;
@@ -477,6 +556,31 @@ gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const floa
         return dk_ == 64 ? launch_bwd_dk<float, 64>(fp, bp, err, stream) : launch_bwd_dk<float, 128>(fp, bp, err, stream);
     return dk_ == 64 ? launch_bwd_dk<__nv_bfloat16, 64>(fp, bp, err, stream)
                      : launch_bwd_dk<__nv_bfloat16, 128>(fp, bp, err, stream);
+}
+
+size_t gdn2_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs) {
+    if (B < 1 || T < 0 || H < 1 || BT != kChunk || (dk != 64 && dk != 128) || dv < 64 || dv > 256 || dv % 64 != 0 ||
+        n_seqs < 0)
+        return 0;
+    return bwd2_workspace_bytes(B, T, H, dk, dv, n_seqs);
+}
+
+gdn_status gdn2_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* b, const float* w,
+                          float scale, const float* h0, const void* d_o, const float* dhT, float* dq, float* dk,
+                          float* dv, float* dg, float* db, float* dw, float* dh0, int B, int T, int H, int dk_, int dv_,
+                          int BT, gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs, void* workspace,
+                          size_t ws_bytes, cudaStream_t stream) {
+    return chunk_bwd2(q, k, v, g, b, w, false, scale, h0, d_o, dhT, dq, dk, dv, dg, db, dw, dh0, B, T, H, dk_, dv_, BT,
+                      dt, cu_seqlens, n_seqs, workspace, ws_bytes, stream);
+}
+
+gdn_status gdn_kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             float scale, const float* h0, const void* d_o, const float* dhT, float* dq, float* dk,
+                             float* dv, float* dg, float* dbeta, float* dh0, int B, int T, int H, int dk_, int dv_,
+                             int BT, gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs, void* workspace,
+                             size_t ws_bytes, cudaStream_t stream) {
+    return chunk_bwd2(q, k, v, g, beta, nullptr, true, scale, h0, d_o, dhT, dq, dk, dv, dg, dbeta, nullptr, dh0, B, T,
+                      H, dk_, dv_, BT, dt, cu_seqlens, n_seqs, workspace, ws_bytes, stream);
 }
 
 gdn_status gdn_set_kernel(gdn_kernel kernel) {

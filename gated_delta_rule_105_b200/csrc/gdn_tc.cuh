@@ -12,8 +12,9 @@
 // (GatedDeltaNet data-flow walkthrough, yfxerp.com/news/367755, section "Chunked parallelism").
 //
 // The WY kernel (gdn_tc_wy_kernel) computes, for every (chunk, head) at once, A from K K^T, the inverse and
-// T', T'' (T'' as a bf16 hi + lo pair), and writes them to the workspace in the exact shared-memory form
-// the MMAs read (24 KB per chunk and head).  Nothing in it depends on the state, so it runs fully parallel.
+// T', T'' (T'' as a bf16 hi + lo pair), and P from Q K^T, and writes them to the workspace in the exact
+// shared-memory form the MMAs read (40 KB per chunk and head).  Nothing in it depends on the state, so it runs
+// fully parallel.
 // The main kernel (gdn_tc_fwd_kernel) then walks each sequence's chunks: one CTA owns one (sequence n,
 // head h, block of 128 value columns j); the state is kept transposed, h^T [j][i] (value column j on the 128
 // TMEM lanes, key channel i on 128 columns), fp32 in TMEM for the whole sequence.  Every contraction is an
@@ -39,7 +40,10 @@ constexpr int kTcThreads = 512;  // main kernel: 16 warps
 constexpr int kWyThreads = 128;  // WY kernel: one warpgroup
 constexpr int kTcDV = 128;       // value columns per CTA
 constexpr int kTcDK = 128;       // key dimension handled by these kernels
-constexpr uint32_t kWyUnit = 24576;  // workspace bytes per (chunk, head): T' | T''_hi | T''_lo, 8 KB each
+// workspace bytes per (chunk, head): T' | T''_hi | T''_lo (bf16 [r][s]) | P columns 0-31 | P columns 32-63
+// (tf32 [r][s]), 8 KB each, every piece in the 128B-swizzled K-major form the chunk kernel's MMAs read
+constexpr uint32_t kWyUnit = 40960;
+constexpr uint32_t kWyP = 24576;  // offset of P in a unit
 
 struct TcGate {  // one chunk's gate data
     float G[64];     // log2(e) * chunk-local cumulative g
@@ -387,25 +391,25 @@ __device__ __forceinline__ void wy_unit_of_slot(const FwdParams& p, long long sl
 
 // ------------------------------------------------------------------------------------------ the WY kernel
 // Shared-memory map (bytes from a 1024-aligned base).  The S1 MMA reads a 128-row A operand per 64-channel
-// panel (rows 0-63: the K tile; rows 64-127: whatever follows it, results unused), so each K panel is
-// followed by 8 KB of other data: the T' and T''_hi emission areas.  T''_lo reuses the first K panel.
+// panel, rows 0-63 the K tile and rows 64-127 the Q tile ([K0 | Q0 | K1 | Q1], as in the chunk kernel), and K
+// as its B operand.  Once S1 is in TMEM the four panels are free: the P rows go to Q0 (columns 0-31) and Q1
+// (columns 32-63) and are stored from there; then the inverse writes T''_lo over K0, T''_hi over Q0 and T' over K1.
 struct WySmem {
-    static constexpr uint32_t K0 = 0;        // K channels 0-63, [64 tokens][128 B] swizzled; then T''_lo
-    static constexpr uint32_t K1 = 8192;     // K channels 64-127; then T'
-    static constexpr uint32_t TPP = 16384;   // T''_hi
-    static constexpr uint32_t TP = K1;       // T' and T''_lo are written by the inverse, once S1 has been
-    static constexpr uint32_t TPPL = K0;     // computed from K
-    static constexpr uint32_t AS = 24576;    // A, then (I+A)^-1, fp32 [64][68]
+    static constexpr uint32_t K0 = 0, Q0 = 8192, K1 = 16384, Q1 = 24576;  // [64 tokens][128 B] swizzled each
+    static constexpr uint32_t PH = Q0, PL = Q1;  // P, columns 0-31 and 32-63 (tf32 [r][s])
+    static constexpr uint32_t TPPL = K0, TPP = Q0, TP = K1;
+    static constexpr uint32_t AS = 32768;  // A, then (I+A)^-1, fp32 [64][68]
     static constexpr uint32_t GATE = AS + 64 * kAsLd * 4;
-    static constexpr uint32_t BARS = GATE + sizeof(TcGate);  // [0] K landed, [1] S1 done
+    static constexpr uint32_t BARS = GATE + sizeof(TcGate);  // [0] K, Q landed, [1] S1 done
     static constexpr uint32_t MISC = BARS + 16;              // tmem base, abort flag, unit info
     static constexpr uint32_t END = MISC + 64;
-    static constexpr uint32_t ALLOC = END + 1024;  // 5 CTAs per SM
+    static constexpr uint32_t ALLOC = END + 1024;  // 4 CTAs per SM
 };
 
-// One CTA per (workspace slot, head): finds the (sequence, chunk) of its slot, builds A, inverts I + A and
-// writes T', T''_hi, T''_lo of that chunk to the workspace.
-__global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_constant__ CUtensorMap tm_k,
+// One CTA per (workspace slot, head): finds the (sequence, chunk) of its slot, builds A and P from S1 = [K; Q] K^T,
+// inverts I + A and writes T', T''_hi, T''_lo and P of that chunk to the workspace.
+__global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                               const __grid_constant__ CUtensorMap tm_k,
                                                                const FwdParams p, uint8_t* ws, unsigned* err) {
     using namespace sm100;
     using L = WySmem;
@@ -430,9 +434,11 @@ __global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_cons
             mbar_init(&bars[1], 1);
             *abort_flag = 0;
             fence_barrier_init();
-            mbar_expect_tx(&bars[0], 16384);
+            mbar_expect_tx(&bars[0], 32768);
             tma_load_3d(sm + L::K0, &tm_k, &bars[0], 0, h, info[1]);
+            tma_load_3d(sm + L::Q0, &tm_q, &bars[0], 0, h, info[1]);
             tma_load_3d(sm + L::K1, &tm_k, &bars[0], 64, h, info[1]);
+            tma_load_3d(sm + L::Q1, &tm_q, &bars[0], 64, h, info[1]);
         }
     }
     __syncthreads();
@@ -448,15 +454,14 @@ __global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     if (tid == 0) {
-        // S1 = K K^T (rows 64-127 of the A operand are the next 8 KB, other data; their results are never
-        // read): k-steps 0-3 read channel panel K0, 4-7 panel K1, 8 KB further
+        // S1 = [K; Q] K^T: k-steps 0-3 read channel panels K0 | Q0, 4-7 panels K1 | Q1, 16 KB further
         if (mbar_wait(&bars[0], 0, abort_flag, err)) {
             tc_fence_after();
             const uint64_t d = desc_k_sw128(smem_u32(sm));
             const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll 1
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t a = d + (kk >> 2) * 512 + (kk & 3) * 2;
+                const uint64_t a = d + (kk >> 2) * 1024 + (kk & 3) * 2;
                 umma_bf16(tmem, a, a, id, kk > 0);
             }
             umma_commit(&bars[1]);
@@ -465,7 +470,14 @@ __global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_cons
     __syncwarp();
     const bool ok = warp_wait(&bars[1], 0, abort_flag, err);
     tc_fence_after();
-    if (ok && warp < 2) tc_row_pass<true>(taddr(tmem, 32 * warp, 0), gs, tid, 0, 63, sA + tid * kAsLd, nullptr, nullptr);
+    // rows of A (warps 0-1, TMEM lanes 0-63) and of P (warps 2-3, lanes 64-127); P rows 0-31 need columns 0-31
+    // only, the chunk kernel's MMA never reads the blocks above the diagonal
+    if (ok) {
+        if (warp < 2) tc_row_pass<true>(taddr(tmem, 32 * warp, 0), gs, tid, 0, 63, sA + tid * kAsLd, nullptr, nullptr);
+        else tc_row_pass<false>(taddr(tmem, 32 * warp, 0), gs, tid - 64, 0, warp == 2 ? 31 : 63, nullptr,
+                                sm + L::PH, sm + L::PL);
+    }
+    fence_proxy_async();
     tc_fence_before();
     const bool all_ok = __syncthreads_and(ok) != 0;  // one outcome for the CTA: the inverse has barriers
     if (warp == 0) {
@@ -473,12 +485,19 @@ __global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_cons
         tmem_dealloc(tmem, 64);
     }
     if (!all_ok) return;
+    uint8_t* dst = ws + ((size_t)slot * p.H + h) * kWyUnit;
+    if (tid == 0) {  // P, read out of shared memory before the inverse writes T''_hi over it
+        bulk_store(dst + kWyP, sm + L::PH, 8192);
+        bulk_store(dst + kWyP + 8192, sm + L::PL, 8192);
+        bulk_commit();
+        bulk_wait_read();
+    }
+    __syncthreads();
     const TEmit em{sm + L::TP, sm + L::TPP, sm + L::TPPL, gs.beta, gs.eG};
     invert_unit_lower64(sA, warp, lane, 1, em);
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
-        uint8_t* dst = ws + ((size_t)slot * p.H + h) * kWyUnit;
         bulk_store(dst, sm + L::TP, 8192);
         bulk_store(dst + 8192, sm + L::TPP, 8192);
         bulk_store(dst + 16384, sm + L::TPPL, 8192);
@@ -495,14 +514,14 @@ struct TcSmem {
     static constexpr uint32_t V = KQ + 2 * KQ_STAGE;  // V tile: j 0-63 | j 64-127, 8 KB each (MN-major A)
     static constexpr uint32_t TW = V + 16384;         // [T''_hi | T''_lo], [r][s] K-major, 8 KB each
     static constexpr uint32_t TP = TW + 16384;        // T': [r][s] K-major, 8 KB
-    static constexpr uint32_t PH = TP + 8192;         // P, tokens 0-31 [2]: [r][s] K-major fp32, 8 KB each
-    static constexpr uint32_t PL = PH + 16384;        // P, tokens 32-63 [2]
+    static constexpr uint32_t PH = TP + 8192;         // P, columns 0-31 [2]: [r][s] K-major tf32, 8 KB each
+    static constexpr uint32_t PL = PH + 16384;        // P, columns 32-63 [2] (both loaded with the K/Q stage)
     static constexpr uint32_t WT = PL + 16384;        // -W^T: lines i (128) x 64 r, MN-major B, 16 KB
     static constexpr uint32_t HT = WT + 16384;        // h^T bf16 [2]: [j][i] K-major, panels i 0-63 | 64-127
     static constexpr uint32_t HT_STAGE = 32768;
     static constexpr uint32_t GATE = HT + 2 * HT_STAGE;  // 4 x TcGate
     static constexpr uint32_t BARS = GATE + 4 * sizeof(TcGate);
-    static constexpr uint32_t N_BARS = 29;
+    static constexpr uint32_t N_BARS = 25;
     static constexpr uint32_t MISC = BARS + 8 * N_BARS;  // tmem base, abort flag
     static constexpr uint32_t END = MISC + 64;
     static constexpr uint32_t ALLOC = END + 1024;  // slack for the 1024-byte alignment of the base
@@ -511,42 +530,38 @@ static_assert(TcSmem::ALLOC <= 232448, "shared memory budget");
 
 // Barrier indices.
 enum TcBar : int {
-    B_KQ_FULL = 0,     // [2] TMA K/Q landed (tx)
+    B_KQ_FULL = 0,     // [2] TMA K/Q and the bulk copy of P landed (tx)
     B_KQ_EMPTY = 2,    // [2] serial MMAs of the stage's chunk done
     B_VT_FULL = 4,     // V, T''_hi, T''_lo landed (tx)
     B_VT_EMPTY = 5,    // U^T MMA reading V and T'' done
     B_GATE = 6,        // [4] gate stage written
-    B_S1_FULL = 10,    // S1 in TMEM
-    B_S1_FREE = 11,    // P rows read S1 (64)
-    B_TP_FULL = 12,    // T' landed (tx)
-    B_W_FULL = 13,     // W^T in TMEM (and T' read)
-    B_PREP = 14,       // [2] -W^T written (128)
-    B_P_READY = 16,    // [2] P written (64)
-    B_U_FULL = 18,     // U^T in TMEM (and -W^T no longer read)
-    B_U_CONV = 19,     // U, U.f split into bf16 hi/lo in TMEM (256)
-    B_H_FULL = 20,     // h^T MMA done
-    B_H_READY = 21,    // bf16 h^T of the next chunk staged in shared memory (256)
-    B_O_FULL = 22,     // O^T MMAs done
-    B_O_FREE = 23,     // O^T TMEM read (128)
-    B_DRAIN = 24,      // [2] final commit of each MMA issuer
-    B_HM_READY = 26,   // fp32 state in TMEM re-scaled by the next chunk's decay (256)
-    B_U_RND = 27,      // U in TMEM rounded to tf32 in place, for the O2 MMA (256)
-    B_STALL = 28,      // diagnostic only: nothing ever arrives on it (gdn_debug_stall)
+    B_TP_FULL = 10,    // T' landed (tx)
+    B_W_FULL = 11,     // W^T in TMEM (and T' read)
+    B_PREP = 12,       // [2] -W^T written (128)
+    B_U_FULL = 14,     // U^T in TMEM (and -W^T no longer read)
+    B_U_CONV = 15,     // U, U.f split into bf16 hi/lo in TMEM (256)
+    B_H_FULL = 16,     // h^T MMA done
+    B_H_READY = 17,    // bf16 h^T of the next chunk staged in shared memory (256)
+    B_O_FULL = 18,     // O^T MMAs done
+    B_O_FREE = 19,     // O^T TMEM read (128)
+    B_DRAIN = 20,      // [2] final commit of each MMA issuer
+    B_HM_READY = 22,   // fp32 state in TMEM re-scaled by the next chunk's decay (256)
+    B_U_RND = 23,      // U in TMEM rounded to tf32 in place, for the O2 MMA (256)
+    B_STALL = 24,      // diagnostic only: nothing ever arrives on it (gdn_debug_stall)
 };
 
 // Limit of the diagnostic wait on B_STALL (~1 ms): short, so the time-out path runs quickly.
 constexpr long long kStallLimitCycles = 2000000LL;
 
 // TMEM columns.  U^T is accumulated in fp32 at TM_U and read there, as tf32, by the O2 MMA; the state
-// warpgroups write U diag f as bf16 hi/lo pairs (two values per column) to TM_UF for the h^T MMA.
-constexpr uint32_t TM_S1 = 0, TM_W = 64, TM_U = 128, TM_UF = 192, TM_O1 = 256, TM_O2 = 320, TM_H = 384,
-                   TM_COLS = 512;
+// warpgroups write U diag f as bf16 hi/lo pairs (two values per column) to TM_UF for the h^T MMA.  Columns
+// 0-63 are not used.
+constexpr uint32_t TM_W = 64, TM_U = 128, TM_UF = 192, TM_O1 = 256, TM_O2 = 320, TM_H = 384, TM_COLS = 512;
 
-// Warp roles (16 warps): 0 TMA producer (K, Q, V, T', T'') and gates; 1 issues S1 and W^T; 2 issues the
-// serial MMAs (U^T, h^T, O^T); 3 idle; 4-7 (prep / output warpgroup) write -W^T, in quadrants 2-3 P, and
-// store o; 8-11 and 12-15 (state warpgroups, one per half of U and of the key channels) split U into bf16
-// operands, refresh the bf16 copy of h^T (double-buffered), re-scale the fp32 state by the next chunk's
-// decay and write hT.
+// Warp roles (16 warps): 0 TMA producer (K, Q, V; bulk copies of T', T'' and P) and gates; 1 issues W^T; 2
+// issues the serial MMAs (U^T, h^T, O^T); 3 idle; 4-7 (prep / output warpgroup) write -W^T and store o; 8-11
+// and 12-15 (state warpgroups, one per half of U and of the key channels) split U into bf16 operands, refresh
+// the bf16 copy of h^T (double-buffered), re-scale the fp32 state by the next chunk's decay and write hT.
 template <bool O_F32>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -600,7 +615,6 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             uint32_t cnt = 1;
             if (b == B_U_CONV || b == B_U_RND || b == B_H_READY || b == B_HM_READY) cnt = 256;
             if (b == B_PREP || b == B_PREP + 1 || b == B_O_FREE) cnt = 128;
-            if (b == B_S1_FREE || b == B_P_READY || b == B_P_READY + 1) cnt = 64;
             mbar_init(&bars[b], cnt);
         }
         *abort_flag = 0;
@@ -661,11 +675,13 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (lane == 0) {
                     uint8_t* dst = sm + L::KQ + st * L::KQ_STAGE;
                     const int tok = (int)(seq_start + c2 * kChunk);
-                    mbar_expect_tx(&bars[B_KQ_FULL + st], 32768);
+                    mbar_expect_tx(&bars[B_KQ_FULL + st], 32768 + 16384);
                     tma_load_3d(dst + 0, &tm_k, &bars[B_KQ_FULL + st], 0, h, tok);
                     tma_load_3d(dst + 8192, &tm_q, &bars[B_KQ_FULL + st], 0, h, tok);
                     tma_load_3d(dst + 16384, &tm_k, &bars[B_KQ_FULL + st], 64, h, tok);
                     tma_load_3d(dst + 24576, &tm_q, &bars[B_KQ_FULL + st], 64, h, tok);
+                    bulk_load(sm + L::PH + st * 8192, wy_unit(c2) + kWyP, 8192, &bars[B_KQ_FULL + st]);
+                    bulk_load(sm + L::PL + st * 8192, wy_unit(c2) + kWyP + 8192, 8192, &bars[B_KQ_FULL + st]);
                 }
                 kq_issued[st]++;
                 tc_make_gates(gates[c2 & 3], p, (size_t)(seq_start + c2 * kChunk), min(kChunk, eos - bos - c2 * kChunk),
@@ -681,25 +697,15 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (vt_issued > 0) drain_wait(&bars[B_VT_FULL], (vt_issued - 1) & 1);
         if (tp_issued > 0) drain_wait(&bars[B_TP_FULL], (tp_issued - 1) & 1);
     } else if (warp == 1) {
-        // ================================================================ S1 = [K; Q] K^T and W^T = K^T T'^T
+        // ================================================================ W^T = K^T T'^T
         if (lane == 0) {
-            const uint32_t id_s1 = idesc_bf16(128, 64, false, false);
             const uint32_t id_w = idesc_bf16(128, 64, true, false);
             const uint32_t n16 = 2u << 17;  // N += 16 in an instruction descriptor (N / 8 at bit 17)
             const uint64_t d_tp = desc_k_sw128(sbase + L::TP);
             for (int c = 0; c < nc; ++c) {
                 const int st = c & 1;
                 if (!mbar_wait(&bars[B_KQ_FULL + st], (c >> 1) & 1, abort_flag, err)) break;
-                if (c >= 1 && !mbar_wait(&bars[B_S1_FREE], (c - 1) & 1, abort_flag, err)) break;
-                tc_fence_after();
-                const uint64_t d = desc_k_sw128(sbase + L::KQ + st * L::KQ_STAGE);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t a = d + (kk >> 2) * 1024 + (kk & 3) * 2;
-                    umma_bf16(tmem + TM_S1, a, a, id_s1, kk > 0);
-                }
-                umma_commit(&bars[B_S1_FULL]);
-                // W^T: T' of this chunk has landed and -W^T of the previous one has been read out of TMEM
+                // W^T: K and T' of this chunk have landed and -W^T of the previous one has been read out of TMEM
                 if (!mbar_wait(&bars[B_TP_FULL], c & 1, abort_flag, err)) break;
                 if (c >= 1 && !mbar_wait(&bars[B_PREP + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, err)) break;
                 tc_fence_after();
@@ -779,11 +785,11 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const uint32_t o = (kk >> 2) * 1024 + (kk & 3) * 2;
                     umma_bf16(tmem + TM_O1, d_ht + o, d_q + o, id_o, kk > 0);
                 }
-                if (!mbar_wait(&bars[B_P_READY + st], (c >> 1) & 1, abort_flag, err)) break;
                 if (!mbar_wait(&bars[B_U_RND], c & 1, abort_flag, err)) break;
                 tc_fence_after();
-                // O2^T = U^T P^T on kind::tf32: U fp32 straight from TM_U, P fp32 (tokens 0-31 in PH, 32-63 in
-                // PL); k-step ks8 covers 8 tokens and, P being lower triangular, only columns r >= 16 (ks8 / 2)
+                // O2^T = U^T P^T on kind::tf32: U fp32 straight from TM_U, P (columns 0-31 in PH, 32-63 in PL,
+                // from the workspace with this chunk's K/Q stage); k-step ks8 covers 8 tokens and, P being lower
+                // triangular, only columns r >= 16 (ks8 / 2)
 #pragma unroll
                 for (int ks8 = 0; ks8 < 8; ++ks8) {
                     const int r0 = 16 * (ks8 >> 1);
@@ -802,13 +808,12 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // idle: its TMEM lane quadrant is served by warps 7, 11 and 15
     } else if (warp < 8) {
         // ================================================================ prep / output warpgroup
-        // Iteration k: (1) -W^T of chunk k, line i = t, from TMEM into shared memory.  (2) The P rows of
-        // chunk k (the quadrant-2/3 warps, whose TMEM lanes hold Q K^T).  (3) The output tile of chunk k - 1:
-        // O1^T and O2^T read from TMEM (then released for the next chunk's O^T MMAs), combined and stored
-        // to global memory, one token row per store (a warp writes 32 consecutive values of the row).  The
-        // warps run independently; a timed-out wait does not break out, the warp finishes the iteration
+        // Iteration k: (1) -W^T of chunk k, line i = t, from TMEM into shared memory.  (2) The output tile of
+        // chunk k - 1: O1^T and O2^T read from TMEM (then released for the next chunk's O^T MMAs), combined and
+        // stored to global memory, one token row per store (a warp writes 32 consecutive values of the row).
+        // The warps run independently; a timed-out wait does not break out, the warp finishes the iteration
         // and leaves at the top of the next.
-        const int t = tid - 128;  // TMEM lane: value column j of O^T / line of W^T / row of S1
+        const int t = tid - 128;  // TMEM lane: value column j of O^T / line of W^T
         const int wid = warp & 3;
         const uint32_t lane_base = 32 * wid;
         for (int k = 0; k <= nc; ++k) {
@@ -828,18 +833,6 @@ gdn_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 fence_proxy_async();
                 tc_fence_before();
                 mbar_arrive(&bars[B_PREP + st]);
-                if (wid >= 2) {
-                    warp_wait(&bars[B_S1_FULL], c & 1, abort_flag, err);
-                    warp_wait(&bars[B_GATE + (c & 3)], (c >> 2) & 1, abort_flag, err);
-                    tc_fence_after();
-                    // rows 0-31 need columns 0-31 only: the O^T MMA never reads the blocks above the diagonal
-                    tc_row_pass<false>(taddr(tmem, lane_base, TM_S1), gates[c & 3], t - 64, 0, wid == 2 ? 31 : 63,
-                                       nullptr, sm + L::PH + st * 8192, sm + L::PL + st * 8192);
-                    fence_proxy_async();
-                    mbar_arrive(&bars[B_P_READY + st]);
-                    tc_fence_before();
-                    mbar_arrive(&bars[B_S1_FREE]);
-                }
             }
             if (k >= 1) {
                 const int c = k - 1;
@@ -1053,7 +1046,8 @@ inline gdn_status launch_tc(const FwdParams& p, bool o_f32, void* ws, size_t ws_
         return GDN_ERR_UNSUPPORTED;
     }
     ProfScope prof_wy(PK_TC_WY, stream);
-    gdn_tc_wy_kernel<<<(unsigned)wy_grid, kWyThreads, WySmem::ALLOC, stream>>>(mk, p, static_cast<uint8_t*>(ws), err);
+    gdn_tc_wy_kernel<<<(unsigned)wy_grid, kWyThreads, WySmem::ALLOC, stream>>>(mq, mk, p, static_cast<uint8_t*>(ws),
+                                                                                err);
     prof_wy.done();
     e = cudaGetLastError();
     if (e != cudaSuccess) {

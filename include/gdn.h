@@ -45,9 +45,10 @@
  * *_fwd call: the caller owns every buffer, and work is enqueued on `stream` (asynchronous).
  *
  * Workspace: the tensor-core path (bf16 inputs, dk == 128, dv a multiple of 128) first computes the WY
- * factors of every (chunk, head) -- T' = T diag(beta e^G) and T'' = T diag(beta) with T = (I + A)^-1 --
- * into `workspace`, then runs the chunk recurrence that reads them; it needs gdn_workspace_bytes() bytes
- * (24 KB per chunk slot and head; slots = ceil(B T / 64) + number of sequences).  The workspace is scratch:
+ * factors of every (chunk, head) -- T' = T diag(beta e^G) and T'' = T diag(beta) with T = (I + A)^-1 -- and
+ * the gated read-out matrix P of every chunk into `workspace`, then runs the chunk recurrence that reads them;
+ * it needs gdn_workspace_bytes() bytes (40 KB per chunk slot and head; slots = ceil(B T / 64) + number of
+ * sequences).  The workspace is scratch:
  * its contents are undefined before and after a call, and it must not be shared by calls in flight at the
  * same time.  With a smaller (or NULL) workspace, AUTO runs the SIMT kernel and TC returns
  * GDN_ERR_UNSUPPORTED.  The GDN-2 and KDA tensor-core path (same shape rule) keeps, per chunk slot and head, an
@@ -104,12 +105,12 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          const int32_t* cu_seqlens, int n_seqs,
                          void* workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Size of the scratch array compiled into the library for gdn_chunk_fwd_noalloc: 128 MiB of device memory.  It is
+/* Size of the scratch array compiled into the library for gdn_chunk_fwd_noalloc: 256 MiB of device memory.  It is
  * part of the library's device code, so the CUDA runtime reserves it on each device where it loads that code and
  * keeps it until the process exits.  With lazy module loading (the CUDA default) that happens during the first
  * call of ANY libgdn entry point on a device -- also in processes that never call gdn_chunk_fwd_noalloc -- and
  * that first call can therefore fail with GDN_ERR_CUDA (out of memory) on a nearly full device. */
-#define GDN_STATIC_WS_BYTES (128u * 1024u * 1024u)
+#define GDN_STATIC_WS_BYTES (256u * 1024u * 1024u)
 
 /* gdn_chunk_fwd for callers that cannot allocate device memory.  (The pages have no counterpart to this entry
  * point: it exists for the library's users.)  Some callers may not call cudaMalloc at all: serving engines that
@@ -216,6 +217,35 @@ gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const floa
                          float* dg, float* dbeta, float* dh0, int B, int T, int H, int dk_, int dv_, int BT,
                          gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs, void* workspace, size_t ws_bytes,
                          cudaStream_t stream);
+
+/* Backward pass of gdn2_chunk_fwd (GDN-2) and of gdn_kda_chunk_fwd (KDA): the gradients of <d_o, o> + <dhT, hT>
+ * with respect to q, k, v, the per-channel decay g, the gates and h0.  (Gated DeltaNet-2 article, section
+ * "Entrenamiento fragmentado y reconocimiento de puertas hacia atras": the gate factors sit inside the gradient's
+ * dot products; the walkthrough's section "Chunked parallelism" names the full backward.)  Same structure as
+ * gdn_chunk_bwd, with the decay of every key channel inside A and P: the states at every chunk start are
+ * recomputed, T = (I + A)^-1 and P of every chunk are formed into the workspace, the state cotangent is carried
+ * from the last chunk to the first, and the input gradients of every chunk are formed in parallel.  The gate
+ * gradient of channel i at row r comes out of the identity dGn_ri = q_ri dq_ri + e_ri de_ri - k_ri dk_ri (every
+ * q and erase key carries exp(+G), every key exp(-G)) plus the chunk-end terms, then a reverse cumulative sum.
+ * Arithmetic is fp32 on CUDA cores for both input dtypes.
+ * GDN-2: g, b [B,T,H,dk], w [B,T,H,dv] fp32; outputs dq, dk, dg, db [B,T,H,dk], dv, dw [B,T,H,dv].
+ * KDA: g [B,T,H,dk], beta [B,T,H] fp32; outputs dq, dk, dg [B,T,H,dk], dv [B,T,H,dv], dbeta [B,T,H] (beta is
+ * both the erase and the write strength, so dbeta sums both shares).
+ * Both: d_o [B,T,H,dv] in `dt`; h0, dhT [N,H,dk,dv] fp32 or NULL (zeros); dh0 [N,H,dk,dv] or NULL (not
+ * written); every output fp32, overwritten.  Workspace: gdn2_bwd_workspace_bytes() bytes (two fp32 states and
+ * the fp32 T and P of every chunk slot and head), required.  Shapes, cu_seqlens and errors as for
+ * gdn_chunk_fwd. */
+size_t gdn2_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs);
+gdn_status gdn2_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* b, const float* w,
+                          float scale, const float* h0, const void* d_o, const float* dhT, float* dq, float* dk,
+                          float* dv, float* dg, float* db, float* dw, float* dh0, int B, int T, int H, int dk_, int dv_,
+                          int BT, gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs, void* workspace,
+                          size_t ws_bytes, cudaStream_t stream);
+gdn_status gdn_kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             float scale, const float* h0, const void* d_o, const float* dhT, float* dq, float* dk,
+                             float* dv, float* dg, float* dbeta, float* dh0, int B, int T, int H, int dk_, int dv_,
+                             int BT, gdn_dtype dt, const int32_t* cu_seqlens, int n_seqs, void* workspace,
+                             size_t ws_bytes, cudaStream_t stream);
 
 /* Selects the kernel family for later calls from any thread (process-wide; default AUTO). */
 gdn_status gdn_set_kernel(gdn_kernel kernel);

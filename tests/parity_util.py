@@ -131,3 +131,14 @@ def unit_slices(inp, o, hT, unit):
     n, h = unit
     row, t0, t1 = seq_spans(inp)[n]
     return f64(o[row, t0:t1, h]), f64(hT[n, h])
+
+
+def cotangents(inp, seed):
+    """Seeded output and final-state cotangents of a backward test: d_o in q's dtype, dhT fp32."""
+    rng = np.random.default_rng(seed)
+    B, T, H, dk = inp["q"].shape
+    dv = inp["v"].shape[-1]
+    n = B if inp["cu_seqlens"] is None else inp["cu_seqlens"].numel() - 1
+    d_o = torch.from_numpy(rng.standard_normal((B, T, H, dv)).astype(np.float32)).to(inp["q"].dtype)
+    dhT = torch.from_numpy((rng.standard_normal((n, H, dk, dv)) * 0.5).astype(np.float32))
+    return d_o, dhT

@@ -31,7 +31,7 @@ def test_header_declares_the_entry_points():
               "gdn_chunk_fwd_noalloc", "gdn_profile_enable", "gdn_profile_take", "gdn2_workspace_bytes",
               "gdn_kda_chunk_fwd", "gdn_debug_stall", "gdn_decode_fwd", "gdn2_decode_fwd",
               "gdn_kda_decode_fwd", "gdn_prelude_fwd", "gdn_output_gate_fwd", "gdn_bwd_workspace_bytes",
-              "gdn_chunk_bwd"]:
+              "gdn_chunk_bwd", "gdn2_bwd_workspace_bytes", "gdn2_chunk_bwd", "gdn_kda_chunk_bwd"]:
         assert n in names
 
 
@@ -129,10 +129,10 @@ def test_status_strings_and_kernel_choice(lib):
         assert lib.gdn_status_string(s).decode() not in ("", "unknown status")
     assert lib.gdn_set_kernel(9) == 1
     assert lib.gdn_set_kernel(0) == 0
-    # the tensor-core path keeps 24 KB of WY factors per (chunk slot, head); slots = ceil(B T / 64) + sequences
-    assert lib.gdn_workspace_bytes(4, 4096, 16, 128, 256, 64, 0) == (256 + 4) * 16 * 24576
-    assert lib.gdn_workspace_bytes(1, 65536, 16, 128, 256, 64, 16) == (1024 + 16) * 16 * 24576
-    assert lib.gdn_workspace_bytes(1, 100, 2, 128, 128, 64, 0) == (2 + 1) * 2 * 24576
+    # the tensor-core path keeps 40 KB of WY factors and P per (chunk slot, head); slots = ceil(B T / 64) + sequences
+    assert lib.gdn_workspace_bytes(4, 4096, 16, 128, 256, 64, 0) == (256 + 4) * 16 * 40960
+    assert lib.gdn_workspace_bytes(1, 65536, 16, 128, 256, 64, 16) == (1024 + 16) * 16 * 40960
+    assert lib.gdn_workspace_bytes(1, 100, 2, 128, 128, 64, 0) == (2 + 1) * 2 * 40960
     assert lib.gdn_workspace_bytes(4, 4096, 16, 64, 64, 64, 0) == 0  # shapes only the SIMT kernel takes
     assert lib.gdn_workspace_bytes(4, 0, 16, 128, 256, 64, 0) == 0
     # GDN-2 / KDA: one 82432-byte unit (T hi/lo, -W^T, P, Q', K~, Lambda) per chunk slot and head
@@ -164,3 +164,48 @@ def test_noalloc_entry_checks_arguments_before_touching_the_device(lib, kw, stat
                                    vp(args["cu"]), args["n_seqs"], None)
     assert st == status
     assert lib.gdn_last_error().decode() != ""
+
+
+def test_gdn2_bwd_workspace_adds_t_and_p_of_every_chunk(lib):
+    lib.gdn_bwd_workspace_bytes.restype = lib.gdn2_bwd_workspace_bytes.restype = ctypes.c_size_t
+    B, T, H, dk, dv = 2, 130, 3, 128, 64
+    slots = -(-B * T // 64) + B
+    states = lib.gdn_bwd_workspace_bytes(B, T, H, dk, dv, 64, 0)
+    assert states == 2 * slots * H * dk * dv * 4
+    assert lib.gdn2_bwd_workspace_bytes(B, T, H, dk, dv, 64, 0) == states + slots * H * 2 * 64 * 64 * 4
+    assert lib.gdn2_bwd_workspace_bytes(B, T, H, 96, dv, 64, 0) == 0  # unsupported dk
+
+
+def call_bwd2(lib, kda=False, **kw):
+    args = dict(q=A, k=A, v=A, g=A, b=A, w=A, d_o=A, dq=A, dk=A, dv=A, dg=A, db=A, dw=A, B=1, T=64, H=1, dk_=64,
+                dv_=64, dt=1, ws=A, ws_bytes=1 << 30)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    tail = (args["B"], args["T"], args["H"], args["dk_"], args["dv_"], 64, args["dt"], None, 0, vp(args["ws"]),
+            ctypes.c_size_t(args["ws_bytes"]), None)
+    if kda:
+        return lib.gdn_kda_chunk_bwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]), vp(args["b"]),
+                                     ctypes.c_float(0.125), None, vp(args["d_o"]), None, vp(args["dq"]),
+                                     vp(args["dk"]), vp(args["dv"]), vp(args["dg"]), vp(args["db"]), None, *tail)
+    return lib.gdn2_chunk_bwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]), vp(args["b"]),
+                              vp(args["w"]), ctypes.c_float(0.125), None, vp(args["d_o"]), None, vp(args["dq"]),
+                              vp(args["dk"]), vp(args["dv"]), vp(args["dg"]), vp(args["db"]), vp(args["dw"]), None,
+                              *tail)
+
+
+@pytest.mark.parametrize("kda", [False, True])
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(d_o=None), 1), (dict(g=None), 1), (dict(b=None), 1), (dict(dq=None), 1),
+    (dict(db=None), 1), (dict(dg=A + 4), 1), (dict(ws_bytes=1024), 1), (dict(ws=None, ws_bytes=0), 1),
+    (dict(dk_=96), 2), (dict(dv_=320), 2), (dict(dt=5), 2),
+])
+def test_gdn2_bwd_host_checks(lib, kda, kw, status):
+    lib.gdn2_chunk_bwd.restype = lib.gdn_kda_chunk_bwd.restype = ctypes.c_int
+    assert call_bwd2(lib, kda, **kw) == status
+    assert lib.gdn_last_error().decode() != ""
+
+
+def test_gdn2_bwd_needs_the_write_gate_and_its_gradient(lib):
+    lib.gdn2_chunk_bwd.restype = ctypes.c_int
+    assert call_bwd2(lib, w=None) == 1
+    assert call_bwd2(lib, dw=None) == 1

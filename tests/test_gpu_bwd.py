@@ -8,22 +8,11 @@ import pytest
 import torch
 
 from gated_delta_rule_105_b200.inputs import WORKLOADS, generate, generate_workload
-from parity_util import TOL, f64, relerr, seq_spans
+from parity_util import TOL, cotangents, f64, relerr, seq_spans
 
 pytestmark = pytest.mark.gpu
 
 GRADS = ("dq", "dk", "dv", "dg", "dbeta", "dh0")
-
-
-def cotangents(inp, seed):
-    """Seeded output and final-state cotangents: d_o in q's dtype, dhT fp32."""
-    rng = np.random.default_rng(seed)
-    B, T, H, dk = inp["q"].shape
-    dv = inp["v"].shape[-1]
-    n = B if inp["cu_seqlens"] is None else inp["cu_seqlens"].numel() - 1
-    d_o = torch.from_numpy(rng.standard_normal((B, T, H, dv)).astype(np.float32)).to(inp["q"].dtype)
-    dhT = torch.from_numpy((rng.standard_normal((n, H, dk, dv)) * 0.5).astype(np.float32))
-    return d_o, dhT
 
 
 def run_gpu(inp, d_o, dhT):
