@@ -104,8 +104,8 @@ __device__ __forceinline__ uint32_t f2tf32(float x) {
 
 // One row r of A (IS_A: beta_r Gamma_rs (k_r . k_s), s < r, fp32 into `arow`) or of P (Gamma_rs (q_r . k_s),
 // s <= r, rounded to tf32 and stored as fp32 in the 128B-swizzled K-major layout of a kind::tf32 operand:
-// columns 0-31 in `ph`, 32-63 in `pl`), columns [s_lo, s_hi], from the dot products in TMEM (`ta` = this
-// warp's lanes, column of s = 0).  Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1) is a
+// columns 0-31 in `ph`, 32-63 in `pl`, in shared or global memory), columns [s_lo, s_hi], from the dot products
+// in TMEM (`ta` = this warp's lanes, column of s = 0).  Gamma_rs = 2^(G_r - G_s) = a_r a_(r-1) ... a_(s+1) is a
 // running product down from the highest column at or below r, started there with one exp2.
 template <bool IS_A>
 __device__ __forceinline__ void tc_row_pass(uint32_t ta, const TcGate& gs, int r, int s_lo, int s_hi, float* arow,
@@ -392,11 +392,10 @@ __device__ __forceinline__ void wy_unit_of_slot(const FwdParams& p, long long sl
 // ------------------------------------------------------------------------------------------ the WY kernel
 // Shared-memory map (bytes from a 1024-aligned base).  The S1 MMA reads a 128-row A operand per 64-channel
 // panel, rows 0-63 the K tile and rows 64-127 the Q tile ([K0 | Q0 | K1 | Q1], as in the chunk kernel), and K
-// as its B operand.  Once S1 is in TMEM the four panels are free: the P rows go to Q0 (columns 0-31) and Q1
-// (columns 32-63) and are stored from there; then the inverse writes T''_lo over K0, T''_hi over Q0 and T' over K1.
+// as its B operand.  Once S1 is in TMEM the four panels are free: the inverse writes T''_lo over K0, T''_hi over
+// Q0 and T' over K1 (the P rows go straight to the workspace).
 struct WySmem {
     static constexpr uint32_t K0 = 0, Q0 = 8192, K1 = 16384, Q1 = 24576;  // [64 tokens][128 B] swizzled each
-    static constexpr uint32_t PH = Q0, PL = Q1;  // P, columns 0-31 and 32-63 (tf32 [r][s])
     static constexpr uint32_t TPPL = K0, TPP = Q0, TP = K1;
     static constexpr uint32_t AS = 32768;  // A, then (I+A)^-1, fp32 [64][68]
     static constexpr uint32_t GATE = AS + 64 * kAsLd * 4;
@@ -470,14 +469,15 @@ __global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_cons
     __syncwarp();
     const bool ok = warp_wait(&bars[1], 0, abort_flag, err);
     tc_fence_after();
-    // rows of A (warps 0-1, TMEM lanes 0-63) and of P (warps 2-3, lanes 64-127); P rows 0-31 need columns 0-31
-    // only, the chunk kernel's MMA never reads the blocks above the diagonal
+    // rows of A (warps 0-1, TMEM lanes 0-63) and of P (warps 2-3, lanes 64-127, written straight to the unit in the
+    // workspace); P rows 0-31 need columns 0-31 only, the chunk kernel's MMA never reads the blocks above the
+    // diagonal
+    uint8_t* dst = ws + ((size_t)slot * p.H + h) * kWyUnit;
     if (ok) {
         if (warp < 2) tc_row_pass<true>(taddr(tmem, 32 * warp, 0), gs, tid, 0, 63, sA + tid * kAsLd, nullptr, nullptr);
         else tc_row_pass<false>(taddr(tmem, 32 * warp, 0), gs, tid - 64, 0, warp == 2 ? 31 : 63, nullptr,
-                                sm + L::PH, sm + L::PL);
+                                dst + kWyP, dst + kWyP + 8192);
     }
-    fence_proxy_async();
     tc_fence_before();
     const bool all_ok = __syncthreads_and(ok) != 0;  // one outcome for the CTA: the inverse has barriers
     if (warp == 0) {
@@ -485,14 +485,6 @@ __global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_cons
         tmem_dealloc(tmem, 64);
     }
     if (!all_ok) return;
-    uint8_t* dst = ws + ((size_t)slot * p.H + h) * kWyUnit;
-    if (tid == 0) {  // P, read out of shared memory before the inverse writes T''_hi over it
-        bulk_store(dst + kWyP, sm + L::PH, 8192);
-        bulk_store(dst + kWyP + 8192, sm + L::PL, 8192);
-        bulk_commit();
-        bulk_wait_read();
-    }
-    __syncthreads();
     const TEmit em{sm + L::TP, sm + L::TPP, sm + L::TPPL, gs.beta, gs.eG};
     invert_unit_lower64(sA, warp, lane, 1, em);
     fence_proxy_async();
@@ -502,7 +494,7 @@ __global__ void __launch_bounds__(kWyThreads) gdn_tc_wy_kernel(const __grid_cons
         bulk_store(dst + 8192, sm + L::TPP, 8192);
         bulk_store(dst + 16384, sm + L::TPPL, 8192);
         bulk_commit();
-        bulk_wait_all();
+        bulk_wait_read();  // the CTA may exit once the stores have read shared memory
     }
 }
 
