@@ -565,9 +565,8 @@ def run_row(args, w):
     profile_enable(False)
     taken = profile_take()
     n_l, ms_l = taken[kname]
-    if args.path == "bwd":  # the backward's forward recompute (the SIMT kernel) belongs to the same step
-        n0, ms0 = taken.get("gdn_simt_fwd_kernel", (n_l, 0.0))
-        ms_l = ms_l + ms0 * n_l / max(n0, 1)
+    if args.path == "bwd":  # the backward's forward recompute (SIMT or tensor-core kernels) belongs to the same step
+        ms_l = sum(ms * n_l / max(n, 1) for name, (n, ms) in taken.items() if name != kname) + ms_l
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
     with sampler:

@@ -417,7 +417,8 @@ def output_gate_fwd(o, z, weight, eps=1e-5, y=None):
 
 
 def bwd_workspace_bytes(B, T, H, dk, dv, BT=64, n_seqs=0) -> int:
-    """Device workspace (bytes) ``gdn_chunk_bwd`` needs: two fp32 states per chunk slot and head."""
+    """Device workspace (bytes) ``gdn_chunk_bwd`` needs: two fp32 states and the fp32 T and P of every chunk slot
+    and head."""
     return int(load_library().gdn_bwd_workspace_bytes(B, T, H, dk, dv, BT, n_seqs))
 
 

@@ -783,7 +783,7 @@ gdn2_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float val = p.scale * (v1[q] + v2[q]);
-                        if (r8 + q < Lc) {
+                        if (r8 + q < Lc && p.o) {  // o is null when only the chunk states are wanted
                             if (O_F32) static_cast<float*>(p.o)[off] = val;
                             else static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(val);
                         }
@@ -800,6 +800,16 @@ gdn2_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
         const int j = tid & 127;
         const uint32_t lane_base = 32 * (warp & 3);
         const float* lam = reinterpret_cast<const float*>(sm + L::LAM);
+        // backward pass only: the state at the start of chunk c, key channels [32 piece, 32 piece + 32)
+        auto dump_state = [&](int c, int piece, const float(&v)[32]) {
+            float* hp = p.h_chunks + ((size_t)wy_slot(n, seq_start, c) * H + h) * kTcDK * (size_t)dv + j0 +
+                        (size_t)(32 * piece) * dv + j;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                *hp = v[q];
+                hp += dv;
+            }
+        };
         // initial state: bf16 copy and fp32 master pre-scaled by the first chunk's per-channel decay
         if (warp_wait(&bars[G_LAM_FULL + 0], 0, abort_flag, err)) {
 #pragma unroll 1
@@ -811,6 +821,7 @@ gdn2_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
                     v[q] = hp ? *hp : 0.f;
                     hp += hp ? dv : 0;
                 }
+                if (p.h_chunks) dump_state(0, piece, v);
                 st_half_line_bf16(sm + L::HT + (piece >> 1) * 16384, j, 4 * (piece & 1), v);
 #pragma unroll
                 for (int q = 0; q < 32; ++q) v[q] *= lam[32 * piece + q];
@@ -861,6 +872,7 @@ gdn2_tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
                 if (!last) {
                     st_half_line_bf16(sm + L::HT + (c1 & 1) * L::HT_STAGE + (piece >> 1) * 16384, j, 4 * (piece & 1),
                                       v);
+                    if (p.h_chunks) dump_state(c1, piece, v);
                 } else if (p.hT) {
                     float* hp = p.hT + state_base + (size_t)(32 * piece) * dv + j;
 #pragma unroll

@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
+#include <type_traits>
 
 #include "gdn.h"
 #include "gdn_common.cuh"
@@ -247,26 +248,59 @@ static gdn_status launch_out_gate(const OutGateParams& p, cudaStream_t stream) {
 }
 
 // ---- backward
-inline size_t bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int n_seqs) {
+// Two fp32 states per chunk slot and head (the chunk-start states, the end-state cotangents), then T and P.
+inline size_t bwd_state_bytes(int B, int T, int H, int dk, int dv, int n_seqs) {
     return 2 * (size_t)wy_slots(B, T, n_seqs) * H * (size_t)dk * dv * sizeof(float);
+}
+inline size_t bwd_tp_bytes(int B, int T, int H, int n_seqs) {
+    return (size_t)wy_slots(B, T, n_seqs) * H * 2 * kChunk * kChunk * sizeof(float);
+}
+inline size_t bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int n_seqs) {
+    return bwd_state_bytes(B, T, H, dk, dv, n_seqs) + bwd_tp_bytes(B, T, H, n_seqs);
+}
+
+// The state at every chunk start, for the backward pass (o not written).  GDN with bf16 inputs of a shape the
+// tensor-core forward takes runs that forward, with the part of the backward workspace that the later kernels
+// fill (`tc_ws`) as its scratch; everything else runs the SIMT forward.  (GDN-2 keeps the SIMT states: its
+// gate gradient sums terms much larger than itself, and the bf16 operands of the tensor-core GDN-2 state,
+// ~3e-3 of its RMS, came out at 3-10e-2 of dg's RMS against a 2e-2 bound.)
+template <typename TIn, int DK, bool GDN2>
+static gdn_status bwd_chunk_states(const FwdParams& fp, void* tc_ws, size_t tc_ws_bytes, unsigned* err,
+                                   cudaStream_t stream) {
+    if (!GDN2 && std::is_same<TIn, __nv_bfloat16>::value && g_kernel_choice.load() != GDN_KERNEL_SIMT &&
+        tc_supported(fp)) {
+        const gdn_status st = launch_tc(fp, false, tc_ws, tc_ws_bytes, err, stream);
+        if (st == GDN_OK) return st;
+        if (st != GDN_ERR_UNSUPPORTED) return fail(st, "tcgen05 forward of the backward pass: %s", tc_last_error());
+    }
+    return launch_simt_dk<TIn, float, DK, GDN2>(fp, err, stream);
 }
 
 template <typename TIn, int DK>
 static gdn_status launch_bwd_dk(const FwdParams& fp, const BwdParams& bp, unsigned* err, cudaStream_t stream) {
-    // (1) the state at every chunk start, from the SIMT forward (no o written)
-    gdn_status st = launch_simt_dk<TIn, float, DK, false>(fp, err, stream);
+    // (1) the state at every chunk start; the state-cotangent array serves as the tensor-core forward's scratch
+    const size_t state_bytes = wy_slots(bp.B, bp.T, bp.n_seq) * (size_t)bp.H * DK * (size_t)bp.vdim * sizeof(float);
+    gdn_status st = bwd_chunk_states<TIn, DK, false>(fp, bp.dh_chunks, state_bytes + bwd_tp_bytes(bp.B, bp.T, bp.H,
+                                                                                                 bp.n_seq), err, stream);
     if (st != GDN_OK) return st;
+    const long long grid = wy_slots(bp.B, bp.T, bp.n_seq) * bp.H;
+    if (grid > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "too many chunks for one launch");
     ProfScope prof(PK_BWD, stream);
-    // (2) the state cotangent, chunk by chunk backwards
+    // (2) T and P of every chunk
+    auto kp = gdn_bwd_prep_kernel<TIn, DK>;
+    cudaError_t e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwPrepSmem<DK>::bytes);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    if (grid > 0) kp<<<(unsigned)grid, kBwThreads, BwPrepSmem<DK>::bytes, stream>>>(bp, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward prep kernel: %s", cudaGetErrorString(e));
+    // (3) the state cotangent, chunk by chunk backwards
     auto kdh = gdn_bwd_dh_kernel<TIn, DK>;
-    cudaError_t e = cudaFuncSetAttribute(kdh, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwDhSmem<DK>::bytes);
+    e = cudaFuncSetAttribute(kdh, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwDhSmem<DK>::bytes);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     kdh<<<dim3(bp.vdim / BwDhSmem<DK>::DVT, bp.H, bp.n_seq), kBwThreads, BwDhSmem<DK>::bytes, stream>>>(bp, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward state kernel: %s", cudaGetErrorString(e));
-    // (3) every input gradient, all chunks at once
-    const long long grid = wy_slots(bp.B, bp.T, bp.n_seq) * bp.H;
-    if (grid > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "too many chunks for one launch");
+    // (4) every input gradient, all chunks at once
     auto kc = gdn_bwd_chunk_kernel<TIn, DK>;
     e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwChunkSmem<DK>::bytes);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -282,13 +316,16 @@ inline size_t bwd2_tp_bytes(int B, int T, int H, int n_seqs) {
     return (size_t)wy_slots(B, T, n_seqs) * H * 2 * kChunk * kChunk * sizeof(float);
 }
 inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv, int n_seqs) {
-    return bwd_workspace_bytes(B, T, H, dk, dv, n_seqs) + bwd2_tp_bytes(B, T, H, n_seqs);
+    return bwd_state_bytes(B, T, H, dk, dv, n_seqs) + bwd2_tp_bytes(B, T, H, n_seqs);
 }
 
 template <typename TIn, int DK>
 static gdn_status launch_bwd2_dk(const FwdParams& fp, const Bwd2Params& bp, unsigned* err, cudaStream_t stream) {
-    // (1) the state at every chunk start, from the SIMT forward (no o written)
-    gdn_status st = launch_simt_dk<TIn, float, DK, true>(fp, err, stream);
+    // (1) the state at every chunk start; the state-cotangent array and the T / P area after it (contiguous)
+    // serve as the tensor-core forward's scratch
+    const size_t state_bytes = wy_slots(bp.B, bp.T, bp.n_seq) * (size_t)bp.H * DK * (size_t)bp.vdim * sizeof(float);
+    gdn_status st = bwd_chunk_states<TIn, DK, true>(fp, bp.dh_chunks, state_bytes + bwd2_tp_bytes(bp.B, bp.T, bp.H,
+                                                                                                  bp.n_seq), err, stream);
     if (st != GDN_OK) return st;
     const long long grid = wy_slots(bp.B, bp.T, bp.n_seq) * bp.H;
     if (grid > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "too many chunks for one launch");
@@ -340,7 +377,7 @@ static gdn_status chunk_bwd2(const void* q, const void* k, const void* v, const 
     gdn_status es;
     unsigned* err = err_word_ptr(&es);
     if (!err) return es;
-    const size_t states = bwd_workspace_bytes(B, T, H, dk_, dv_, ns) / sizeof(float);
+    const size_t states = bwd_state_bytes(B, T, H, dk_, dv_, ns) / sizeof(float);
     float* hc = static_cast<float*>(workspace);
     float* dhc = hc + states / 2;
     float* tp = hc + states;
@@ -546,11 +583,13 @@ gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const floa
     gdn_status es;
     unsigned* err = err_word_ptr(&es);
     if (!err) return es;
+    const size_t states = bwd_state_bytes(B, T, H, dk_, dv_, cu_seqlens ? n_seq : 0) / sizeof(float);
     float* hc = static_cast<float*>(workspace);
-    float* dhc = hc + need / 2 / sizeof(float);
+    float* dhc = hc + states / 2;
+    float* tp = hc + states;
     FwdParams fp{q, k, v, g, beta, nullptr, h0, nullptr, nullptr, cu_seqlens, scale, B, T, H, dk_, dv_, n_seq};
     fp.h_chunks = hc;
-    BwdParams bp{q, k, v, g, beta, d_o, dhT, hc, dhc, dq, dk, dv, dg, dbeta, dh0, cu_seqlens, scale,
+    BwdParams bp{q, k, v, g, beta, d_o, dhT, hc, dhc, tp, dq, dk, dv, dg, dbeta, dh0, cu_seqlens, scale,
                  B, T, H, dk_, dv_, n_seq};
     if (dt == GDN_F32)
         return dk_ == 64 ? launch_bwd_dk<float, 64>(fp, bp, err, stream) : launch_bwd_dk<float, 128>(fp, bp, err, stream);

@@ -13,11 +13,12 @@
 // and from A, P, X, F, f, gamma to q, k, v, beta and the chunk-local cumulative gate; dg is the reverse cumulative
 // sum of the gate's gradient inside the chunk.
 //
-// Three kernels: (1) the SIMT forward kernel, asked to write the state at every chunk start (FwdParams::h_chunks);
-// (2) gdn_bwd_dh_kernel walks each sequence's chunks backwards with the state cotangent dh in shared memory (one
-// CTA per (sequence, head, 32 value columns), the value columns of dh never mix) and writes dh' of every chunk;
-// (3) gdn_bwd_chunk_kernel forms every input gradient of one (chunk, head), all chunks at once, walking the value
-// columns in tiles of 16 and keeping the key-side sums in registers.
+// Four kernels: (1) a forward kernel (the tensor-core one for bf16 inputs, else the SIMT one) writes the state at
+// every chunk start (FwdParams::h_chunks); (2) gdn_bwd_prep_kernel forms T and P of every chunk into the
+// workspace; (3) gdn_bwd_dh_kernel walks each sequence's chunks backwards with the state cotangent dh in shared
+// memory (one CTA per (sequence, head, 32 value columns), the value columns of dh never mix) and writes dh' of
+// every chunk; (4) gdn_bwd_chunk_kernel forms every input gradient of one (chunk, head), all chunks at once,
+// walking the value columns in tiles of 16 and keeping the key-side sums in registers.
 #pragma once
 
 #include "gdn_common.cuh"
@@ -36,6 +37,7 @@ struct BwdParams {
     const float* dhT;         // [N,H,dk,dv] or null
     const float* h_chunks;    // [slot][H][dk][dv]: the state at each chunk's start (from the forward)
     float* dh_chunks;         // [slot][H][dk][dv]: the cotangent of the state at each chunk's end
+    float* tp;                // [slot][H][2][64][64]: T, then P, of every chunk (from the prep kernel)
     float* dq;                // [B,T,H,dk] fp32
     float* dk;
     float* dv;                // [B,T,H,dv] fp32
@@ -135,6 +137,59 @@ __device__ void bw_chunk_prep(const BwChunk<DK>& c, const BwdParams& p, size_t t
     }
 }
 
+// Loads one chunk as bw_chunk_prep does, but takes T and P from the prep kernel's output (`tp`: T then P,
+// [64][64] each) instead of forming A, P and the inverse again; Gamma (0 above the diagonal) is formed only when
+// `want_gm`.  The padded rows of K and Q are zero, as there.
+template <typename TIn, int DK>
+__device__ void bw_chunk_load(const BwChunk<DK>& c, const BwdParams& p, size_t tok0, int h, int Lc, const float* tp,
+                              bool want_gm) {
+    constexpr int LDK = BwChunk<DK>::LDK, LDT = BwChunk<DK>::LDT, NT = kBwThreads;
+    const int tid = threadIdx.x, H = p.H;
+    const TIn* q = static_cast<const TIn*>(p.q);
+    const TIn* k = static_cast<const TIn*>(p.k);
+    __syncthreads();  // the previous user of these buffers is done
+    for (int e = tid; e < kChunk * DK; e += NT) {
+        const int r = e / DK, i = e % DK;
+        float kv = 0.f, qv = 0.f;
+        if (r < Lc) {
+            const size_t idx = ((tok0 + r) * H + h) * DK + i;
+            kv = to_f32(k[idx]);
+            qv = to_f32(q[idx]);
+        }
+        c.K[r * LDK + i] = kv;
+        c.Q[r * LDK + i] = qv;
+    }
+    for (int e = tid; e < kChunk * kChunk; e += NT) {
+        c.T[(e / kChunk) * LDT + e % kChunk] = tp[e];
+        c.P[(e / kChunk) * LDT + e % kChunk] = tp[kChunk * kChunk + e];
+    }
+    if (tid < kChunk) {
+        const bool ok = tid < Lc;
+        c.beta[tid] = ok ? p.beta[(tok0 + tid) * H + h] : 0.f;
+        c.G[tid] = ok ? (double)p.g[(tok0 + tid) * H + h] : 0.0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double acc = 0.0;
+        for (int r = 0; r < kChunk; ++r) {
+            acc += c.G[r];
+            c.G[r] = acc * kLog2eD;
+        }
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        c.F[tid] = exp2f((float)c.G[tid]);
+        c.f[tid] = exp2f((float)(c.G[kChunk - 1] - c.G[tid]));
+        if (tid == 0) c.gamma[0] = exp2f((float)c.G[kChunk - 1]);
+    }
+    if (want_gm)
+        for (int e = tid; e < kChunk * kChunk; e += NT) {
+            const int r = e / kChunk, s2 = e % kChunk;
+            c.Gm[r * LDT + s2] = s2 <= r ? exp2f((float)(c.G[r] - c.G[s2])) : 0.f;
+        }
+    __syncthreads();
+}
+
 // Sequence bounds (row, first token, end) of sequence n; false (and the error word) for a bad cu_seqlens entry.
 __device__ __forceinline__ bool bw_seq_bounds(const BwdParams& p, int n, int& row, int& bos, int& eos, unsigned* err) {
     if (p.cu_seqlens) {
@@ -151,6 +206,28 @@ __device__ __forceinline__ bool bw_seq_bounds(const BwdParams& p, int n, int& ro
         eos = p.T;
     }
     return true;
+}
+
+// The (first global token, length) of the chunk in workspace slot `slot` into info[0], info[1] (length 0 for a slot
+// no chunk uses): the largest sequence n with wy_slot(n, start_n, 0) <= slot, then the chunk within it.
+__device__ __forceinline__ void bw_slot_chunk(const BwdParams& p, long long slot, int* info, unsigned* err) {
+    int lo = 0, hi = p.n_seq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        const long long st0 = p.cu_seqlens ? (long long)p.cu_seqlens[mid] : (long long)mid * p.T;
+        if (wy_slot(mid, st0, 0) <= slot) lo = mid;
+        else hi = mid - 1;
+    }
+    int row, bos, eos, Lc = 0;
+    if (bw_seq_bounds(p, lo, row, bos, eos, err)) {
+        const long long start = (long long)row * p.T + bos;
+        const long long cc = slot - wy_slot(lo, start, 0);
+        if (cc >= 0 && cc * kChunk < eos - bos) {
+            Lc = min(kChunk, (int)(eos - bos - cc * kChunk));
+            info[0] = (int)(start + cc * kChunk);
+        }
+    }
+    info[1] = Lc;
 }
 
 template <int DK>
@@ -196,13 +273,14 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams 
     for (int ci = nc - 1; ci >= 0; --ci) {
         const int Lc = min(kChunk, eos - bos - ci * kChunk);
         const size_t tok0 = (size_t)(start + (long long)ci * kChunk);
-        bw_chunk_prep<TIn, DK>(c, p, tok0, h, Lc);
+        const long long slot = wy_slot(n, start, ci);
+        bw_chunk_load<TIn, DK>(c, p, tok0, h, Lc, p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk, false);
         for (int e = tid; e < kChunk * DVT; e += NT) {
             const int r = e / DVT, j = e % DVT;
             sDo[r * LDV + j] = r < Lc ? to_f32(dout[((tok0 + r) * H + h) * dv + j0 + j]) : 0.f;
         }
         // dh' of this chunk (its end state's cotangent) for the gradient kernel
-        float* dh_out = p.dh_chunks + ((size_t)wy_slot(n, start, ci) * H + h) * DK * (size_t)dv + j0;
+        float* dh_out = p.dh_chunks + ((size_t)slot * H + h) * DK * (size_t)dv + j0;
         for (int e = tid; e < DK * DVT; e += NT) {
             const int i = e / DVT, j = e % DVT;
             dh_out[(size_t)i * dv + j] = sDh[i * LDV + j];
@@ -252,6 +330,44 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams 
             const int i = e / DVT, j = e % DVT;
             p.dh0[state_base + (size_t)i * dv + j] = sDh[i * LDV + j];
         }
+}
+
+// (2) One CTA per (chunk slot, head): T = (I + A)^-1 and P of the chunk (bw_chunk_prep) into the workspace, so
+// that the state-cotangent kernel (every value slice of every chunk) and the gradient kernel read them instead
+// of forming them again.
+template <int DK>
+struct BwPrepSmem {  // 4-byte words: the bw_chunk_prep operands
+    static constexpr int LDK = DK + 1, LDT = kChunk + 1;
+    static constexpr int oK = 0, oQ = oK + kChunk * LDK, oGm = oQ + kChunk * LDK, oT = oGm + kChunk * LDT;
+    static constexpr int oP = oT + kChunk * LDT, oA = oP + kChunk * LDT;
+    static constexpr int oG = oA + kChunk * LDT;  // double [64]
+    static constexpr int oBeta = oG + 2 * kChunk, oF = oBeta + kChunk, of = oF + kChunk, oGam = of + kChunk;
+    static constexpr int total = oGam + 4;
+    static constexpr size_t bytes = sizeof(float) * (size_t)total;
+};
+
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(kBwThreads) gdn_bwd_prep_kernel(const BwdParams p, unsigned* err) {
+    using L = BwPrepSmem<DK>;
+    extern __shared__ __align__(16) float bsm[];
+    const BwChunk<DK> c{bsm + L::oK, bsm + L::oQ, bsm + L::oGm, bsm + L::oT, bsm + L::oP, bsm + L::oA,
+                        reinterpret_cast<double*>(bsm + L::oG), bsm + L::oBeta, bsm + L::oF, bsm + L::of,
+                        bsm + L::oGam};
+    __shared__ int info[2];
+    const int tid = threadIdx.x, H = p.H;
+    const long long slot = blockIdx.x / H;
+    const int h = blockIdx.x % H;
+    if (tid == 0) bw_slot_chunk(p, slot, info, err);
+    __syncthreads();
+    const int Lc = info[1];
+    if (Lc == 0) return;
+    bw_chunk_prep<TIn, DK>(c, p, (size_t)info[0], h, Lc);
+    __syncthreads();
+    float* out = p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk;
+    for (int e = tid; e < kChunk * kChunk; e += kBwThreads) {
+        out[e] = c.T[(e / kChunk) * L::LDT + e % kChunk];
+        out[kChunk * kChunk + e] = c.P[(e / kChunk) * L::LDT + e % kChunk];
+    }
 }
 
 template <int DK>
@@ -306,26 +422,7 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
     const int tid = threadIdx.x, H = p.H, dv = p.vdim;
     const long long slot = blockIdx.x / H;
     const int h = blockIdx.x % H;
-    if (tid == 0) {
-        // the (sequence, chunk) of this slot: largest n with wy_slot(n, start_n, 0) <= slot
-        int lo = 0, hi = p.n_seq - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            const long long st0 = p.cu_seqlens ? (long long)p.cu_seqlens[mid] : (long long)mid * p.T;
-            if (wy_slot(mid, st0, 0) <= slot) lo = mid;
-            else hi = mid - 1;
-        }
-        int row, bos, eos, Lc = 0;
-        if (bw_seq_bounds(p, lo, row, bos, eos, err)) {
-            const long long start = (long long)row * p.T + bos;
-            const long long cc = slot - wy_slot(lo, start, 0);
-            if (cc >= 0 && cc * kChunk < eos - bos) {
-                Lc = min(kChunk, (int)(eos - bos - cc * kChunk));
-                info[0] = (int)(start + cc * kChunk);
-            }
-        }
-        info[1] = Lc;
-    }
+    if (tid == 0) bw_slot_chunk(p, slot, info, err);
     __syncthreads();
     const int Lc = info[1];
     if (Lc == 0) return;
@@ -335,7 +432,7 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
     const float* hc = p.h_chunks + ((size_t)slot * H + h) * DK * (size_t)dv;
     const float* dhc = p.dh_chunks + ((size_t)slot * H + h) * DK * (size_t)dv;
 
-    bw_chunk_prep<TIn, DK>(c, p, tok0, h, Lc);
+    bw_chunk_load<TIn, DK>(c, p, tok0, h, Lc, p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk, true);
     for (int e = tid; e < kChunk * LDT; e += NT) {
         sdT[e] = 0.f;
         sdP[e] = 0.f;

@@ -210,7 +210,9 @@ gdn_status gdn_output_gate_fwd(const void* o, const void* z, const float* weight
  * Layouts: q, k, v, d_o as for gdn_chunk_fwd (d_o [B,T,H,dv] in `dt`); g, beta [B,T,H] fp32; h0, dhT
  * [N,H,dk,dv] fp32 or NULL (zeros); outputs dq, dk [B,T,H,dk], dv [B,T,H,dv], dg, dbeta [B,T,H] and dh0
  * [N,H,dk,dv] (NULL: not written), all fp32, overwritten.  Workspace: gdn_bwd_workspace_bytes() bytes (two fp32
- * states per chunk slot and head), required.  Shapes, cu_seqlens and errors as for gdn_chunk_fwd. */
+ * states and the fp32 T and P of every chunk slot and head), required.  bf16 inputs of a tensor-core shape
+ * recompute the chunk-start states with the tensor-core forward, everything else with the SIMT forward.
+ * Shapes, cu_seqlens and errors as for gdn_chunk_fwd. */
 size_t gdn_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int BT, int n_seqs);
 gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta, float scale,
                          const float* h0, const void* d_o, const float* dhT, float* dq, float* dk, float* dv,

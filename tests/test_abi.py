@@ -166,13 +166,13 @@ def test_noalloc_entry_checks_arguments_before_touching_the_device(lib, kw, stat
     assert lib.gdn_last_error().decode() != ""
 
 
-def test_gdn2_bwd_workspace_adds_t_and_p_of_every_chunk(lib):
+def test_bwd_workspace_holds_two_states_and_t_and_p_of_every_chunk(lib):
     lib.gdn_bwd_workspace_bytes.restype = lib.gdn2_bwd_workspace_bytes.restype = ctypes.c_size_t
     B, T, H, dk, dv = 2, 130, 3, 128, 64
     slots = -(-B * T // 64) + B
-    states = lib.gdn_bwd_workspace_bytes(B, T, H, dk, dv, 64, 0)
-    assert states == 2 * slots * H * dk * dv * 4
-    assert lib.gdn2_bwd_workspace_bytes(B, T, H, dk, dv, 64, 0) == states + slots * H * 2 * 64 * 64 * 4
+    need = 2 * slots * H * dk * dv * 4 + slots * H * 2 * 64 * 64 * 4
+    assert lib.gdn_bwd_workspace_bytes(B, T, H, dk, dv, 64, 0) == need
+    assert lib.gdn2_bwd_workspace_bytes(B, T, H, dk, dv, 64, 0) == need
     assert lib.gdn2_bwd_workspace_bytes(B, T, H, 96, dv, 64, 0) == 0  # unsupported dk
 
 
