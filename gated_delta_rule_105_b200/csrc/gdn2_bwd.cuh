@@ -21,10 +21,11 @@
 // chunk; db = K . dE and dk = dK + b . dE; dv = w . dX and dw = V . dX (KDA: dbeta_r = sum_i K_ri dE_ri +
 // sum_j V_rj dX_rj, dv = beta dX).
 //
-// Four kernels: (1) the SIMT forward kernel writes the state at every chunk start (FwdParams::h_chunks);
-// (2) gdn2_bwd_prep_kernel forms T and P of every (chunk, head) into the workspace; (3) gdn2_bwd_dh_kernel walks
-// each sequence's chunks backwards with dh in shared memory (one CTA per (sequence, head, 32 value columns)) and
-// writes dh' of every chunk; (4) gdn2_bwd_chunk_kernel forms every input gradient of one (chunk, head).
+// Four kernels: (1) gdn2_bwd_prep_kernel forms T and P of every (chunk, head) into the workspace;
+// (2) gdn2_bwd_states_kernel walks each sequence's chunks forward with T and writes the state at every chunk start;
+// (3) gdn2_bwd_dh_kernel walks them backwards with dh in shared memory (one CTA per (sequence, head, 32 value
+// columns)) and writes dh' of every chunk; (4) gdn2_bwd_chunk_kernel forms every input gradient of one
+// (chunk, head).
 #pragma once
 
 #include "gdn_common.cuh"
@@ -55,6 +56,7 @@ struct Bwd2Params {
     const int32_t* cu_seqlens;
     float scale;
     int B, T, H, kdim, vdim, n_seq, kda;
+    const float* h0;          // [N,H,dk,dv] or null (zeros): the initial state of the forward walk
 };
 
 // Sequence bounds (row, first token, end) of sequence n; false (and the error word) for a bad cu_seqlens entry.
@@ -133,7 +135,7 @@ __device__ __forceinline__ void bw2_invert_lower(const float* A, float* T, int l
     }
 }
 
-// (2) One CTA per (chunk slot, head): T and P of the chunk into the workspace.
+// (0) One CTA per (chunk slot, head): T and P of the chunk into the workspace.
 template <int DK>
 struct Bw2PrepSmem {  // 4-byte words; the cumulative gate is fp64, transposed [channel][row]
     static constexpr int LDK = DK + 1, LDT = kChunk + 1;
@@ -233,6 +235,105 @@ __device__ void bw2_scaled_rows(const Bwd2Params& p, size_t tok0, int h, int Lc,
             if (QF) QF[r * ldk + i] = qv * F;
             if (EF) EF[r * ldk + i] = bv * kv * F;
             if (Kf) Kf[r * ldk + i] = kv * f;
+        }
+    }
+}
+
+// (1) One CTA per (sequence, head, 32 value columns): the state at every chunk start, walked forward with T from
+// the prep kernel (the forward's recurrence without its output): X = Z - (E . F) h, U = T X,
+// h' = Diag(Lambda) h + (K . f)^T U.  The value columns of the state never mix, so the slices are exact.
+template <int DK>
+struct Bw2StSmem {  // 4-byte words
+    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 32, LDV = DVT + 1;
+    static constexpr int oT = 0, oEF = oT + kChunk * LDT, oKf = oEF + kChunk * LDK, oLam = oKf + kChunk * LDK;
+    static constexpr int oH = oLam + DK;         // h [DK][LDV]
+    static constexpr int oZ = oH + DK * LDV;     // Z = w . V [64][LDV]
+    static constexpr int oX = oZ + kChunk * LDV, oU = oX + kChunk * LDV;
+    static constexpr int total = oU + kChunk * LDV;
+    static constexpr size_t bytes = sizeof(float) * (size_t)total;
+};
+
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_states_kernel(const Bwd2Params p, unsigned* err) {
+    using L = Bw2StSmem<DK>;
+    constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBw2Threads;
+    extern __shared__ __align__(16) float bsm[];
+    float* sT = bsm + L::oT;
+    float* sEF = bsm + L::oEF;
+    float* sKf = bsm + L::oKf;
+    float* sLam = bsm + L::oLam;
+    float* sH = bsm + L::oH;
+    float* sZ = bsm + L::oZ;
+    float* sX = bsm + L::oX;
+    float* sU = bsm + L::oU;
+    const int tid = threadIdx.x, j0 = blockIdx.x * DVT, h = blockIdx.y, n = blockIdx.z;
+    const int H = p.H, dv = p.vdim;
+    int row, bos, eos;
+    if (!bw2_seq_bounds(p, n, row, bos, eos, err)) return;
+    const long long start = (long long)row * p.T + bos;
+    const size_t state_base = ((size_t)n * H + h) * DK * (size_t)dv + j0;
+    for (int e = tid; e < DK * DVT; e += NT) {
+        const int i = e / DVT, j = e % DVT;
+        sH[i * LDV + j] = p.h0 ? p.h0[state_base + (size_t)i * dv + j] : 0.f;
+    }
+    // the states go into the workspace this launch owns (the parameter block holds them as read-only for the
+    // kernels that read them)
+    float* h_chunks = const_cast<float*>(p.h_chunks);
+    const TIn* vin = static_cast<const TIn*>(p.v);
+    const int nc = (eos - bos + kChunk - 1) / kChunk;
+    for (int ci = 0; ci < nc; ++ci) {
+        const int Lc = min(kChunk, eos - bos - ci * kChunk);
+        const size_t tok0 = (size_t)(start + (long long)ci * kChunk);
+        const long long slot = wy_slot(n, start, ci);
+        __syncthreads();  // the previous chunk is done with every buffer
+        float* h_out = h_chunks + ((size_t)slot * H + h) * DK * (size_t)dv + j0;
+        for (int e = tid; e < DK * DVT; e += NT) {
+            const int i = e / DVT, j = e % DVT;
+            h_out[(size_t)i * dv + j] = sH[i * LDV + j];
+        }
+        const float* tp = p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk;
+        for (int e = tid; e < kChunk * kChunk; e += NT) sT[(e / kChunk) * LDT + e % kChunk] = tp[e];
+        bw2_scaled_rows<TIn, DK>(p, tok0, h, Lc, nullptr, sEF, sKf, sLam, LDK);
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int r = e / DVT, j = e % DVT;
+            float z = 0.f;
+            if (r < Lc) {
+                const size_t tok = tok0 + r;
+                z = bw2_w(p, tok, h, j0 + j) * to_f32(vin[(tok * H + h) * dv + j0 + j]);
+            }
+            sZ[r * LDV + j] = z;
+        }
+        __syncthreads();
+        // X = Z - (E . F) h
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int r = e / DVT, j = e % DVT;
+            float acc = 0.f;
+            for (int i = 0; i < DK; ++i) acc = fmaf(sEF[r * LDK + i], sH[i * LDV + j], acc);
+            sX[r * LDV + j] = sZ[r * LDV + j] - acc;
+        }
+        __syncthreads();
+        // U = T X
+        for (int e = tid; e < kChunk * DVT; e += NT) {
+            const int r = e / DVT, j = e % DVT;
+            float acc = 0.f;
+            for (int s2 = 0; s2 <= r; ++s2) acc = fmaf(sT[r * LDT + s2], sX[s2 * LDV + j], acc);
+            sU[r * LDV + j] = acc;
+        }
+        __syncthreads();
+        // h' = Diag(Lambda) h + (K . f)^T U
+        float nh[DK * DVT / NT];
+#pragma unroll
+        for (int m = 0; m < DK * DVT / NT; ++m) {
+            const int e = tid + m * NT, i = e / DVT, j = e % DVT;
+            float acc = sLam[i] * sH[i * LDV + j];
+            for (int r = 0; r < kChunk; ++r) acc = fmaf(sKf[r * LDK + i], sU[r * LDV + j], acc);
+            nh[m] = acc;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < DK * DVT / NT; ++m) {
+            const int e = tid + m * NT;
+            sH[(e / DVT) * LDV + e % DVT] = nh[m];
         }
     }
 }

@@ -321,22 +321,24 @@ inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv, int n_se
 
 template <typename TIn, int DK>
 static gdn_status launch_bwd2_dk(const FwdParams& fp, const Bwd2Params& bp, unsigned* err, cudaStream_t stream) {
-    // (1) the state at every chunk start; the state-cotangent array and the T / P area after it (contiguous)
-    // serve as the tensor-core forward's scratch
-    const size_t state_bytes = wy_slots(bp.B, bp.T, bp.n_seq) * (size_t)bp.H * DK * (size_t)bp.vdim * sizeof(float);
-    gdn_status st = bwd_chunk_states<TIn, DK, true>(fp, bp.dh_chunks, state_bytes + bwd2_tp_bytes(bp.B, bp.T, bp.H,
-                                                                                                  bp.n_seq), err, stream);
-    if (st != GDN_OK) return st;
+    (void)fp;
     const long long grid = wy_slots(bp.B, bp.T, bp.n_seq) * bp.H;
     if (grid > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "too many chunks for one launch");
     ProfScope prof(PK_BWD, stream);
-    // (2) T and P of every chunk
+    // (0) T and P of every chunk
     auto kp = gdn2_bwd_prep_kernel<TIn, DK>;
     cudaError_t e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Bw2PrepSmem<DK>::bytes);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     if (grid > 0) kp<<<(unsigned)grid, kBw2Threads, Bw2PrepSmem<DK>::bytes, stream>>>(bp, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward prep kernel: %s", cudaGetErrorString(e));
+    // (1) the state at every chunk start, walked forward with T
+    auto kst = gdn2_bwd_states_kernel<TIn, DK>;
+    e = cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Bw2StSmem<DK>::bytes);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    kst<<<dim3(bp.vdim / Bw2StSmem<DK>::DVT, bp.H, bp.n_seq), kBw2Threads, Bw2StSmem<DK>::bytes, stream>>>(bp, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward state kernel: %s", cudaGetErrorString(e));
     // (3) the state cotangent, chunk by chunk backwards
     auto kdh = gdn2_bwd_dh_kernel<TIn, DK>;
     e = cudaFuncSetAttribute(kdh, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Bw2DhSmem<DK>::bytes);
@@ -385,7 +387,7 @@ static gdn_status chunk_bwd2(const void* q, const void* k, const void* v, const 
     fp.kda = kda ? 1 : 0;
     fp.h_chunks = hc;
     Bwd2Params bp{q, k, v, g, b, kda ? nullptr : w, d_o, dhT, hc, dhc, tp, dq, dk, dv, dg, db, kda ? nullptr : dw,
-                  dh0, cu_seqlens, scale, B, T, H, dk_, dv_, n_seq, kda ? 1 : 0};
+                  dh0, cu_seqlens, scale, B, T, H, dk_, dv_, n_seq, kda ? 1 : 0, h0};
     if (dt == GDN_F32)
         return dk_ == 64 ? launch_bwd2_dk<float, 64>(fp, bp, err, stream) : launch_bwd2_dk<float, 128>(fp, bp, err, stream);
     return dk_ == 64 ? launch_bwd2_dk<__nv_bfloat16, 64>(fp, bp, err, stream)
