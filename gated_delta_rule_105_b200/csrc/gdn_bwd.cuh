@@ -233,9 +233,10 @@ __device__ __forceinline__ void bw_slot_chunk(const BwdParams& p, long long slot
 template <int DK>
 struct BwDhSmem {  // 4-byte words
     static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 32, LDV = DVT + 1;
-    static constexpr int oK = 0, oQ = oK + kChunk * LDK, oGm = oQ + kChunk * LDK, oT = oGm + kChunk * LDT;
-    static constexpr int oP = oT + kChunk * LDT, oA = oP + kChunk * LDT;
-    static constexpr int oG = oA + kChunk * LDT;  // double [64]
+    // Q is scaled in place to scale diag(F) Q; KB = -diag(beta F) K
+    static constexpr int oK = 0, oQ = oK + kChunk * LDK, oKB = oQ + kChunk * LDK, oT = oKB + kChunk * LDK;
+    static constexpr int oP = oT + kChunk * LDT;
+    static constexpr int oG = oP + kChunk * LDT;  // double [64]
     static constexpr int oBeta = oG + 2 * kChunk, oF = oBeta + kChunk, of = oF + kChunk, oGam = of + kChunk;
     static constexpr int oDh = oGam + 4;          // dh [DK][LDV]
     static constexpr int oDo = oDh + DK * LDV;    // dO [64][LDV]
@@ -251,9 +252,10 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams 
     using L = BwDhSmem<DK>;
     constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBwThreads;
     extern __shared__ __align__(16) float bsm[];
-    const BwChunk<DK> c{bsm + L::oK, bsm + L::oQ, bsm + L::oGm, bsm + L::oT, bsm + L::oP, bsm + L::oA,
+    const BwChunk<DK> c{bsm + L::oK, bsm + L::oQ, nullptr, bsm + L::oT, bsm + L::oP, nullptr,
                         reinterpret_cast<double*>(bsm + L::oG), bsm + L::oBeta, bsm + L::oF, bsm + L::of,
                         bsm + L::oGam};
+    float* sKB = bsm + L::oKB;
     float* sDh = bsm + L::oDh;
     float* sDo = bsm + L::oDo;
     float* sDu = bsm + L::oDu;
@@ -275,6 +277,11 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams 
         const size_t tok0 = (size_t)(start + (long long)ci * kChunk);
         const long long slot = wy_slot(n, start, ci);
         bw_chunk_load<TIn, DK>(c, p, tok0, h, Lc, p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk, false);
+        for (int e = tid; e < kChunk * DK; e += NT) {  // the row factors of the dh update, once per chunk
+            const int r = e / DK, i = e % DK;
+            sKB[r * LDK + i] = -c.beta[r] * c.F[r] * c.K[r * LDK + i];
+            c.Q[r * LDK + i] *= p.scale * c.F[r];
+        }
         for (int e = tid; e < kChunk * DVT; e += NT) {
             const int r = e / DVT, j = e % DVT;
             sDo[r * LDV + j] = r < Lc ? to_f32(dout[((tok0 + r) * H + h) * dv + j0 + j]) : 0.f;
@@ -312,8 +319,8 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams 
             const int e = tid + m * NT, i = e / DVT, j = e % DVT;
             float a = 0.f;
             for (int r = 0; r < kChunk; ++r) {
-                a = fmaf(p.scale * c.F[r] * c.Q[r * LDK + i], sDo[r * LDV + j], a);
-                a = fmaf(-c.beta[r] * c.F[r] * c.K[r * LDK + i], sDx[r * LDV + j], a);
+                a = fmaf(c.Q[r * LDK + i], sDo[r * LDV + j], a);  // scale F_r q_r, scaled above
+                a = fmaf(sKB[r * LDK + i], sDx[r * LDV + j], a);
             }
             nd[m] = a + gam * sDh[i * LDV + j];
         }
