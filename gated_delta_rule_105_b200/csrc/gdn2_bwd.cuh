@@ -543,16 +543,33 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
             sDO[r * LDV + j] = ok ? to_f32(dout[idx]) : 0.f;
         }
         __syncthreads();
-        // X = w . V - (E . F) h ; (K . f) dh' (into dU for now)
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            float eh = 0.f, kd = 0.f;
+        // X = w . V - (E . F) h ; (K . f) dh' (into dU for now).  Each thread forms a 2 x 2 block (rows ra, ra + 32;
+        // columns jb, jb + 8), so every shared-memory operand it loads feeds two products.
+        static_assert(kChunk * DVT == 4 * NT && DVT == 16, "2 x 2 blocks cover the tile");
+        {
+            const int ra = tid >> 3, jb = tid & 7;
+            float eh[2][2] = {}, kd[2][2] = {};
+#pragma unroll 4
             for (int i = 0; i < DK; ++i) {
-                eh = fmaf(sEF[r * LDK + i], sH[i * LDV + j], eh);
-                kd = fmaf(sKf[r * LDK + i], sDH[i * LDV + j], kd);
+                const float h0 = sH[i * LDV + jb], h1 = sH[i * LDV + jb + 8];
+                const float d0 = sDH[i * LDV + jb], d1 = sDH[i * LDV + jb + 8];
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    const float ev = sEF[(ra + 32 * a) * LDK + i], kv = sKf[(ra + 32 * a) * LDK + i];
+                    eh[a][0] = fmaf(ev, h0, eh[a][0]);
+                    eh[a][1] = fmaf(ev, h1, eh[a][1]);
+                    kd[a][0] = fmaf(kv, d0, kd[a][0]);
+                    kd[a][1] = fmaf(kv, d1, kd[a][1]);
+                }
             }
-            sX[r * LDV + j] = sW[r * LDV + j] * sV[r * LDV + j] - eh;
-            sDU[r * LDV + j] = kd;
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const int r = ra + 32 * a, j = jb + 8 * b;
+                    sX[r * LDV + j] = sW[r * LDV + j] * sV[r * LDV + j] - eh[a][b];
+                    sDU[r * LDV + j] = kd[a][b];
+                }
         }
         __syncthreads();
         // U = T X ; dU = scale P^T dO + (K . f) dh'
