@@ -206,7 +206,8 @@ template <typename TIn, typename TOut>
 static gdn_status launch_decode_io(const DecodeParams& p, cudaStream_t stream) {
     auto kern = p.dk == 64 ? gdn_decode_kernel<TIn, TOut, 64> : gdn_decode_kernel<TIn, TOut, 128>;
     ProfScope prof(PK_DECODE, stream);
-    kern<<<(unsigned)((long long)p.N * p.H), p.dv / 4 * kDecRowGroups, 0, stream>>>(p);
+    const int tw = p.dv % 128 == 0 ? 128 : 64;  // value columns per CTA
+    kern<<<dim3((unsigned)((long long)p.N * p.H), (unsigned)(p.dv / tw)), tw / 4 * kDecRowGroups, 0, stream>>>(p);
     prof.done();
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "decode kernel launch: %s", cudaGetErrorString(e));
