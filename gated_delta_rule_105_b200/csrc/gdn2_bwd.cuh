@@ -28,6 +28,7 @@
 // (chunk, head).
 #pragma once
 
+#include "gdn_bwd_tiles.cuh"
 #include "gdn_common.cuh"
 
 namespace gdn {
@@ -110,15 +111,6 @@ __device__ __forceinline__ float bw2_b(const Bwd2Params& p, size_t tok, int h, i
 // Write-gate value w_rj.
 __device__ __forceinline__ float bw2_w(const Bwd2Params& p, size_t tok, int h, int j) {
     return p.kda ? p.b[tok * p.H + h] : p.w[(tok * p.H + h) * p.vdim + j];
-}
-
-// Chunk-local cumulative gate of channel i, in base 2: the value of row 63 (G_L; rows past Lc add 0).  The sum
-// runs in fp64; every kernel rounds it the same way, so T and P from the prep kernel and the gate terms of the
-// gradient kernel see identical G.
-__device__ __forceinline__ double bw2_gate_last(const Bwd2Params& p, size_t tok0, int h, int i, int Lc) {
-    double acc = 0.0;
-    for (int r = 0; r < Lc; ++r) acc += (double)p.g[((tok0 + r) * p.H + h) * p.kdim + i];
-    return acc * kLog2eD;
 }
 
 // T = (I + A)^-1 of a strictly lower A (row-major, leading dimension ldt), row by row, four adjacent threads per
@@ -211,44 +203,112 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_prep_kernel(const Bwd2Pa
 }
 
 // Per-channel chunk quantities from the inputs: QF = Q . F, EF = E . F, Kf = K . f and Lambda (any pointer may be
-// null).  One thread per channel walks the rows (the cumulative sum runs along them).
+// null).  Two threads per channel, one per half of the rows (threads past 2 * DK idle).  The cumulative sum runs
+// along the rows in fp64 in the prep kernel's order (row 0 first, rows past the chunk's end adding nothing): the
+// first half's total is handed to the second half, whose total is G_L.  Called by every thread of the block (it synchronises twice).
 template <typename TIn, int DK>
 __device__ void bw2_scaled_rows(const Bwd2Params& p, size_t tok0, int h, int Lc, float* QF, float* EF, float* Kf,
                                 float* Lam, int ldk) {
+    constexpr int RH = kChunk / 2;
+    __shared__ double carry[2 * DK];
     const TIn* q = static_cast<const TIn*>(p.q);
     const TIn* k = static_cast<const TIn*>(p.k);
-    for (int i = threadIdx.x; i < DK; i += blockDim.x) {
-        const double gl = bw2_gate_last(p, tok0, h, i, Lc);
-        if (Lam) Lam[i] = exp2f((float)gl);
-        double acc = 0.0;
-        for (int r = 0; r < kChunk; ++r) {
-            float kv = 0.f, qv = 0.f, bv = 0.f;
-            if (r < Lc) {
-                const size_t tok = tok0 + r, idx = (tok * p.H + h) * DK + i;
-                acc += (double)p.g[idx];
-                kv = to_f32(k[idx]);
-                if (QF) qv = to_f32(q[idx]);
-                bv = bw2_b(p, tok, h, i);
-            }
-            const double G = acc * kLog2eD;
-            const float F = exp2f((float)G), f = exp2f((float)(gl - G));
-            if (QF) QF[r * ldk + i] = qv * F;
-            if (EF) EF[r * ldk + i] = bv * kv * F;
-            if (Kf) Kf[r * ldk + i] = kv * f;
+    const int i = threadIdx.x % DK, half = threadIdx.x / DK, r0 = half * RH;
+    const bool act = half < 2;
+    const size_t H = p.H;
+    float gv[RH];
+#pragma unroll
+    for (int m = 0; m < RH; ++m) gv[m] = act && r0 + m < Lc ? p.g[((tok0 + r0 + m) * H + h) * DK + i] : 0.f;
+    double acc = 0.0;
+    if (half == 0) {
+#pragma unroll
+        for (int m = 0; m < RH; ++m) acc += (double)gv[m];
+        carry[i] = acc;
+    }
+    __syncthreads();
+    if (half == 1) {
+        acc = carry[i];
+#pragma unroll
+        for (int m = 0; m < RH; ++m) acc += (double)gv[m];
+        carry[DK + i] = acc;
+    }
+    __syncthreads();
+    if (!act) return;
+    const double gl = carry[DK + i] * kLog2eD;
+    if (Lam && half == 0) Lam[i] = exp2f((float)gl);
+    acc = half == 0 ? 0.0 : carry[i];
+#pragma unroll
+    for (int m = 0; m < RH; ++m) {
+        const int r = r0 + m;
+        float kv = 0.f, qv = 0.f, bv = 0.f;
+        if (r < Lc) {
+            const size_t tok = tok0 + r, idx = (tok * H + h) * DK + i;
+            kv = to_f32(k[idx]);
+            if (QF) qv = to_f32(q[idx]);
+            if (EF) bv = bw2_b(p, tok, h, i);
         }
+        acc += (double)gv[m];
+        const double G = acc * kLog2eD;
+        const float F = exp2f((float)G), f = exp2f((float)(gl - G));
+        if (QF) QF[r * ldk + i] = qv * F;
+        if (EF) EF[r * ldk + i] = bv * kv * F;
+        if (Kf) Kf[r * ldk + i] = kv * f;
+    }
+}
+
+// The same quantities from raw rows already in shared memory ([64][ldk]: g in G, q in QF, the erase gate b in EF
+// or, for KDA, beta per row in bt, k in Kf; rows past the chunk's end zero), in place: QF <- q F, EF <- b k F,
+// Kf <- k f, Lambda = 2^G_L.  Same threads, same fp64 sum order and same roundings as bw2_scaled_rows.  Called by
+// every thread of the block (it synchronises twice).
+template <int DK>
+__device__ void bw2_scale_rows_smem(const float* G, float* QF, float* EF, float* Kf, const float* bt, float* Lam,
+                                    int ldk) {
+    constexpr int RH = kChunk / 2;
+    __shared__ double carry[2 * DK];
+    const int i = threadIdx.x % DK, half = threadIdx.x / DK, r0 = half * RH;
+    double acc = 0.0;
+    if (half == 0) {
+#pragma unroll 8
+        for (int m = 0; m < RH; ++m) acc += (double)G[(r0 + m) * ldk + i];
+        carry[i] = acc;
+    }
+    __syncthreads();
+    if (half == 1) {
+        acc = carry[i];
+#pragma unroll 8
+        for (int m = 0; m < RH; ++m) acc += (double)G[(r0 + m) * ldk + i];
+        carry[DK + i] = acc;
+    }
+    __syncthreads();
+    if (half >= 2) return;
+    const double gl = carry[DK + i] * kLog2eD;
+    if (Lam && half == 0) Lam[i] = exp2f((float)gl);
+    acc = half == 0 ? 0.0 : carry[i];
+#pragma unroll 4
+    for (int m = 0; m < RH; ++m) {
+        const int e = (r0 + m) * ldk + i;
+        acc += (double)G[e];
+        const double Gd = acc * kLog2eD;
+        const float F = exp2f((float)Gd), f = exp2f((float)(gl - Gd));
+        const float kv = Kf[e];
+        if (QF) QF[e] *= F;
+        EF[e] = (bt ? bt[r0 + m] : EF[e]) * kv * F;
+        Kf[e] = kv * f;
     }
 }
 
 // (1) One CTA per (sequence, head, 32 value columns): the state at every chunk start, walked forward with T from
 // the prep kernel (the forward's recurrence without its output): X = Z - (E . F) h, U = T X,
-// h' = Diag(Lambda) h + (K . f)^T U.  The value columns of the state never mix, so the slices are exact.
+// h' = Diag(Lambda) h + (K . f)^T U, each as register tiles (gdn_bwd_tiles.cuh).  The value columns of the state
+// never mix, so the slices are exact.
 template <int DK>
-struct Bw2StSmem {  // 4-byte words
-    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 32, LDV = DVT + 1;
-    static constexpr int oT = 0, oEF = oT + kChunk * LDT, oKf = oEF + kChunk * LDK, oLam = oKf + kChunk * LDK;
-    static constexpr int oH = oLam + DK;         // h [DK][LDV]
-    static constexpr int oZ = oH + DK * LDV;     // Z = w . V [64][LDV]
-    static constexpr int oX = oZ + kChunk * LDV, oU = oX + kChunk * LDV;
+struct Bw2StSmem {  // 4-byte words; row strides padded to 16 bytes
+    static constexpr int LDK = DK + 4, LDT = kChunk + 4, DVT = kTileDv, LDV = kTileLdv;
+    static constexpr int oT = 0, oEF = oT + kChunk * LDT, oKf = oEF + kChunk * LDK, oG = oKf + kChunk * LDK;
+    static constexpr int oLam = oG + kChunk * LDK, oBt = oLam + DK;  // Lambda [DK]; KDA beta [64]
+    static constexpr int oH = oBt + kChunk;      // h [DK][LDV]
+    static constexpr int oZ = oH + DK * LDV;     // V [64][LDV]
+    static constexpr int oX = oZ + kChunk * LDV, oU = oX + kChunk * LDV;  // X (first the write gate w) and U
     static constexpr int total = oU + kChunk * LDV;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
@@ -256,12 +316,15 @@ struct Bw2StSmem {  // 4-byte words
 template <typename TIn, int DK>
 __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_states_kernel(const Bwd2Params p, unsigned* err) {
     using L = Bw2StSmem<DK>;
-    constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBw2Threads;
+    constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, IP = DK / 32;
+    static_assert(kBw2Threads == kTileThreads, "the register tiles assume 256 threads");
     extern __shared__ __align__(16) float bsm[];
     float* sT = bsm + L::oT;
     float* sEF = bsm + L::oEF;
     float* sKf = bsm + L::oKf;
+    float* sG = bsm + L::oG;
     float* sLam = bsm + L::oLam;
+    float* sBt = bsm + L::oBt;
     float* sH = bsm + L::oH;
     float* sZ = bsm + L::oZ;
     float* sX = bsm + L::oX;
@@ -272,96 +335,122 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_states_kernel(const Bwd2
     if (!bw2_seq_bounds(p, n, row, bos, eos, err)) return;
     const long long start = (long long)row * p.T + bos;
     const size_t state_base = ((size_t)n * H + h) * DK * (size_t)dv + j0;
-    for (int e = tid; e < DK * DVT; e += NT) {
-        const int i = e / DVT, j = e % DVT;
-        sH[i * LDV + j] = p.h0 ? p.h0[state_base + (size_t)i * dv + j] : 0.f;
-    }
+    tile_load_state(sH, p.h0 ? p.h0 + state_base : nullptr, dv, DK);
     // the states go into the workspace this launch owns (the parameter block holds them as read-only for the
     // kernels that read them)
     float* h_chunks = const_cast<float*>(p.h_chunks);
     const TIn* vin = static_cast<const TIn*>(p.v);
+    const TIn* k = static_cast<const TIn*>(p.k);
+    const int s0 = tile_s0(), tj = tile_j0(), wr = tile_warp_row(), i0 = tile_i0<DK>();
     const int nc = (eos - bos + kChunk - 1) / kChunk;
-    for (int ci = 0; ci < nc; ++ci) {
+    // the next chunk's operands, loaded into registers while the current one computes
+    RowBlock<float, kChunk> rt;
+    RowBlock<TIn, DVT> rv;
+    RowBlock<float, DVT> rw;
+    RowBlock<float, DK> rg, rb;
+    RowBlock<TIn, DK> rk;
+    float rbt = 0.f;
+    auto fetch = [&](int ci) {
         const int Lc = min(kChunk, eos - bos - ci * kChunk);
-        const size_t tok0 = (size_t)(start + (long long)ci * kChunk);
+        const size_t tok0 = (size_t)(start + (long long)ci * kChunk), rs = (size_t)H * DK;
+        rt.load(p.tp + ((size_t)wy_slot(n, start, ci) * H + h) * 2 * kChunk * kChunk, kChunk, kChunk);
+        rv.load(vin + (tok0 * H + h) * dv + j0, (size_t)H * dv, Lc);
+        rg.load(p.g + (tok0 * H + h) * DK, rs, Lc);
+        rk.load(k + (tok0 * H + h) * DK, rs, Lc);
+        if (p.kda) {
+            if (tid < kChunk) rbt = tid < Lc ? p.b[(tok0 + tid) * H + h] : 0.f;
+        } else {
+            rw.load(p.w + (tok0 * H + h) * dv + j0, (size_t)H * dv, Lc);
+            rb.load(p.b + (tok0 * H + h) * DK, rs, Lc);
+        }
+    };
+    if (nc > 0) fetch(0);
+    for (int ci = 0; ci < nc; ++ci) {
         const long long slot = wy_slot(n, start, ci);
         __syncthreads();  // the previous chunk is done with every buffer
-        float* h_out = h_chunks + ((size_t)slot * H + h) * DK * (size_t)dv + j0;
-        for (int e = tid; e < DK * DVT; e += NT) {
-            const int i = e / DVT, j = e % DVT;
-            h_out[(size_t)i * dv + j] = sH[i * LDV + j];
+        tile_store_state(h_chunks + ((size_t)slot * H + h) * DK * (size_t)dv + j0, dv, sH, DK);
+        rt.store(sT, LDT);
+        rv.store(sZ, LDV);
+        rg.store(sG, LDK);
+        rk.store(sKf, LDK);
+        if (p.kda) {
+            if (tid < kChunk) sBt[tid] = rbt;
+        } else {
+            rw.store(sX, LDV);
+            rb.store(sEF, LDK);
         }
-        const float* tp = p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk;
-        for (int e = tid; e < kChunk * kChunk; e += NT) sT[(e / kChunk) * LDT + e % kChunk] = tp[e];
-        bw2_scaled_rows<TIn, DK>(p, tok0, h, Lc, nullptr, sEF, sKf, sLam, LDK);
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            float z = 0.f;
-            if (r < Lc) {
-                const size_t tok = tok0 + r;
-                z = bw2_w(p, tok, h, j0 + j) * to_f32(vin[(tok * H + h) * dv + j0 + j]);
+        __syncthreads();
+        if (ci + 1 < nc) fetch(ci + 1);
+        bw2_scale_rows_smem<DK>(sG, nullptr, sEF, sKf, p.kda ? sBt : nullptr, sLam, LDK);
+        __syncthreads();
+        {  // X = w . V - (E . F) h (KDA: w = beta of the row); sX holds w until the thread's own tile is read
+            float a[2][4] = {};
+            tile_acc_AD<LDK>(sEF, sH, DK, a);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int s = s0 + u;
+                const float4 v = lds4(sZ + s * LDV + tj);
+                const float4 w = p.kda ? make_float4(sBt[s], sBt[s], sBt[s], sBt[s]) : lds4(sX + s * LDV + tj);
+                sts4(sX + s * LDV + tj, w.x * v.x - a[u][0], w.y * v.y - a[u][1], w.z * v.z - a[u][2],
+                     w.w * v.w - a[u][3]);
             }
-            sZ[r * LDV + j] = z;
         }
         __syncthreads();
-        // X = Z - (E . F) h
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            float acc = 0.f;
-            for (int i = 0; i < DK; ++i) acc = fmaf(sEF[r * LDK + i], sH[i * LDV + j], acc);
-            sX[r * LDV + j] = sZ[r * LDV + j] - acc;
-        }
-        __syncthreads();
-        // U = T X
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            float acc = 0.f;
-            for (int s2 = 0; s2 <= r; ++s2) acc = fmaf(sT[r * LDT + s2], sX[s2 * LDV + j], acc);
-            sU[r * LDV + j] = acc;
-        }
-        __syncthreads();
-        // h' = Diag(Lambda) h + (K . f)^T U
-        float nh[DK * DVT / NT];
+        {  // U = T X (T lower triangular: the warp's rows reach column 8w + 7 at most)
+            float a[2][4] = {};
+            tile_acc_AD<LDT>(sT, sX, wr + 8, a);
 #pragma unroll
-        for (int m = 0; m < DK * DVT / NT; ++m) {
-            const int e = tid + m * NT, i = e / DVT, j = e % DVT;
-            float acc = sLam[i] * sH[i * LDV + j];
-            for (int r = 0; r < kChunk; ++r) acc = fmaf(sKf[r * LDK + i], sU[r * LDV + j], acc);
-            nh[m] = acc;
+            for (int u = 0; u < 2; ++u) sts4(sU + (s0 + u) * LDV + tj, a[u][0], a[u][1], a[u][2], a[u][3]);
         }
         __syncthreads();
+        {  // h' = Diag(Lambda) h + (K . f)^T U on the thread's own rows and columns of h
+            float a[IP][4];
 #pragma unroll
-        for (int m = 0; m < DK * DVT / NT; ++m) {
-            const int e = tid + m * NT;
-            sH[(e / DVT) * LDV + e % DVT] = nh[m];
+            for (int u = 0; u < IP; ++u) {
+                const float lam = sLam[i0 + u];
+                const float4 d = lds4(sH + (i0 + u) * LDV + tj);
+                a[u][0] = lam * d.x;
+                a[u][1] = lam * d.y;
+                a[u][2] = lam * d.z;
+                a[u][3] = lam * d.w;
+            }
+            tile_acc_KtX<DK, LDK>(sKf, sU, a);
+#pragma unroll
+            for (int u = 0; u < IP; ++u) sts4(sH + (i0 + u) * LDV + tj, a[u][0], a[u][1], a[u][2], a[u][3]);
         }
     }
 }
 
 template <int DK>
-struct Bw2DhSmem {  // 4-byte words
-    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 32, LDV = DVT + 1;
+struct Bw2DhSmem {  // 4-byte words; row strides padded to 16 bytes
+    static constexpr int LDK = DK + 4, LDT = kChunk + 4, DVT = kTileDv, LDV = kTileLdv;
     static constexpr int oT = 0, oP = oT + kChunk * LDT, oQF = oP + kChunk * LDT, oEF = oQF + kChunk * LDK;
-    static constexpr int oKf = oEF + kChunk * LDK, oLam = oKf + kChunk * LDK;
-    static constexpr int oDh = oLam + DK;        // dh [DK][LDV]
-    static constexpr int oDo = oDh + DK * LDV;   // dO [64][LDV]
-    static constexpr int oDu = oDo + kChunk * LDV, oDx = oDu + kChunk * LDV;
+    static constexpr int oKf = oEF + kChunk * LDK, oG = oKf + kChunk * LDK, oLam = oG + kChunk * LDK;
+    static constexpr int oBt = oLam + DK;        // KDA beta [64]
+    static constexpr int oDh = oBt + kChunk;     // dh [DK][LDV]
+    static constexpr int oDo = oDh + DK * LDV;   // dO [64][LDV], then scale dO
+    static constexpr int oDu = oDo + kChunk * LDV, oDx = oDu + kChunk * LDV;  // dU; -dX
     static constexpr int total = oDx + kChunk * LDV;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
 
 // (3) One CTA per (sequence, head, 32 value columns): the state cotangent, walked from the last chunk to the first.
+// Per chunk: dU = scale P^T dO + (K . f) dh', dX = T^T dU, dh = (Q . F)^T (scale dO) + (E . F)^T (-dX)
+// + Diag(Lambda) dh', each as register tiles.
 template <typename TIn, int DK>
 __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_dh_kernel(const Bwd2Params p, unsigned* err) {
     using L = Bw2DhSmem<DK>;
-    constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBw2Threads;
+    constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, IP = DK / 32;
+    static_assert(kBw2Threads == kTileThreads, "the register tiles assume 256 threads");
     extern __shared__ __align__(16) float bsm[];
     float* sT = bsm + L::oT;
     float* sP = bsm + L::oP;
     float* sQF = bsm + L::oQF;
     float* sEF = bsm + L::oEF;
     float* sKf = bsm + L::oKf;
+    float* sG = bsm + L::oG;
     float* sLam = bsm + L::oLam;
+    float* sBt = bsm + L::oBt;
     float* sDh = bsm + L::oDh;
     float* sDo = bsm + L::oDo;
     float* sDu = bsm + L::oDu;
@@ -372,77 +461,98 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_dh_kernel(const Bwd2Para
     if (!bw2_seq_bounds(p, n, row, bos, eos, err)) return;
     const long long start = (long long)row * p.T + bos;
     const size_t state_base = ((size_t)n * H + h) * DK * (size_t)dv + j0;
-    for (int e = tid; e < DK * DVT; e += NT) {
-        const int i = e / DVT, j = e % DVT;
-        sDh[i * LDV + j] = p.dhT ? p.dhT[state_base + (size_t)i * dv + j] : 0.f;
-    }
+    tile_load_state(sDh, p.dhT ? p.dhT + state_base : nullptr, dv, DK);
+    const TIn* q = static_cast<const TIn*>(p.q);
+    const TIn* k = static_cast<const TIn*>(p.k);
     const TIn* dout = static_cast<const TIn*>(p.dout);
+    const int s0 = tile_s0(), tj = tile_j0(), wr = tile_warp_row(), i0 = tile_i0<DK>();
     const int nc = (eos - bos + kChunk - 1) / kChunk;
-    for (int ci = nc - 1; ci >= 0; --ci) {
+    // the next chunk's operands, loaded into registers while the current one computes
+    RowBlock<float, kChunk> rt, rp;
+    RowBlock<TIn, DVT> rdo;
+    RowBlock<float, DK> rg, rb;
+    RowBlock<TIn, DK> rk, rq;
+    float rbt = 0.f;
+    auto fetch = [&](int ci) {
         const int Lc = min(kChunk, eos - bos - ci * kChunk);
-        const size_t tok0 = (size_t)(start + (long long)ci * kChunk);
+        const size_t tok0 = (size_t)(start + (long long)ci * kChunk), rs = (size_t)H * DK;
+        const float* tp = p.tp + ((size_t)wy_slot(n, start, ci) * H + h) * 2 * kChunk * kChunk;
+        rt.load(tp, kChunk, kChunk);
+        rp.load(tp + kChunk * kChunk, kChunk, kChunk);
+        rdo.load(dout + (tok0 * H + h) * dv + j0, (size_t)H * dv, Lc);
+        rg.load(p.g + (tok0 * H + h) * DK, rs, Lc);
+        rk.load(k + (tok0 * H + h) * DK, rs, Lc);
+        rq.load(q + (tok0 * H + h) * DK, rs, Lc);
+        if (p.kda) {
+            if (tid < kChunk) rbt = tid < Lc ? p.b[(tok0 + tid) * H + h] : 0.f;
+        } else {
+            rb.load(p.b + (tok0 * H + h) * DK, rs, Lc);
+        }
+    };
+    if (nc > 0) fetch(nc - 1);
+    for (int ci = nc - 1; ci >= 0; --ci) {
         const long long slot = wy_slot(n, start, ci);
         __syncthreads();  // the previous chunk is done with every buffer
-        const float* tp = p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk;
-        for (int e = tid; e < kChunk * kChunk; e += NT) {
-            sT[(e / kChunk) * LDT + e % kChunk] = tp[e];
-            sP[(e / kChunk) * LDT + e % kChunk] = tp[kChunk * kChunk + e];
-        }
-        bw2_scaled_rows<TIn, DK>(p, tok0, h, Lc, sQF, sEF, sKf, sLam, LDK);
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            sDo[r * LDV + j] = r < Lc ? to_f32(dout[((tok0 + r) * H + h) * dv + j0 + j]) : 0.f;
+        rt.store(sT, LDT);
+        rp.store(sP, LDT);
+        rdo.store(sDo, LDV);
+        rg.store(sG, LDK);
+        rk.store(sKf, LDK);
+        rq.store(sQF, LDK);
+        if (p.kda) {
+            if (tid < kChunk) sBt[tid] = rbt;
+        } else {
+            rb.store(sEF, LDK);
         }
         // dh' of this chunk (its end state's cotangent) for the gradient kernel
-        float* dh_out = p.dh_chunks + ((size_t)slot * H + h) * DK * (size_t)dv + j0;
-        for (int e = tid; e < DK * DVT; e += NT) {
-            const int i = e / DVT, j = e % DVT;
-            dh_out[(size_t)i * dv + j] = sDh[i * LDV + j];
-        }
+        tile_store_state(p.dh_chunks + ((size_t)slot * H + h) * DK * (size_t)dv + j0, dv, sDh, DK);
         __syncthreads();
-        // dU = scale P^T dO + (K . f) dh'
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int s = e / DVT, j = e % DVT;
-            float acc = 0.f;
-            for (int r = s; r < kChunk; ++r) acc = fmaf(sP[r * LDT + s], sDo[r * LDV + j], acc);
-            float kd = 0.f;
-            for (int i = 0; i < DK; ++i) kd = fmaf(sKf[s * LDK + i], sDh[i * LDV + j], kd);
-            sDu[s * LDV + j] = p.scale * acc + kd;
-        }
+        if (ci > 0) fetch(ci - 1);
+        bw2_scale_rows_smem<DK>(sG, sQF, sEF, sKf, p.kda ? sBt : nullptr, sLam, LDK);
         __syncthreads();
-        // dX = T^T dU
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int s = e / DVT, j = e % DVT;
-            float acc = 0.f;
-            for (int r = s; r < kChunk; ++r) acc = fmaf(sT[r * LDT + s], sDu[r * LDV + j], acc);
-            sDx[s * LDV + j] = acc;
-        }
-        __syncthreads();
-        // dh = scale (Q . F)^T dO + Diag(Lambda) dh' - (E . F)^T dX
-        float nd[DK * DVT / NT];
+        {  // dU = scale P^T dO + (K . f) dh'
+            float a[2][4] = {};
+            tile_acc_AtX<LDT>(sP, sDo, wr, a);
 #pragma unroll
-        for (int m = 0; m < DK * DVT / NT; ++m) {
-            const int e = tid + m * NT, i = e / DVT, j = e % DVT;
-            float a = 0.f;
-            for (int r = 0; r < kChunk; ++r) {
-                a = fmaf(p.scale * sQF[r * LDK + i], sDo[r * LDV + j], a);
-                a = fmaf(-sEF[r * LDK + i], sDx[r * LDV + j], a);
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) a[u][c] *= p.scale;
+            tile_acc_AD<LDK>(sKf, sDh, DK, a);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) sts4(sDu + (s0 + u) * LDV + tj, a[u][0], a[u][1], a[u][2], a[u][3]);
+        }
+        __syncthreads();
+        {  // dX = T^T dU, kept as -dX; the thread's own tile of dO becomes scale dO
+            float x[2][4] = {};
+            tile_acc_AtX<LDT>(sT, sDu, wr, x);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int s = s0 + u;
+                sts4(sDx + s * LDV + tj, -x[u][0], -x[u][1], -x[u][2], -x[u][3]);
+                const float4 d = lds4(sDo + s * LDV + tj);
+                sts4(sDo + s * LDV + tj, p.scale * d.x, p.scale * d.y, p.scale * d.z, p.scale * d.w);
             }
-            nd[m] = a + sLam[i] * sDh[i * LDV + j];
         }
         __syncthreads();
+        {  // dh = (Q . F)^T (scale dO) + (E . F)^T (-dX) + Diag(Lambda) dh' on the thread's own tile of dh
+            float a[IP][4];
 #pragma unroll
-        for (int m = 0; m < DK * DVT / NT; ++m) {
-            const int e = tid + m * NT;
-            sDh[(e / DVT) * LDV + e % DVT] = nd[m];
+            for (int u = 0; u < IP; ++u) {
+                const float lam = sLam[i0 + u];
+                const float4 d = lds4(sDh + (i0 + u) * LDV + tj);
+                a[u][0] = lam * d.x;
+                a[u][1] = lam * d.y;
+                a[u][2] = lam * d.z;
+                a[u][3] = lam * d.w;
+            }
+            tile_acc_KtX<DK, LDK>(sQF, sDo, a);
+            tile_acc_KtX<DK, LDK>(sEF, sDx, a);
+#pragma unroll
+            for (int u = 0; u < IP; ++u) sts4(sDh + (i0 + u) * LDV + tj, a[u][0], a[u][1], a[u][2], a[u][3]);
         }
     }
     __syncthreads();
-    if (p.dh0)
-        for (int e = tid; e < DK * DVT; e += NT) {
-            const int i = e / DVT, j = e % DVT;
-            p.dh0[state_base + (size_t)i * dv + j] = sDh[i * LDV + j];
-        }
+    if (p.dh0) tile_store_state(p.dh0 + state_base, dv, sDh, DK);
 }
 
 template <int DK>

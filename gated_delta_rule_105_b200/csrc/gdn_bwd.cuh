@@ -21,6 +21,7 @@
 // walking the value columns in tiles of 16 and keeping the key-side sums in registers.
 #pragma once
 
+#include "gdn_bwd_tiles.cuh"
 #include "gdn_common.cuh"
 
 namespace gdn {
@@ -231,31 +232,61 @@ __device__ __forceinline__ void bw_slot_chunk(const BwdParams& p, long long slot
 }
 
 template <int DK>
-struct BwDhSmem {  // 4-byte words
-    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 32, LDV = DVT + 1;
-    // Q is scaled in place to scale diag(F) Q; KB = -diag(beta F) K
-    static constexpr int oK = 0, oQ = oK + kChunk * LDK, oKB = oQ + kChunk * LDK, oT = oKB + kChunk * LDK;
-    static constexpr int oP = oT + kChunk * LDT;
+struct BwDhSmem {  // 4-byte words; row strides padded to 16 bytes for the register-blocked products
+    static constexpr int LDK = DK + 4, LDT = kChunk + 4, DVT = kTileDv, LDV = kTileLdv;
+    static constexpr int oK = 0, oQ = oK + kChunk * LDK, oT = oQ + kChunk * LDK, oP = oT + kChunk * LDT;
     static constexpr int oG = oP + kChunk * LDT;  // double [64]
     static constexpr int oBeta = oG + 2 * kChunk, oF = oBeta + kChunk, of = oF + kChunk, oGam = of + kChunk;
     static constexpr int oDh = oGam + 4;          // dh [DK][LDV]
-    static constexpr int oDo = oDh + DK * LDV;    // dO [64][LDV]
+    static constexpr int oDo = oDh + DK * LDV;    // dO [64][LDV], then scale F dO
     static constexpr int oDu = oDo + kChunk * LDV;
-    static constexpr int oDx = oDu + kChunk * LDV;
+    static constexpr int oDx = oDu + kChunk * LDV;  // -beta F dX
     static constexpr int total = oDx + kChunk * LDV;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
 
+// Warp 0 of the block: G <- log2(e) * (chunk-local cumulative sum of g) in fp64 (G holds g on entry, 0 past the
+// chunk's end), F = 2^G, f = 2^(G_63 - G), gamma = 2^G_63.  A scan over the lanes, two rows a lane.
+__device__ __forceinline__ void bw_gate_scan(double* G, float* F, float* f, float* gam) {
+    const int l = threadIdx.x & 31;
+    const double a = G[2 * l], b = G[2 * l + 1];
+    double incl = a + b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (l >= o) incl += t;
+    }
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (l == 0) excl = 0.0;
+    const double g0 = (excl + a) * kLog2eD, g1 = incl * kLog2eD;
+    const double gl = __shfl_sync(0xffffffffu, incl, 31) * kLog2eD;
+    G[2 * l] = g0;
+    G[2 * l + 1] = g1;
+    F[2 * l] = exp2f((float)g0);
+    F[2 * l + 1] = exp2f((float)g1);
+    f[2 * l] = exp2f((float)(gl - g0));
+    f[2 * l + 1] = exp2f((float)(gl - g1));
+    if (l == 31) gam[0] = exp2f((float)gl);
+}
+
 // (2) One CTA per (sequence, head, 32 value columns): the state cotangent, walked from the last chunk to the first.
+// Per chunk: dU = scale P^T dO + diag(f) K dh', dX = T^T dU, dh = Q^T (scale F dO) + K^T (-beta F dX) + gamma dh',
+// each as register tiles (gdn_bwd_tiles.cuh).
 template <typename TIn, int DK>
 __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams p, unsigned* err) {
     using L = BwDhSmem<DK>;
-    constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBwThreads;
+    constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, IP = DK / 32;
+    static_assert(kBwThreads == kTileThreads, "the register tiles assume 256 threads");
     extern __shared__ __align__(16) float bsm[];
-    const BwChunk<DK> c{bsm + L::oK, bsm + L::oQ, nullptr, bsm + L::oT, bsm + L::oP, nullptr,
-                        reinterpret_cast<double*>(bsm + L::oG), bsm + L::oBeta, bsm + L::oF, bsm + L::of,
-                        bsm + L::oGam};
-    float* sKB = bsm + L::oKB;
+    float* sK = bsm + L::oK;
+    float* sQ = bsm + L::oQ;
+    float* sT = bsm + L::oT;
+    float* sP = bsm + L::oP;
+    double* sG = reinterpret_cast<double*>(bsm + L::oG);
+    float* sBeta = bsm + L::oBeta;
+    float* sF = bsm + L::oF;
+    float* sf = bsm + L::of;
+    float* sGam = bsm + L::oGam;
     float* sDh = bsm + L::oDh;
     float* sDo = bsm + L::oDo;
     float* sDu = bsm + L::oDu;
@@ -266,77 +297,96 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams 
     if (!bw_seq_bounds(p, n, row, bos, eos, err)) return;
     const long long start = (long long)row * p.T + bos;
     const size_t state_base = ((size_t)n * H + h) * DK * (size_t)dv + j0;
-    for (int e = tid; e < DK * DVT; e += NT) {
-        const int i = e / DVT, j = e % DVT;
-        sDh[i * LDV + j] = p.dhT ? p.dhT[state_base + (size_t)i * dv + j] : 0.f;
-    }
+    tile_load_state(sDh, p.dhT ? p.dhT + state_base : nullptr, dv, DK);
+    const TIn* q = static_cast<const TIn*>(p.q);
+    const TIn* k = static_cast<const TIn*>(p.k);
     const TIn* dout = static_cast<const TIn*>(p.dout);
+    const int s0 = tile_s0(), tj = tile_j0(), wr = tile_warp_row(), i0 = tile_i0<DK>();
     const int nc = (eos - bos + kChunk - 1) / kChunk;
-    for (int ci = nc - 1; ci >= 0; --ci) {
+    // the next chunk's operands, loaded into registers while the current one computes
+    RowBlock<TIn, DK> rk, rq;
+    RowBlock<float, kChunk> rt, rp;
+    RowBlock<TIn, DVT> rdo;
+    float rbeta = 0.f, rg = 0.f;
+    auto fetch = [&](int ci) {
         const int Lc = min(kChunk, eos - bos - ci * kChunk);
         const size_t tok0 = (size_t)(start + (long long)ci * kChunk);
-        const long long slot = wy_slot(n, start, ci);
-        bw_chunk_load<TIn, DK>(c, p, tok0, h, Lc, p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk, false);
-        for (int e = tid; e < kChunk * DK; e += NT) {  // the row factors of the dh update, once per chunk
-            const int r = e / DK, i = e % DK;
-            sKB[r * LDK + i] = -c.beta[r] * c.F[r] * c.K[r * LDK + i];
-            c.Q[r * LDK + i] *= p.scale * c.F[r];
+        const float* tp = p.tp + ((size_t)wy_slot(n, start, ci) * H + h) * 2 * kChunk * kChunk;
+        rk.load(k + (tok0 * H + h) * DK, (size_t)H * DK, Lc);
+        rq.load(q + (tok0 * H + h) * DK, (size_t)H * DK, Lc);
+        rt.load(tp, kChunk, kChunk);
+        rp.load(tp + kChunk * kChunk, kChunk, kChunk);
+        rdo.load(dout + (tok0 * H + h) * dv + j0, (size_t)H * dv, Lc);
+        if (tid < kChunk) {
+            const bool ok = tid < Lc;
+            rbeta = ok ? p.beta[(tok0 + tid) * H + h] : 0.f;
+            rg = ok ? p.g[(tok0 + tid) * H + h] : 0.f;
         }
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            sDo[r * LDV + j] = r < Lc ? to_f32(dout[((tok0 + r) * H + h) * dv + j0 + j]) : 0.f;
+    };
+    if (nc > 0) fetch(nc - 1);
+    for (int ci = nc - 1; ci >= 0; --ci) {
+        const long long slot = wy_slot(n, start, ci);
+        __syncthreads();  // the previous chunk is done with every buffer
+        rk.store(sK, LDK);
+        rq.store(sQ, LDK);
+        rt.store(sT, LDT);
+        rp.store(sP, LDT);
+        rdo.store(sDo, LDV);
+        if (tid < kChunk) {
+            sBeta[tid] = rbeta;
+            sG[tid] = (double)rg;
         }
         // dh' of this chunk (its end state's cotangent) for the gradient kernel
-        float* dh_out = p.dh_chunks + ((size_t)slot * H + h) * DK * (size_t)dv + j0;
-        for (int e = tid; e < DK * DVT; e += NT) {
-            const int i = e / DVT, j = e % DVT;
-            dh_out[(size_t)i * dv + j] = sDh[i * LDV + j];
-        }
+        tile_store_state(p.dh_chunks + ((size_t)slot * H + h) * DK * (size_t)dv + j0, dv, sDh, DK);
         __syncthreads();
-        // dU = scale P^T dO + diag(f) K dh'
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int s = e / DVT, j = e % DVT;
-            float acc = 0.f;
-            for (int r = s; r < kChunk; ++r) acc = fmaf(c.P[r * LDT + s], sDo[r * LDV + j], acc);
-            float kd = 0.f;
-            for (int i = 0; i < DK; ++i) kd = fmaf(c.K[s * LDK + i], sDh[i * LDV + j], kd);
-            sDu[s * LDV + j] = p.scale * acc + c.f[s] * kd;
-        }
+        if (ci > 0) fetch(ci - 1);
+        if (tid < 32) bw_gate_scan(sG, sF, sf, sGam);
         __syncthreads();
-        // dX = T^T dU
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int s = e / DVT, j = e % DVT;
-            float acc = 0.f;
-            for (int r = s; r < kChunk; ++r) acc = fmaf(c.T[r * LDT + s], sDu[r * LDV + j], acc);
-            sDx[s * LDV + j] = acc;
-        }
-        __syncthreads();
-        // dh = scale (diag(F) Q)^T dO + gamma dh' - K^T diag(beta F) dX
-        float nd[DK * DVT / NT];
-        const float gam = c.gamma[0];
+        {  // dU = scale P^T dO + diag(f) K dh'
+            float a[2][4] = {}, b[2][4] = {};
+            tile_acc_AtX<LDT>(sP, sDo, wr, a);
+            tile_acc_AD<LDK>(sK, sDh, DK, b);
 #pragma unroll
-        for (int m = 0; m < DK * DVT / NT; ++m) {
-            const int e = tid + m * NT, i = e / DVT, j = e % DVT;
-            float a = 0.f;
-            for (int r = 0; r < kChunk; ++r) {
-                a = fmaf(c.Q[r * LDK + i], sDo[r * LDV + j], a);  // scale F_r q_r, scaled above
-                a = fmaf(sKB[r * LDK + i], sDx[r * LDV + j], a);
+            for (int u = 0; u < 2; ++u) {
+                const float fs = sf[s0 + u];
+                sts4(sDu + (s0 + u) * LDV + tj, fmaf(p.scale, a[u][0], fs * b[u][0]),
+                     fmaf(p.scale, a[u][1], fs * b[u][1]), fmaf(p.scale, a[u][2], fs * b[u][2]),
+                     fmaf(p.scale, a[u][3], fs * b[u][3]));
             }
-            nd[m] = a + gam * sDh[i * LDV + j];
         }
         __syncthreads();
+        {  // dX = T^T dU, kept as -beta F dX; the thread's own tile of dO becomes scale F dO
+            float x[2][4] = {};
+            tile_acc_AtX<LDT>(sT, sDu, wr, x);
 #pragma unroll
-        for (int m = 0; m < DK * DVT / NT; ++m) {
-            const int e = tid + m * NT;
-            sDh[(e / DVT) * LDV + e % DVT] = nd[m];
+            for (int u = 0; u < 2; ++u) {
+                const int s = s0 + u;
+                const float xs = -sBeta[s] * sF[s], ds = p.scale * sF[s];
+                sts4(sDx + s * LDV + tj, xs * x[u][0], xs * x[u][1], xs * x[u][2], xs * x[u][3]);
+                const float4 d = lds4(sDo + s * LDV + tj);
+                sts4(sDo + s * LDV + tj, ds * d.x, ds * d.y, ds * d.z, ds * d.w);
+            }
+        }
+        __syncthreads();
+        {  // dh = Q^T (scale F dO) + K^T (-beta F dX) + gamma dh' on the thread's own rows and columns of dh
+            const float gam = sGam[0];
+            float a[IP][4];
+#pragma unroll
+            for (int u = 0; u < IP; ++u) {
+                const float4 d = lds4(sDh + (i0 + u) * LDV + tj);
+                a[u][0] = gam * d.x;
+                a[u][1] = gam * d.y;
+                a[u][2] = gam * d.z;
+                a[u][3] = gam * d.w;
+            }
+            tile_acc_KtX<DK, LDK>(sQ, sDo, a);
+            tile_acc_KtX<DK, LDK>(sK, sDx, a);
+#pragma unroll
+            for (int u = 0; u < IP; ++u) sts4(sDh + (i0 + u) * LDV + tj, a[u][0], a[u][1], a[u][2], a[u][3]);
         }
     }
     __syncthreads();
-    if (p.dh0)
-        for (int e = tid; e < DK * DVT; e += NT) {
-            const int i = e / DVT, j = e % DVT;
-            p.dh0[state_base + (size_t)i * dv + j] = sDh[i * LDV + j];
-        }
+    if (p.dh0) tile_store_state(p.dh0 + state_base, dv, sDh, DK);
 }
 
 // (2) One CTA per (chunk slot, head): T = (I + A)^-1 and P of the chunk (bw_chunk_prep) into the workspace, so
