@@ -557,16 +557,16 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_dh_kernel(const Bwd2Para
 
 template <int DK>
 struct Bw2ChunkSmem {  // 4-byte words
-    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 16, LDV = DVT + 1;
+    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 16, LDV = DVT + 4;  // value tiles: 16-byte rows
     // T and dT adjacent: after dA is formed they hold dGn [64][LDK]
     static constexpr int oT = 0, odT = oT + kChunk * LDT, oP = odT + kChunk * LDT, odP = oP + kChunk * LDT;
     static constexpr int odA = odP + kChunk * LDT;
     static constexpr int oLam = odA + kChunk * LDT, odLam = oLam + DK;
     static constexpr int odB = odLam + DK;  // KDA: dbeta per row
     static constexpr int oR = odB + kChunk;
-    // region R, gradient phase: EF, Kf [64][LDK]; h, dh' [DK][LDV]; V, W (write gate), dO, X, U, dU, dX [64][LDV]
+    // region R, gradient phase: EF, Kf [64][LDK]; h, dh' [DK][LDV]; dO, X, U, dU, dX [64][LDV]
     static constexpr int rEF = oR, rKf = rEF + kChunk * LDK, rH = rKf + kChunk * LDK, rDH = rH + DK * LDV;
-    static constexpr int rV = rDH + DK * LDV, rW = rV + kChunk * LDV, rDO = rW + kChunk * LDV;
+    static constexpr int rDO = rDH + DK * LDV;
     static constexpr int rX = rDO + kChunk * LDV, rU = rX + kChunk * LDV, rDU = rU + kChunk * LDV;
     static constexpr int rDX = rDU + kChunk * LDV, rEnd1 = rDX + kChunk * LDV;
     static constexpr int rM = rH;  // dT T^T scratch [64][LDT] once the tiles are done
@@ -577,6 +577,7 @@ struct Bw2ChunkSmem {  // 4-byte words
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
     static_assert(kChunk * LDK <= 2 * kChunk * LDT, "dGn fits over T and dT");
     static_assert(rM + kChunk * LDT <= rEnd1, "the dT T^T scratch fits over the tiles");
+    static_assert(rH % 4 == 0 && rDO % 4 == 0, "16-byte aligned value tiles");
 };
 
 // (4) One CTA per (chunk slot, head): every input gradient of the chunk.
@@ -584,8 +585,7 @@ template <typename TIn, int DK>
 __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bwd2Params p, unsigned* err) {
     using L = Bw2ChunkSmem<DK>;
     constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBw2Threads;
-    constexpr int ACC = DK / 4;            // key channels per thread in the register sums (row tid / 4)
-    constexpr int TPC = NT / DK;           // threads per channel in the Lambda sums
+    constexpr int CH = DK / 8;             // key channels per thread in the register sums
     extern __shared__ __align__(16) float bsm[];
     float* sT = bsm + L::oT;
     float* sdT = bsm + L::odT;
@@ -599,8 +599,6 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
     float* sKf = bsm + L::rKf;
     float* sH = bsm + L::rH;
     float* sDH = bsm + L::rDH;
-    float* sV = bsm + L::rV;
-    float* sW = bsm + L::rW;
     float* sDO = bsm + L::rDO;
     float* sX = bsm + L::rX;
     float* sU = bsm + L::rU;
@@ -630,126 +628,168 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
     if (tid < kChunk) sdB[tid] = 0.f;
     bw2_scaled_rows<TIn, DK>(p, tok0, h, Lc, nullptr, sEF, sKf, sLam, LDK);
 
-    const int ar = tid >> 2, ai = tid & 3;  // register sums: row ar, channels ai + 4 m
-    float aQ[ACC], aE[ACC], aK[ACC];        // (dO h^T), (dX h^T), (U dh'^T) of row ar
+    // Thread roles over a 64 x 16 value tile: row tr = tid / 4, columns tc .. tc + 3 (the row products); rows qr,
+    // qr + 32 and channels qc + 8 m (the key-side register sums, and later the gate phase); rows 4 (tid / 16) ..
+    // + 3 and columns tid % 16 + 16 v (the dT, dP blocks).
+    const int tr = tid >> 2, tc = 4 * (tid & 3);
+    const int qr = tid >> 3, qc = tid & 7;
+    const int pr = 4 * (tid >> 4), pc = tid & 15;
+    constexpr int HV = DK * DVT / 4 / NT;  // float4 of each state slice per thread (channels tid / 4 + 64 m)
+    static_assert(DK * DVT == 4 * NT * HV && kChunk * DVT == 4 * NT, "tile shapes");
+    float aQ[2][CH], aE[2][CH], aK[2][CH];  // (dO h^T), (dX h^T), (U dh'^T) of rows qr, qr + 32
 #pragma unroll
-    for (int m = 0; m < ACC; ++m) aQ[m] = aE[m] = aK[m] = 0.f;
-    const int lc = tid / TPC, lpart = tid % TPC;  // Lambda sums: channel lc, value columns lpart + TPC * x
-    float dlam = 0.f;
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int m = 0; m < CH; ++m) aQ[a][m] = aE[a][m] = aK[a][m] = 0.f;
+    float dlam[HV], rdb = 0.f;  // sum_j h dh' of this thread's channels; KDA: row tr's share of dbeta
+#pragma unroll
+    for (int m = 0; m < HV; ++m) dlam[m] = 0.f;
 
     for (int j0 = 0; j0 < dv; j0 += DVT) {
         __syncthreads();  // the previous tile is done (and, the first time, the scaled rows are in place)
-        for (int e = tid; e < DK * DVT; e += NT) {
-            const int i = e / DVT, j = e % DVT;
-            sH[i * LDV + j] = hc[(size_t)i * dv + j0 + j];
-            sDH[i * LDV + j] = dhc[(size_t)i * dv + j0 + j];
-        }
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            const bool ok = r < Lc;
-            const size_t tok = tok0 + r, idx = (tok * H + h) * dv + j0 + j;
-            sV[r * LDV + j] = ok ? to_f32(vin[idx]) : 0.f;
-            sW[r * LDV + j] = ok ? bw2_w(p, tok, h, j0 + j) : 0.f;
-            sDO[r * LDV + j] = ok ? to_f32(dout[idx]) : 0.f;
-        }
-        __syncthreads();
-        // X = w . V - (E . F) h ; (K . f) dh' (into dU for now).  Each thread forms a 2 x 2 block (rows ra, ra + 32;
-        // columns jb, jb + 8), so every shared-memory operand it loads feeds two products.
-        static_assert(kChunk * DVT == 4 * NT && DVT == 16, "2 x 2 blocks cover the tile");
-        {
-            const int ra = tid >> 3, jb = tid & 7;
-            float eh[2][2] = {}, kd[2][2] = {};
-#pragma unroll 4
-            for (int i = 0; i < DK; ++i) {
-                const float h0 = sH[i * LDV + jb], h1 = sH[i * LDV + jb + 8];
-                const float d0 = sDH[i * LDV + jb], d1 = sDH[i * LDV + jb + 8];
+        float4 vv, wv, dov;  // row tr, columns tc .. tc + 3 of V, the write gate and dO
+        {  // every load of the tile first, then the stores
+            float4 hv[HV], dhv[HV];
 #pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    const float ev = sEF[(ra + 32 * a) * LDK + i], kv = sKf[(ra + 32 * a) * LDK + i];
-                    eh[a][0] = fmaf(ev, h0, eh[a][0]);
-                    eh[a][1] = fmaf(ev, h1, eh[a][1]);
-                    kd[a][0] = fmaf(kv, d0, kd[a][0]);
-                    kd[a][1] = fmaf(kv, d1, kd[a][1]);
-                }
+            for (int m = 0; m < HV; ++m) {
+                const int e = tid + m * NT, i = e / (DVT / 4), cc = 4 * (e % (DVT / 4));
+                hv[m] = __ldg(reinterpret_cast<const float4*>(hc + (size_t)i * dv + j0 + cc));
+                dhv[m] = __ldg(reinterpret_cast<const float4*>(dhc + (size_t)i * dv + j0 + cc));
+            }
+            const bool ok = tr < Lc;
+            const size_t tok = tok0 + tr, idx = (tok * H + h) * dv + j0 + tc;
+            const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            vv = ok ? ldg4(vin + idx) : z4;
+            dov = ok ? ldg4(dout + idx) : z4;
+            if (p.kda) {
+                const float bt = ok ? p.b[tok * H + h] : 0.f;
+                wv = make_float4(bt, bt, bt, bt);
+            } else {
+                wv = ok ? ldg4(p.w + idx) : z4;
             }
 #pragma unroll
-            for (int a = 0; a < 2; ++a)
-#pragma unroll
-                for (int b = 0; b < 2; ++b) {
-                    const int r = ra + 32 * a, j = jb + 8 * b;
-                    sX[r * LDV + j] = sW[r * LDV + j] * sV[r * LDV + j] - eh[a][b];
-                    sDU[r * LDV + j] = kd[a][b];
-                }
+            for (int m = 0; m < HV; ++m) {
+                const int e = tid + m * NT, i = e / (DVT / 4), cc = 4 * (e % (DVT / 4));
+                *reinterpret_cast<float4*>(sH + i * LDV + cc) = hv[m];
+                *reinterpret_cast<float4*>(sDH + i * LDV + cc) = dhv[m];
+                dlam[m] = fmaf(hv[m].x, dhv[m].x, dlam[m]);
+                dlam[m] = fmaf(hv[m].y, dhv[m].y, dlam[m]);
+                dlam[m] = fmaf(hv[m].z, dhv[m].z, dlam[m]);
+                dlam[m] = fmaf(hv[m].w, dhv[m].w, dlam[m]);
+            }
+            *reinterpret_cast<float4*>(sDO + tr * LDV + tc) = dov;
         }
         __syncthreads();
+        // X = w . V - (E . F) h ; (K . f) dh' of row tr
+        float eh[4] = {}, kd[4] = {};
+#pragma unroll 4
+        for (int i = 0; i < DK; ++i) {
+            const float ev = sEF[tr * LDK + i], kv = sKf[tr * LDK + i];
+            fma4(eh, ev, lds4(sH + i * LDV + tc));
+            fma4(kd, kv, lds4(sDH + i * LDV + tc));
+        }
+        const float vr[4] = {vv.x, vv.y, vv.z, vv.w}, wr4[4] = {wv.x, wv.y, wv.z, wv.w};
+        sts4(sX + tr * LDV + tc, wr4[0] * vr[0] - eh[0], wr4[1] * vr[1] - eh[1], wr4[2] * vr[2] - eh[2],
+             wr4[3] * vr[3] - eh[3]);
+        __syncthreads();
         // U = T X ; dU = scale P^T dO + (K . f) dh'
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            float u = 0.f, du = 0.f;
-            for (int s = 0; s <= r; ++s) u = fmaf(sT[r * LDT + s], sX[s * LDV + j], u);
-            for (int t = r; t < kChunk; ++t) du = fmaf(sP[t * LDT + r], sDO[t * LDV + j], du);
-            sU[r * LDV + j] = u;
-            sDU[r * LDV + j] = fmaf(p.scale, du, sDU[r * LDV + j]);
+        {
+            float ur[4] = {}, du[4] = {};
+            for (int s2 = 0; s2 <= tr; ++s2) fma4(ur, sT[tr * LDT + s2], lds4(sX + s2 * LDV + tc));
+            for (int t = tr; t < kChunk; ++t) fma4(du, sP[t * LDT + tr], lds4(sDO + t * LDV + tc));
+            sts4(sU + tr * LDV + tc, ur[0], ur[1], ur[2], ur[3]);
+            sts4(sDU + tr * LDV + tc, fmaf(p.scale, du[0], kd[0]), fmaf(p.scale, du[1], kd[1]),
+                 fmaf(p.scale, du[2], kd[2]), fmaf(p.scale, du[3], kd[3]));
         }
         __syncthreads();
         // dX = T^T dU ; dv = w . dX ; dw = V . dX (KDA: summed into dbeta)
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int s = e / DVT, j = e % DVT;
-            float acc = 0.f;
-            for (int r = s; r < kChunk; ++r) acc = fmaf(sT[r * LDT + s], sDU[r * LDV + j], acc);
-            sDX[s * LDV + j] = acc;
-            if (s < Lc) {
-                const size_t idx = ((tok0 + s) * H + h) * dv + j0 + j;
-                p.dv[idx] = sW[s * LDV + j] * acc;
-                if (!p.kda) p.dw[idx] = sV[s * LDV + j] * acc;
+        {
+            float dx[4] = {};
+            for (int t = tr; t < kChunk; ++t) fma4(dx, sT[t * LDT + tr], lds4(sDU + t * LDV + tc));
+            sts4(sDX + tr * LDV + tc, dx[0], dx[1], dx[2], dx[3]);
+            if (tr < Lc) {
+                const size_t idx = ((tok0 + tr) * H + h) * dv + j0 + tc;
+                *reinterpret_cast<float4*>(p.dv + idx) =
+                    make_float4(wr4[0] * dx[0], wr4[1] * dx[1], wr4[2] * dx[2], wr4[3] * dx[3]);
+                if (!p.kda)
+                    *reinterpret_cast<float4*>(p.dw + idx) =
+                        make_float4(vr[0] * dx[0], vr[1] * dx[1], vr[2] * dx[2], vr[3] * dx[3]);
             }
+            if (p.kda)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) rdb = fmaf(vr[q], dx[q], rdb);
         }
         __syncthreads();
-        // dT += dU X^T, dP += scale dO U^T (lower parts)
-        for (int e = tid; e < kChunk * kChunk; e += NT) {
-            const int r = e / kChunk, s = e % kChunk;
-            if (s > r) continue;
-            float t = 0.f, pp = 0.f;
+        {  // dT += dU X^T, dP += scale dO U^T: 4 x 4 blocks, the lower parts kept
+            float bt[4][4] = {}, bp[4][4] = {};
 #pragma unroll
-            for (int j = 0; j < DVT; ++j) {
-                t = fmaf(sDU[r * LDV + j], sX[s * LDV + j], t);
-                pp = fmaf(sDO[r * LDV + j], sU[s * LDV + j], pp);
+            for (int jg = 0; jg < DVT; jg += 4) {
+                float4 xa[4], ua[4];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    xa[v] = lds4(sX + (pc + 16 * v) * LDV + jg);
+                    ua[v] = lds4(sU + (pc + 16 * v) * LDV + jg);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 dua = lds4(sDU + (pr + u) * LDV + jg), doa = lds4(sDO + (pr + u) * LDV + jg);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        bt[u][v] = fmaf(dua.x, xa[v].x, fmaf(dua.y, xa[v].y, fmaf(dua.z, xa[v].z,
+                                   fmaf(dua.w, xa[v].w, bt[u][v]))));
+                        bp[u][v] = fmaf(doa.x, ua[v].x, fmaf(doa.y, ua[v].y, fmaf(doa.z, ua[v].z,
+                                   fmaf(doa.w, ua[v].w, bp[u][v]))));
+                    }
+                }
             }
-            sdT[r * LDT + s] += t;
-            sdP[r * LDT + s] += p.scale * pp;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int r = pr + u, s2 = pc + 16 * v;
+                    if (s2 <= r) {
+                        sdT[r * LDT + s2] += bt[u][v];
+                        sdP[r * LDT + s2] += p.scale * bp[u][v];
+                    }
+                }
         }
-        if (p.kda && tid < kChunk) {  // the write gate's share of dbeta
-            float a = 0.f;
+        // register sums of rows qr, qr + 32: dO h^T, dX h^T, U dh'^T
 #pragma unroll
-            for (int j = 0; j < DVT; ++j) a = fmaf(sV[tid * LDV + j], sDX[tid * LDV + j], a);
-            sdB[tid] += a;
-        }
-        // sum_j h_ij dh'_ij
+        for (int jg = 0; jg < DVT; jg += 4) {
+            float4 o[2], x[2], u4[2];
 #pragma unroll
-        for (int x = 0; x < DVT / TPC; ++x) {
-            const int j = lpart + TPC * x;
-            dlam = fmaf(sH[lc * LDV + j], sDH[lc * LDV + j], dlam);
-        }
-        // register sums of row ar: dO h^T, dX h^T, U dh'^T
-#pragma unroll
-        for (int m = 0; m < ACC; ++m) {
-            const int i = ai + 4 * m;
-            float q1 = 0.f, e1 = 0.f, k1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < DVT; ++j) {
-                const float hv = sH[i * LDV + j];
-                q1 = fmaf(sDO[ar * LDV + j], hv, q1);
-                e1 = fmaf(sDX[ar * LDV + j], hv, e1);
-                k1 = fmaf(sU[ar * LDV + j], sDH[i * LDV + j], k1);
+            for (int a = 0; a < 2; ++a) {
+                const int r = qr + 32 * a;
+                o[a] = lds4(sDO + r * LDV + jg);
+                x[a] = lds4(sDX + r * LDV + jg);
+                u4[a] = lds4(sU + r * LDV + jg);
             }
-            aQ[m] += q1;
-            aE[m] += e1;
-            aK[m] += k1;
+#pragma unroll
+            for (int m = 0; m < CH; ++m) {
+                const int i = qc + 8 * m;
+                const float4 hv = lds4(sH + i * LDV + jg), dhv = lds4(sDH + i * LDV + jg);
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    aQ[a][m] = fmaf(o[a].x, hv.x, fmaf(o[a].y, hv.y, fmaf(o[a].z, hv.z, fmaf(o[a].w, hv.w,
+                               aQ[a][m]))));
+                    aE[a][m] = fmaf(x[a].x, hv.x, fmaf(x[a].y, hv.y, fmaf(x[a].z, hv.z, fmaf(x[a].w, hv.w,
+                               aE[a][m]))));
+                    aK[a][m] = fmaf(u4[a].x, dhv.x, fmaf(u4[a].y, dhv.y, fmaf(u4[a].z, dhv.z,
+                               fmaf(u4[a].w, dhv.w, aK[a][m]))));
+                }
+            }
         }
     }
+    // the sums over the four threads that share a channel (dLambda) or a row (KDA dbeta)
 #pragma unroll
-    for (int o = 1; o < TPC; o <<= 1) dlam += __shfl_xor_sync(0xffffffffu, dlam, o);
-    if (lpart == 0) sdLam[lc] = dlam;
+    for (int m = 0; m < HV; ++m) {
+        dlam[m] += __shfl_xor_sync(0xffffffffu, dlam[m], 1);
+        dlam[m] += __shfl_xor_sync(0xffffffffu, dlam[m], 2);
+        if ((tid & 3) == 0) sdLam[(tid + m * NT) / (DVT / 4)] = dlam[m];
+    }
+    rdb += __shfl_xor_sync(0xffffffffu, rdb, 1);
+    rdb += __shfl_xor_sync(0xffffffffu, rdb, 2);
+    if (p.kda && (tid & 3) == 0) sdB[tr] = rdb;
     __syncthreads();
     // dA = -T^T dT T^T on the strictly lower part (dT's diagonal and upper part do not reach A)
     float* sM = bsm + L::rM;
@@ -801,50 +841,63 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
     // G_L terms.
     float* sDG = sT;  // dGn [64][LDK] over T and dT (both done)
     float* sLr = sQ;  // the G_L terms of every row [64][LDK], once Q is no longer read
-    float dGn[ACC], lt[ACC];
-    float kdb = 0.f;  // KDA: this thread's share of sum_i k_ri dE_ri
+    float dGn[2][CH], lt[2][CH];
+    float kdb[2] = {0.f, 0.f};  // KDA: this thread's share of sum_i k_ri dE_ri of its two rows
 #pragma unroll
-    for (int m = 0; m < ACC; ++m) {
-        const int i = ai + 4 * m;
-        const float kv = sK[ar * LDK + i], qv = sQ[ar * LDK + i], ev = sE[ar * LDK + i];
-        float dEa = 0.f, dQp = 0.f, dKap = 0.f, F = sAd[ar * LDK + i], f = 1.f;
-        for (int s = ar - 1; s >= 0; --s) {
-            const float ks = sK[s * LDK + i] * F;
-            dEa = fmaf(sdA[ar * LDT + s], ks, dEa);
-            dQp = fmaf(sdP[ar * LDT + s], ks, dQp);
-            F *= sAd[s * LDK + i];
-        }
-        for (int r = ar + 1; r < kChunk; ++r) {
-            f *= sAd[r * LDK + i];
-            dKap = fmaf(fmaf(sdA[r * LDT + ar], sE[r * LDK + i], sdP[r * LDT + ar] * sQ[r * LDK + i]), f, dKap);
-        }
-        const float pd = sdP[ar * LDT + ar];
-        const float dQo = fmaf(p.scale * F, aQ[m], dQp);  // without P's diagonal
-        const float dE = fmaf(-F, aE[m], dEa);
-        const float kf = f * aK[m];
-        const bool last = ar == kChunk - 1;
-        const float dKo = (last ? 0.f : kf) + dKap;  // without P's diagonal (and, on row L, without its G_L share)
-        dGn[m] = (float)((double)qv * dQo + (double)ev * dE - (double)kv * dKo);
-        lt[m] = last ? 0.f : kv * kf;
-        if (ar < Lc) {
-            const size_t tok = tok0 + ar, idx = (tok * H + h) * DK + i;
-            const float bv = bw2_b(p, tok, h, i);
-            const float dK = kf + dKap + pd * qv;
-            p.dq[idx] = fmaf(pd, kv, dQo);
-            p.dk[idx] = fmaf(bv, dE, dK);
-            if (p.kda) kdb = fmaf(kv, dE, kdb);
-            else p.db[idx] = kv * dE;
+    for (int a = 0; a < 2; ++a) {
+        const int ar = qr + 32 * a;
+#pragma unroll
+        for (int m = 0; m < CH; ++m) {
+            const int i = qc + 8 * m;
+            const float kv = sK[ar * LDK + i], qv = sQ[ar * LDK + i], ev = sE[ar * LDK + i];
+            float dEa = 0.f, dQp = 0.f, dKap = 0.f, F = sAd[ar * LDK + i], f = 1.f;
+            for (int s = ar - 1; s >= 0; --s) {
+                const float ks = sK[s * LDK + i] * F;
+                dEa = fmaf(sdA[ar * LDT + s], ks, dEa);
+                dQp = fmaf(sdP[ar * LDT + s], ks, dQp);
+                F *= sAd[s * LDK + i];
+            }
+            for (int r = ar + 1; r < kChunk; ++r) {
+                f *= sAd[r * LDK + i];
+                dKap = fmaf(fmaf(sdA[r * LDT + ar], sE[r * LDK + i], sdP[r * LDT + ar] * sQ[r * LDK + i]), f, dKap);
+            }
+            const float pd = sdP[ar * LDT + ar];
+            const float dQo = fmaf(p.scale * F, aQ[a][m], dQp);  // without P's diagonal
+            const float dE = fmaf(-F, aE[a][m], dEa);
+            const float kf = f * aK[a][m];
+            const bool last = ar == kChunk - 1;
+            const float dKo = (last ? 0.f : kf) + dKap;  // without P's diagonal (and, on row L, without its G_L share)
+            dGn[a][m] = (float)((double)qv * dQo + (double)ev * dE - (double)kv * dKo);
+            lt[a][m] = last ? 0.f : kv * kf;
+            if (ar < Lc) {
+                const size_t tok = tok0 + ar, idx = (tok * H + h) * DK + i;
+                const float bv = bw2_b(p, tok, h, i);
+                const float dK = kf + dKap + pd * qv;
+                p.dq[idx] = fmaf(pd, kv, dQo);
+                p.dk[idx] = fmaf(bv, dE, dK);
+                if (p.kda) kdb[a] = fmaf(kv, dE, kdb[a]);
+                else p.db[idx] = kv * dE;
+            }
         }
     }
-    kdb += __shfl_xor_sync(0xffffffffu, kdb, 1);  // the four threads of row ar are adjacent lanes
-    kdb += __shfl_xor_sync(0xffffffffu, kdb, 2);
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {  // the eight threads of a row are adjacent lanes, in a fixed order
+        kdb[a] += __shfl_xor_sync(0xffffffffu, kdb[a], 1);
+        kdb[a] += __shfl_xor_sync(0xffffffffu, kdb[a], 2);
+        kdb[a] += __shfl_xor_sync(0xffffffffu, kdb[a], 4);
+    }
     __syncthreads();  // every thread is done reading T, dT and Q
 #pragma unroll
-    for (int m = 0; m < ACC; ++m) {
-        sDG[ar * LDK + ai + 4 * m] = dGn[m];
-        sLr[ar * LDK + ai + 4 * m] = lt[m];
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int m = 0; m < CH; ++m) {
+            sDG[(qr + 32 * a) * LDK + qc + 8 * m] = dGn[a][m];
+            sLr[(qr + 32 * a) * LDK + qc + 8 * m] = lt[a][m];
+        }
+    if (p.kda && qc == 0) {
+        sdB[qr] += kdb[0];
+        sdB[qr + 32] += kdb[1];
     }
-    if (p.kda && ai == 0) sdB[ar] += kdb;
     __syncthreads();
     // dg: reverse cumulative sum of dGn along the rows, with the terms of G_L on row 63
     for (int i = tid; i < DK; i += NT) {

@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_prep_kernel(const BwdParam
 
 template <int DK>
 struct BwChunkSmem {  // 4-byte words
-    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 16, LDV = DVT + 1;
+    static constexpr int LDK = DK + 1, LDT = kChunk + 1, DVT = 16, LDV = DVT + 4;  // value tiles: 16-byte rows
     static constexpr int oK = 0, oQ = oK + kChunk * LDK, oGm = oQ + kChunk * LDK, oT = oGm + kChunk * LDT;
     static constexpr int oP = oT + kChunk * LDT, oA = oP + kChunk * LDT;  // A, then dT
     static constexpr int odP = oA + kChunk * LDT;
@@ -437,11 +437,10 @@ struct BwChunkSmem {  // 4-byte words
     static constexpr int oBeta = oG + 2 * kChunk, oF = oBeta + kChunk, of = oF + kChunk, oGam = of + kChunk;
     static constexpr int odBeta = oGam + 4, odF = odBeta + kChunk, odf = odF + kChunk, odGn = odf + kChunk;
     static constexpr int odGam = odGn + kChunk;
-    static constexpr int oH = odGam + 4;          // h tile [DK][LDV]
-    static constexpr int oDH = oH + DK * LDV;     // dh' tile [DK][LDV]
-    static constexpr int oV = oDH + DK * LDV;     // [64][LDV] tiles: V, dO, Kh, Qh, Kdh, X, U, dU, dX
-    static constexpr int oDO = oV + kChunk * LDV, oKh = oDO + kChunk * LDV, oQh = oKh + kChunk * LDV;
-    static constexpr int oKd = oQh + kChunk * LDV, oX = oKd + kChunk * LDV, oU = oX + kChunk * LDV;
+    static constexpr int oH = (odGam + 4 + 3) / 4 * 4;  // h tile [DK][LDV] (16-byte aligned)
+    static constexpr int oDH = oH + DK * LDV;           // dh' tile [DK][LDV]
+    static constexpr int oDO = oDH + DK * LDV;          // [64][LDV] tiles: dO, X, U, dU, dX
+    static constexpr int oX = oDO + kChunk * LDV, oU = oX + kChunk * LDV;
     static constexpr int oDU = oU + kChunk * LDV, oDX = oDU + kChunk * LDV;
     static constexpr int total = oDX + kChunk * LDV;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
@@ -452,7 +451,6 @@ template <typename TIn, int DK>
 __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdParams p, unsigned* err) {
     using L = BwChunkSmem<DK>;
     constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBwThreads;
-    constexpr int ACC = DK / 4;  // key channels per thread in the register sums (row tid / 4)
     extern __shared__ __align__(16) float bsm[];
     const BwChunk<DK> c{bsm + L::oK, bsm + L::oQ, bsm + L::oGm, bsm + L::oT, bsm + L::oP, bsm + L::oA,
                         reinterpret_cast<double*>(bsm + L::oG), bsm + L::oBeta, bsm + L::oF, bsm + L::of,
@@ -466,11 +464,7 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
     float* sdGam = bsm + L::odGam;
     float* sH = bsm + L::oH;
     float* sDH = bsm + L::oDH;
-    float* sV = bsm + L::oV;
     float* sDO = bsm + L::oDO;
-    float* sKh = bsm + L::oKh;
-    float* sQh = bsm + L::oQh;
-    float* sKd = bsm + L::oKd;
     float* sX = bsm + L::oX;
     float* sU = bsm + L::oU;
     float* sDU = bsm + L::oDU;
@@ -494,124 +488,176 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
         sdT[e] = 0.f;
         sdP[e] = 0.f;
     }
-    if (tid < kChunk) sdBeta[tid] = sdF[tid] = sdf[tid] = 0.f;
     if (tid == 0) sdGam[0] = 0.f;
-    const int ar = tid >> 2, ai = tid & 3;  // register sums: row ar, channels ai + 4 m
-    float aQ[ACC], aK[ACC];
+    // Thread roles over a 64 x 16 value tile: row tr = tid / 4, columns tc .. tc + 3 (the row products and the
+    // per-row sums); rows qr, qr + 32 and channels qc + 8 m (the key-side register sums); rows 4 (tid / 16) ..
+    // + 3 and columns tid % 16 + 16 v (the dT, dP blocks).
+    const int tr = tid >> 2, tc = 4 * (tid & 3);
+    const int qr = tid >> 3, qc = tid & 7;
+    const int pr = 4 * (tid >> 4), pc = tid & 15;
+    constexpr int HV = DK * DVT / 4 / NT;  // float4 of each state slice per thread
+    static_assert(DK * DVT == 4 * NT * HV && kChunk * DVT == 4 * NT, "tile shapes");
+    float aQ[2][16], aK[2][16];            // dq, dk of rows qr, qr + 32, channels qc + 8 m (DK / 8 of them)
+    static_assert(DK / 8 <= 16, "register sums");
 #pragma unroll
-    for (int m = 0; m < ACC; ++m) aQ[m] = aK[m] = 0.f;
-    float dgam = 0.f;
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int m = 0; m < 16; ++m) aQ[a][m] = aK[a][m] = 0.f;
+    float dgam = 0.f, rdb = 0.f, rdF = 0.f, rdf = 0.f;  // <h, dh'>; row tr's partial dbeta, dF, df
 
     for (int j0 = 0; j0 < dv; j0 += DVT) {
         __syncthreads();  // the previous tile is done
-        for (int e = tid; e < DK * DVT; e += NT) {
-            const int i = e / DVT, j = e % DVT;
-            sH[i * LDV + j] = hc[(size_t)i * dv + j0 + j];
-            sDH[i * LDV + j] = dhc[(size_t)i * dv + j0 + j];
-        }
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            const bool ok = r < Lc;
-            const size_t idx = ((tok0 + r) * H + h) * dv + j0 + j;
-            sV[r * LDV + j] = ok ? to_f32(vin[idx]) : 0.f;
-            sDO[r * LDV + j] = ok ? to_f32(dout[idx]) : 0.f;
+        float4 vv, dov;   // row tr, columns tc .. tc + 3 of V and dO
+        {  // every load of the tile first, then the stores
+            float4 hv[HV], dhv[HV];
+#pragma unroll
+            for (int m = 0; m < HV; ++m) {
+                const int e = tid + m * NT, i = e / (DVT / 4), cc = 4 * (e % (DVT / 4));
+                hv[m] = __ldg(reinterpret_cast<const float4*>(hc + (size_t)i * dv + j0 + cc));
+                dhv[m] = __ldg(reinterpret_cast<const float4*>(dhc + (size_t)i * dv + j0 + cc));
+            }
+            const bool ok = tr < Lc;
+            const size_t idx = ((tok0 + tr) * H + h) * dv + j0 + tc;
+            vv = ok ? ldg4(vin + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+            dov = ok ? ldg4(dout + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int m = 0; m < HV; ++m) {
+                const int e = tid + m * NT, i = e / (DVT / 4), cc = 4 * (e % (DVT / 4));
+                *reinterpret_cast<float4*>(sH + i * LDV + cc) = hv[m];
+                *reinterpret_cast<float4*>(sDH + i * LDV + cc) = dhv[m];
+                dgam = fmaf(hv[m].x, dhv[m].x, dgam);
+                dgam = fmaf(hv[m].y, dhv[m].y, dgam);
+                dgam = fmaf(hv[m].z, dhv[m].z, dgam);
+                dgam = fmaf(hv[m].w, dhv[m].w, dgam);
+            }
+            *reinterpret_cast<float4*>(sDO + tr * LDV + tc) = dov;
         }
         __syncthreads();
-        // K h, Q h, K dh' ; X = beta V - beta F (K h)
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            float kh = 0.f, qh = 0.f, kd = 0.f;
-            for (int i = 0; i < DK; ++i) {
-                const float hv = sH[i * LDV + j], dh = sDH[i * LDV + j];
-                kh = fmaf(c.K[r * LDK + i], hv, kh);
-                qh = fmaf(c.Q[r * LDK + i], hv, qh);
-                kd = fmaf(c.K[r * LDK + i], dh, kd);
-            }
-            sKh[r * LDV + j] = kh;
-            sQh[r * LDV + j] = qh;
-            sKd[r * LDV + j] = kd;
-            sX[r * LDV + j] = c.beta[r] * (sV[r * LDV + j] - c.F[r] * kh);
+        // K h, Q h, K dh' of row tr ; X = beta V - beta F (K h)
+        float kh[4] = {}, qh[4] = {}, kd[4] = {};
+#pragma unroll 4
+        for (int i = 0; i < DK; ++i) {
+            const float kv = c.K[tr * LDK + i], qv = c.Q[tr * LDK + i];
+            const float4 hv = lds4(sH + i * LDV + tc), dhv = lds4(sDH + i * LDV + tc);
+            fma4(kh, kv, hv);
+            fma4(qh, qv, hv);
+            fma4(kd, kv, dhv);
         }
+        const float br = c.beta[tr], Fr = c.F[tr], fr = c.f[tr];
+        const float vr[4] = {vv.x, vv.y, vv.z, vv.w}, dor[4] = {dov.x, dov.y, dov.z, dov.w};
+        float xr[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xr[q] = br * (vr[q] - Fr * kh[q]);
+        sts4(sX + tr * LDV + tc, xr[0], xr[1], xr[2], xr[3]);
         __syncthreads();
         // U = T X ; dU = scale P^T dO + diag(f) K dh'
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int r = e / DVT, j = e % DVT;
-            float u = 0.f, du = 0.f;
-            for (int s = 0; s <= r; ++s) u = fmaf(c.T[r * LDT + s], sX[s * LDV + j], u);
-            for (int t = r; t < kChunk; ++t) du = fmaf(c.P[t * LDT + r], sDO[t * LDV + j], du);
-            sU[r * LDV + j] = u;
-            sDU[r * LDV + j] = p.scale * du + c.f[r] * sKd[r * LDV + j];
-        }
-        __syncthreads();
-        // dX = T^T dU ; dv = beta dX
-        for (int e = tid; e < kChunk * DVT; e += NT) {
-            const int s = e / DVT, j = e % DVT;
-            float acc = 0.f;
-            for (int r = s; r < kChunk; ++r) acc = fmaf(c.T[r * LDT + s], sDU[r * LDV + j], acc);
-            sDX[s * LDV + j] = acc;
-            if (s < Lc) p.dv[((tok0 + s) * H + h) * dv + j0 + j] = c.beta[s] * acc;
-        }
-        __syncthreads();
-        // dT += dU X^T, dP += scale dO U^T (lower parts)
-        for (int e = tid; e < kChunk * kChunk; e += NT) {
-            const int r = e / kChunk, s = e % kChunk;
-            if (s > r) continue;
-            float t = 0.f, pp = 0.f;
+        float ur[4] = {}, du[4] = {};
+        for (int s2 = 0; s2 <= tr; ++s2) fma4(ur, c.T[tr * LDT + s2], lds4(sX + s2 * LDV + tc));
+        for (int t = tr; t < kChunk; ++t) fma4(du, c.P[t * LDT + tr], lds4(sDO + t * LDV + tc));
 #pragma unroll
-            for (int j = 0; j < DVT; ++j) {
-                t = fmaf(sDU[r * LDV + j], sX[s * LDV + j], t);
-                pp = fmaf(sDO[r * LDV + j], sU[s * LDV + j], pp);
-            }
-            sdT[r * LDT + s] += t;
-            sdP[r * LDT + s] += p.scale * pp;
-        }
-        // per-row sums: dbeta, dF, df
-        if (tid < kChunk) {
-            const int r = tid;
-            float db = 0.f, dF = 0.f, df = 0.f;
-#pragma unroll
-            for (int j = 0; j < DVT; ++j) {
-                const float dx = sDX[r * LDV + j], kh = sKh[r * LDV + j];
-                db = fmaf(dx, sV[r * LDV + j] - c.F[r] * kh, db);
-                dF = fmaf(-c.beta[r] * dx, kh, dF);
-                dF = fmaf(p.scale * sDO[r * LDV + j], sQh[r * LDV + j], dF);
-                df = fmaf(sU[r * LDV + j], sKd[r * LDV + j], df);
-            }
-            sdBeta[r] += db;
-            sdF[r] += dF;
-            sdf[r] += df;
-        }
-        // dgamma: <h, dh'> over the tile
-        for (int e = tid; e < DK * DVT; e += NT) {
-            const int i = e / DVT, j = e % DVT;
-            dgam = fmaf(sH[i * LDV + j], sDH[i * LDV + j], dgam);
-        }
-        // register sums: dQ += scale F_r dO h^T ; dK += f_r U dh'^T - beta_r F_r dX h^T
+        for (int q = 0; q < 4; ++q) du[q] = p.scale * du[q] + fr * kd[q];
+        sts4(sU + tr * LDV + tc, ur[0], ur[1], ur[2], ur[3]);
+        sts4(sDU + tr * LDV + tc, du[0], du[1], du[2], du[3]);
+        __syncthreads();
+        // dX = T^T dU ; dv = beta dX ; the per-row sums of dbeta, dF, df
         {
-            const float sF = p.scale * c.F[ar], fr = c.f[ar], bF = -c.beta[ar] * c.F[ar];
+            float dx[4] = {};
+            for (int t = tr; t < kChunk; ++t) fma4(dx, c.T[t * LDT + tr], lds4(sDU + t * LDV + tc));
+            sts4(sDX + tr * LDV + tc, dx[0], dx[1], dx[2], dx[3]);
+            if (tr < Lc)
+                *reinterpret_cast<float4*>(p.dv + ((tok0 + tr) * H + h) * dv + j0 + tc) =
+                    make_float4(br * dx[0], br * dx[1], br * dx[2], br * dx[3]);
 #pragma unroll
-            for (int m = 0; m < ACC; ++m) {
-                const int i = ai + 4 * m;
-                float q1 = 0.f, k1 = 0.f, k2 = 0.f;
+            for (int q = 0; q < 4; ++q) {
+                rdb = fmaf(dx[q], vr[q] - Fr * kh[q], rdb);
+                rdF = fmaf(-br * dx[q], kh[q], rdF);
+                rdF = fmaf(p.scale * dor[q], qh[q], rdF);
+                rdf = fmaf(ur[q], kd[q], rdf);
+            }
+        }
+        __syncthreads();
+        {  // dT += dU X^T, dP += scale dO U^T: 4 x 4 blocks, the lower parts kept
+            float bt[4][4] = {}, bp[4][4] = {};
 #pragma unroll
-                for (int j = 0; j < DVT; ++j) {
-                    const float hv = sH[i * LDV + j];
-                    q1 = fmaf(sDO[ar * LDV + j], hv, q1);
-                    k1 = fmaf(sU[ar * LDV + j], sDH[i * LDV + j], k1);
-                    k2 = fmaf(sDX[ar * LDV + j], hv, k2);
+            for (int jg = 0; jg < DVT; jg += 4) {
+                float4 xa[4], ua[4];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    xa[v] = lds4(sX + (pc + 16 * v) * LDV + jg);
+                    ua[v] = lds4(sU + (pc + 16 * v) * LDV + jg);
                 }
-                aQ[m] = fmaf(sF, q1, aQ[m]);
-                aK[m] = fmaf(fr, k1, fmaf(bF, k2, aK[m]));
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 dua = lds4(sDU + (pr + u) * LDV + jg), doa = lds4(sDO + (pr + u) * LDV + jg);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        bt[u][v] = fmaf(dua.x, xa[v].x, fmaf(dua.y, xa[v].y, fmaf(dua.z, xa[v].z,
+                                   fmaf(dua.w, xa[v].w, bt[u][v]))));
+                        bp[u][v] = fmaf(doa.x, ua[v].x, fmaf(doa.y, ua[v].y, fmaf(doa.z, ua[v].z,
+                                   fmaf(doa.w, ua[v].w, bp[u][v]))));
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int r = pr + u, s2 = pc + 16 * v;
+                    if (s2 <= r) {
+                        sdT[r * LDT + s2] += bt[u][v];
+                        sdP[r * LDT + s2] += p.scale * bp[u][v];
+                    }
+                }
+        }
+        {  // register sums: dq += scale F_r dO h^T ; dk += f_r U dh'^T - beta_r F_r dX h^T
+#pragma unroll
+            for (int jg = 0; jg < DVT; jg += 4) {
+                float4 o[2], x[2], u4[2];
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    const int r = qr + 32 * a;
+                    const float so = p.scale * c.F[r], sx = -c.beta[r] * c.F[r], su = c.f[r];
+                    const float4 o0 = lds4(sDO + r * LDV + jg), x0 = lds4(sDX + r * LDV + jg);
+                    const float4 u0 = lds4(sU + r * LDV + jg);
+                    o[a] = make_float4(so * o0.x, so * o0.y, so * o0.z, so * o0.w);
+                    x[a] = make_float4(sx * x0.x, sx * x0.y, sx * x0.z, sx * x0.w);
+                    u4[a] = make_float4(su * u0.x, su * u0.y, su * u0.z, su * u0.w);
+                }
+#pragma unroll
+                for (int m = 0; m < DK / 8; ++m) {
+                    const int i = qc + 8 * m;
+                    const float4 hv = lds4(sH + i * LDV + jg), dhv = lds4(sDH + i * LDV + jg);
+#pragma unroll
+                    for (int a = 0; a < 2; ++a) {
+                        aQ[a][m] = fmaf(o[a].x, hv.x, fmaf(o[a].y, hv.y, fmaf(o[a].z, hv.z, fmaf(o[a].w, hv.w,
+                                   aQ[a][m]))));
+                        aK[a][m] = fmaf(u4[a].x, dhv.x, fmaf(u4[a].y, dhv.y, fmaf(u4[a].z, dhv.z,
+                                   fmaf(u4[a].w, dhv.w, aK[a][m]))));
+                        aK[a][m] = fmaf(x[a].x, hv.x, fmaf(x[a].y, hv.y, fmaf(x[a].z, hv.z, fmaf(x[a].w, hv.w,
+                                   aK[a][m]))));
+                    }
+                }
             }
         }
     }
-    // dgamma over the CTA
+    // the per-row sums over the four threads of a row; dgamma over the CTA
+    rdb += __shfl_xor_sync(0xffffffffu, rdb, 1);
+    rdb += __shfl_xor_sync(0xffffffffu, rdb, 2);
+    rdF += __shfl_xor_sync(0xffffffffu, rdF, 1);
+    rdF += __shfl_xor_sync(0xffffffffu, rdF, 2);
+    rdf += __shfl_xor_sync(0xffffffffu, rdf, 1);
+    rdf += __shfl_xor_sync(0xffffffffu, rdf, 2);
+    if ((tid & 3) == 0) {
+        sdBeta[tr] = rdb;
+        sdF[tr] = rdF;
+        sdf[tr] = rdf;
+    }
     for (int o = 16; o > 0; o >>= 1) dgam += __shfl_xor_sync(0xffffffffu, dgam, o);
     __syncthreads();
     if ((tid & 31) == 0) atomicAdd(sdGam, dgam);
     // dA = -T^T dT T^T on the strictly lower part (dT's diagonal and upper part do not reach A)
-    float* sM = sV;  // [64][LDT] scratch over the tile buffers (V, dO, Kh, Qh ... are no longer needed)
-    static_assert(kChunk * (kChunk + 1) <= 9 * kChunk * (16 + 1), "scratch fits the tile buffers");
+    float* sM = sDO;  // [64][LDT] scratch over the tile buffers (dO, X, U ... are no longer needed)
+    static_assert(kChunk * (kChunk + 1) <= 5 * kChunk * L::LDV, "scratch fits the tile buffers");
     __syncthreads();
     for (int e = tid; e < kChunk * kChunk; e += NT) {  // M = dT T^T, dT strictly lower
         const int r = e / kChunk, s = e % kChunk;
@@ -669,29 +715,37 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
         }
         sdGn[r] = d;
     }
-    // dQ += dQK K ; dK += dQK^T Q + dKK^T K + dKK K   (register sums of row ar)
+    // dQ += dQK K ; dK += dQK^T Q + dKK^T K + dKK K   (register sums of rows qr, qr + 32)
 #pragma unroll
-    for (int m = 0; m < ACC; ++m) {
-        const int i = ai + 4 * m;
-        float qa = 0.f, ka = 0.f;
-        for (int s = 0; s <= ar; ++s) {
-            qa = fmaf(sdP[ar * LDT + s], c.K[s * LDK + i], qa);
-            ka = fmaf(sdT[ar * LDT + s], c.K[s * LDK + i], ka);
+    for (int a = 0; a < 2; ++a) {
+        const int r = qr + 32 * a;
+        for (int s2 = 0; s2 <= r; ++s2) {
+            const float wq = sdP[r * LDT + s2], wk = sdT[r * LDT + s2];
+#pragma unroll
+            for (int m = 0; m < DK / 8; ++m) {
+                const float kv = c.K[s2 * LDK + qc + 8 * m];
+                aQ[a][m] = fmaf(wq, kv, aQ[a][m]);
+                aK[a][m] = fmaf(wk, kv, aK[a][m]);
+            }
         }
-        for (int r = ar; r < kChunk; ++r) {
-            ka = fmaf(sdP[r * LDT + ar], c.Q[r * LDK + i], ka);
-            ka = fmaf(sdT[r * LDT + ar], c.K[r * LDK + i], ka);
+        for (int t = r; t < kChunk; ++t) {
+            const float wq = sdP[t * LDT + r], wk = sdT[t * LDT + r];
+#pragma unroll
+            for (int m = 0; m < DK / 8; ++m)
+                aK[a][m] = fmaf(wq, c.Q[t * LDK + qc + 8 * m], fmaf(wk, c.K[t * LDK + qc + 8 * m], aK[a][m]));
         }
-        aQ[m] += qa;
-        aK[m] += ka;
     }
     __syncthreads();
-    if (ar < Lc) {
 #pragma unroll
-        for (int m = 0; m < ACC; ++m) {
-            const size_t idx = ((tok0 + ar) * H + h) * DK + ai + 4 * m;
-            p.dq[idx] = aQ[m];
-            p.dk[idx] = aK[m];
+    for (int a = 0; a < 2; ++a) {
+        const int r = qr + 32 * a;
+        if (r < Lc) {
+#pragma unroll
+            for (int m = 0; m < DK / 8; ++m) {
+                const size_t idx = ((tok0 + r) * H + h) * DK + qc + 8 * m;
+                p.dq[idx] = aQ[a][m];
+                p.dk[idx] = aK[a][m];
+            }
         }
     }
     if (tid < Lc) {
