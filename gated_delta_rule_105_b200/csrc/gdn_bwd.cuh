@@ -728,8 +728,10 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
                 aK[a][m] = fmaf(wk, kv, aK[a][m]);
             }
         }
-        for (int t = r; t < kChunk; ++t) {
-            const float wq = sdP[t * LDT + r], wk = sdT[t * LDT + r];
+        // from the warp's first row, so that the warp's four row groups read the same K and Q rows (the rows
+        // before r add zero)
+        for (int t = (tid >> 5) * 4 + 32 * a; t < kChunk; ++t) {
+            const float wq = t >= r ? sdP[t * LDT + r] : 0.f, wk = t >= r ? sdT[t * LDT + r] : 0.f;
 #pragma unroll
             for (int m = 0; m < DK / 8; ++m)
                 aK[a][m] = fmaf(wq, c.Q[t * LDK + qc + 8 * m], fmaf(wk, c.K[t * LDK + qc + 8 * m], aK[a][m]));
