@@ -16,6 +16,7 @@ head) units are independent, so there is no data-path collective); time is the m
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -606,12 +607,19 @@ def main(argv=None):
                          "(its extra bytes are reported as roofline.overhead_bytes, not as algorithmic work)")
     ap.add_argument("--path", default="chunk", choices=["chunk", "decode", "prelude", "output_gate", "bwd"],
                     help="chunk: the chunked forward (the headline); the others time that row's kernel alone")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="run the workload with this many sequences instead of its own B (a smaller case of the same "
+                         "shapes, e.g. for an ncu capture); not for packed-sequence workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds for the whole reference arm")
     args = ap.parse_args(argv)
     from gated_delta_rule_105_b200.inputs import WORKLOADS
     w = WORKLOADS[args.workload]
+    if args.batch:
+        if w.n_seqs or args.batch < 1:
+            ap.error("--batch needs a positive count and a workload of equal-length sequences")
+        w = dataclasses.replace(w, B=args.batch, name=f"{w.name}_batch{args.batch}")
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args, w)

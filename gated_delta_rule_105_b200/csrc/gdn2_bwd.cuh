@@ -202,64 +202,12 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_prep_kernel(const Bwd2Pa
     for (int e = tid; e < kChunk * kChunk; e += NT) Tg[e] = sT[(e / kChunk) * LDT + e % kChunk];
 }
 
-// Per-channel chunk quantities from the inputs: QF = Q . F, EF = E . F, Kf = K . f and Lambda (any pointer may be
-// null).  Two threads per channel, one per half of the rows (threads past 2 * DK idle).  The cumulative sum runs
-// along the rows in fp64 in the prep kernel's order (row 0 first, rows past the chunk's end adding nothing): the
-// first half's total is handed to the second half, whose total is G_L.  Called by every thread of the block (it synchronises twice).
-template <typename TIn, int DK>
-__device__ void bw2_scaled_rows(const Bwd2Params& p, size_t tok0, int h, int Lc, float* QF, float* EF, float* Kf,
-                                float* Lam, int ldk) {
-    constexpr int RH = kChunk / 2;
-    __shared__ double carry[2 * DK];
-    const TIn* q = static_cast<const TIn*>(p.q);
-    const TIn* k = static_cast<const TIn*>(p.k);
-    const int i = threadIdx.x % DK, half = threadIdx.x / DK, r0 = half * RH;
-    const bool act = half < 2;
-    const size_t H = p.H;
-    float gv[RH];
-#pragma unroll
-    for (int m = 0; m < RH; ++m) gv[m] = act && r0 + m < Lc ? p.g[((tok0 + r0 + m) * H + h) * DK + i] : 0.f;
-    double acc = 0.0;
-    if (half == 0) {
-#pragma unroll
-        for (int m = 0; m < RH; ++m) acc += (double)gv[m];
-        carry[i] = acc;
-    }
-    __syncthreads();
-    if (half == 1) {
-        acc = carry[i];
-#pragma unroll
-        for (int m = 0; m < RH; ++m) acc += (double)gv[m];
-        carry[DK + i] = acc;
-    }
-    __syncthreads();
-    if (!act) return;
-    const double gl = carry[DK + i] * kLog2eD;
-    if (Lam && half == 0) Lam[i] = exp2f((float)gl);
-    acc = half == 0 ? 0.0 : carry[i];
-#pragma unroll
-    for (int m = 0; m < RH; ++m) {
-        const int r = r0 + m;
-        float kv = 0.f, qv = 0.f, bv = 0.f;
-        if (r < Lc) {
-            const size_t tok = tok0 + r, idx = (tok * H + h) * DK + i;
-            kv = to_f32(k[idx]);
-            if (QF) qv = to_f32(q[idx]);
-            if (EF) bv = bw2_b(p, tok, h, i);
-        }
-        acc += (double)gv[m];
-        const double G = acc * kLog2eD;
-        const float F = exp2f((float)G), f = exp2f((float)(gl - G));
-        if (QF) QF[r * ldk + i] = qv * F;
-        if (EF) EF[r * ldk + i] = bv * kv * F;
-        if (Kf) Kf[r * ldk + i] = kv * f;
-    }
-}
-
-// The same quantities from raw rows already in shared memory ([64][ldk]: g in G, q in QF, the erase gate b in EF
+// Per-channel chunk quantities from raw rows in shared memory ([64][ldk]: g in G, q in QF, the erase gate b in EF
 // or, for KDA, beta per row in bt, k in Kf; rows past the chunk's end zero), in place: QF <- q F, EF <- b k F,
-// Kf <- k f, Lambda = 2^G_L.  Same threads, same fp64 sum order and same roundings as bw2_scaled_rows.  Called by
-// every thread of the block (it synchronises twice).
+// Kf <- k f, Lambda = 2^G_L (QF and Lam may be null).  Two threads per channel, one per half of the rows (threads
+// past 2 * DK idle).  The cumulative sum runs along the rows in fp64 in the prep kernel's order (row 0 first, rows
+// past the chunk's end adding nothing): the first half's total is handed to the second half, whose total is G_L.
+// Called by every thread of the block (it synchronises twice).
 template <int DK>
 __device__ void bw2_scale_rows_smem(const float* G, float* QF, float* EF, float* Kf, const float* bt, float* Lam,
                                     int ldk) {
@@ -585,7 +533,8 @@ template <typename TIn, int DK>
 __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bwd2Params p, unsigned* err) {
     using L = Bw2ChunkSmem<DK>;
     constexpr int LDK = L::LDK, LDT = L::LDT, DVT = L::DVT, LDV = L::LDV, NT = kBw2Threads;
-    constexpr int CH = DK / 8;             // key channels per thread in the register sums
+    constexpr int CM = DK / 32;            // key channels per thread in the register sums (8 rows each)
+    constexpr int QA = kChunk / (NT / 32); // rows per thread in the register sums
     extern __shared__ __align__(16) float bsm[];
     float* sT = bsm + L::oT;
     float* sdT = bsm + L::odT;
@@ -618,29 +567,60 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
     const float* dhc = p.dh_chunks + ((size_t)slot * H + h) * DK * (size_t)dv;
     const float* tp = p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk;
 
-    for (int e = tid; e < kChunk * kChunk; e += NT) {
-        const int r = e / kChunk, s = e % kChunk;
+#pragma unroll 8
+    for (int m = 0; m < kChunk * kChunk / NT; ++m) {
+        const int e = tid + m * NT, r = e / kChunk, s = e % kChunk;
         sT[r * LDT + s] = tp[e];
         sP[r * LDT + s] = tp[kChunk * kChunk + e];
         sdT[r * LDT + s] = 0.f;
         sdP[r * LDT + s] = 0.f;
     }
     if (tid < kChunk) sdB[tid] = 0.f;
-    bw2_scaled_rows<TIn, DK>(p, tok0, h, Lc, nullptr, sEF, sKf, sLam, LDK);
+    {  // the raw rows of g, the erase gate (KDA: beta per row) and k, then E . F, K . f and Lambda in place
+        float* sG = bsm + L::rH;  // the value tiles are free until the first tile
+        float* sBt = sG + kChunk * LDK;
+        static_assert(L::rH + kChunk * LDK + kChunk <= L::rEnd1, "raw gate rows fit over the value tiles");
+        const TIn* k = static_cast<const TIn*>(p.k);
+        constexpr int PER = kChunk * DK / NT, BATCH = 8;
+        for (int m0 = 0; m0 < PER; m0 += BATCH) {
+            float gv[BATCH], bv[BATCH], kv[BATCH];
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                const int e = tid + (m0 + u) * NT, r = e / DK, i = e % DK;
+                gv[u] = bv[u] = kv[u] = 0.f;
+                if (r < Lc) {
+                    const size_t idx = ((tok0 + r) * H + h) * DK + i;
+                    gv[u] = p.g[idx];
+                    if (!p.kda) bv[u] = p.b[idx];
+                    kv[u] = to_f32(k[idx]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                const int e = tid + (m0 + u) * NT, r = e / DK, i = e % DK;
+                sG[r * LDK + i] = gv[u];
+                sEF[r * LDK + i] = bv[u];
+                sKf[r * LDK + i] = kv[u];
+            }
+        }
+        if (p.kda && tid < kChunk) sBt[tid] = tid < Lc ? p.b[(tok0 + tid) * H + h] : 0.f;
+        __syncthreads();
+        bw2_scale_rows_smem<DK>(sG, nullptr, sEF, sKf, p.kda ? sBt : nullptr, sLam, LDK);
+    }
 
-    // Thread roles over a 64 x 16 value tile: row tr = tid / 4, columns tc .. tc + 3 (the row products); rows qr,
-    // qr + 32 and channels qc + 8 m (the key-side register sums, and later the gate phase); rows 4 (tid / 16) ..
-    // + 3 and columns tid % 16 + 16 v (the dT, dP blocks).
+    // Thread roles over a 64 x 16 value tile: row tr = tid / 4, columns tc .. tc + 3 (the row products); rows
+    // qw + 8 a and channels lane + 32 m (the key-side register sums, and later the gate phase: a warp's lanes
+    // share their rows); rows 4 (tid / 16) .. + 3 and columns tid % 16 + 16 v (the dT, dP blocks).
     const int tr = tid >> 2, tc = 4 * (tid & 3);
-    const int qr = tid >> 3, qc = tid & 7;
+    const int qw = tid >> 5, lane = tid & 31;
     const int pr = 4 * (tid >> 4), pc = tid & 15;
     constexpr int HV = DK * DVT / 4 / NT;  // float4 of each state slice per thread (channels tid / 4 + 64 m)
     static_assert(DK * DVT == 4 * NT * HV && kChunk * DVT == 4 * NT, "tile shapes");
-    float aQ[2][CH], aE[2][CH], aK[2][CH];  // (dO h^T), (dX h^T), (U dh'^T) of rows qr, qr + 32
+    float aQ[QA][CM], aE[QA][CM], aK[QA][CM];  // (dO h^T), (dX h^T), (U dh'^T) of rows qw + 8 a
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int a = 0; a < QA; ++a)
 #pragma unroll
-        for (int m = 0; m < CH; ++m) aQ[a][m] = aE[a][m] = aK[a][m] = 0.f;
+        for (int m = 0; m < CM; ++m) aQ[a][m] = aE[a][m] = aK[a][m] = 0.f;
     float dlam[HV], rdb = 0.f;  // sum_j h dh' of this thread's channels; KDA: row tr's share of dbeta
 #pragma unroll
     for (int m = 0; m < HV; ++m) dlam[m] = 0.f;
@@ -753,29 +733,25 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
                     }
                 }
         }
-        // register sums of rows qr, qr + 32: dO h^T, dX h^T, U dh'^T
+        // register sums of rows qw + 8 a: dO h^T, dX h^T, U dh'^T
 #pragma unroll
         for (int jg = 0; jg < DVT; jg += 4) {
-            float4 o[2], x[2], u4[2];
+            float4 hv[CM], dhv[CM];
 #pragma unroll
-            for (int a = 0; a < 2; ++a) {
-                const int r = qr + 32 * a;
-                o[a] = lds4(sDO + r * LDV + jg);
-                x[a] = lds4(sDX + r * LDV + jg);
-                u4[a] = lds4(sU + r * LDV + jg);
+            for (int m = 0; m < CM; ++m) {
+                hv[m] = lds4(sH + (lane + 32 * m) * LDV + jg);
+                dhv[m] = lds4(sDH + (lane + 32 * m) * LDV + jg);
             }
 #pragma unroll
-            for (int m = 0; m < CH; ++m) {
-                const int i = qc + 8 * m;
-                const float4 hv = lds4(sH + i * LDV + jg), dhv = lds4(sDH + i * LDV + jg);
+            for (int a = 0; a < QA; ++a) {
+                const int r = qw + 8 * a;
+                const float4 o = lds4(sDO + r * LDV + jg), x = lds4(sDX + r * LDV + jg), u4 = lds4(sU + r * LDV + jg);
 #pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    aQ[a][m] = fmaf(o[a].x, hv.x, fmaf(o[a].y, hv.y, fmaf(o[a].z, hv.z, fmaf(o[a].w, hv.w,
-                               aQ[a][m]))));
-                    aE[a][m] = fmaf(x[a].x, hv.x, fmaf(x[a].y, hv.y, fmaf(x[a].z, hv.z, fmaf(x[a].w, hv.w,
-                               aE[a][m]))));
-                    aK[a][m] = fmaf(u4[a].x, dhv.x, fmaf(u4[a].y, dhv.y, fmaf(u4[a].z, dhv.z,
-                               fmaf(u4[a].w, dhv.w, aK[a][m]))));
+                for (int m = 0; m < CM; ++m) {
+                    aQ[a][m] = fmaf(o.x, hv[m].x, fmaf(o.y, hv[m].y, fmaf(o.z, hv[m].z, fmaf(o.w, hv[m].w, aQ[a][m]))));
+                    aE[a][m] = fmaf(x.x, hv[m].x, fmaf(x.y, hv[m].y, fmaf(x.z, hv[m].z, fmaf(x.w, hv[m].w, aE[a][m]))));
+                    aK[a][m] = fmaf(u4.x, dhv[m].x, fmaf(u4.y, dhv[m].y, fmaf(u4.z, dhv[m].z,
+                               fmaf(u4.w, dhv[m].w, aK[a][m]))));
                 }
             }
         }
@@ -814,23 +790,32 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
     float* sQ = bsm + L::rQ;
     float* sE = bsm + L::rE;
     float* sAd = bsm + L::rA;
-    {
+    {  // eight elements of each tensor in flight per thread
         const TIn* q = static_cast<const TIn*>(p.q);
         const TIn* k = static_cast<const TIn*>(p.k);
-        for (int e = tid; e < kChunk * DK; e += NT) {
-            const int r = e / DK, i = e % DK;
-            float kv = 0.f, qv = 0.f, bv = 0.f, gv = 0.f;
-            if (r < Lc) {
-                const size_t idx = ((tok0 + r) * H + h) * DK + i;
-                kv = to_f32(k[idx]);
-                qv = to_f32(q[idx]);
-                bv = bw2_b(p, tok0 + r, h, i);
-                gv = p.g[idx];
+        constexpr int PER = kChunk * DK / NT, BATCH = 8;
+        for (int m0 = 0; m0 < PER; m0 += BATCH) {
+            float kv[BATCH], qv[BATCH], bv[BATCH], gv[BATCH];
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                const int e = tid + (m0 + u) * NT, r = e / DK, i = e % DK;
+                kv[u] = qv[u] = bv[u] = gv[u] = 0.f;
+                if (r < Lc) {
+                    const size_t idx = ((tok0 + r) * H + h) * DK + i;
+                    kv[u] = to_f32(k[idx]);
+                    qv[u] = to_f32(q[idx]);
+                    bv[u] = bw2_b(p, tok0 + r, h, i);
+                    gv[u] = p.g[idx];
+                }
             }
-            sK[r * LDK + i] = kv;
-            sQ[r * LDK + i] = qv;
-            sE[r * LDK + i] = bv * kv;
-            sAd[r * LDK + i] = expf(gv);
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                const int e = tid + (m0 + u) * NT, r = e / DK, i = e % DK;
+                sK[r * LDK + i] = kv[u];
+                sQ[r * LDK + i] = qv[u];
+                sE[r * LDK + i] = bv[u] * kv[u];
+                sAd[r * LDK + i] = expf(gv[u]);
+            }
         }
     }
     __syncthreads();
@@ -841,14 +826,15 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
     // G_L terms.
     float* sDG = sT;  // dGn [64][LDK] over T and dT (both done)
     float* sLr = sQ;  // the G_L terms of every row [64][LDK], once Q is no longer read
-    float dGn[2][CH], lt[2][CH];
-    float kdb[2] = {0.f, 0.f};  // KDA: this thread's share of sum_i k_ri dE_ri of its two rows
+    float lt[QA][CM];
+    float kdb[QA];  // KDA: this thread's share of sum_i k_ri dE_ri of its rows
 #pragma unroll
-    for (int a = 0; a < 2; ++a) {
-        const int ar = qr + 32 * a;
+    for (int a = 0; a < QA; ++a) {
+        const int ar = qw + 8 * a;
+        kdb[a] = 0.f;
 #pragma unroll
-        for (int m = 0; m < CH; ++m) {
-            const int i = qc + 8 * m;
+        for (int m = 0; m < CM; ++m) {
+            const int i = lane + 32 * m;
             const float kv = sK[ar * LDK + i], qv = sQ[ar * LDK + i], ev = sE[ar * LDK + i];
             float dEa = 0.f, dQp = 0.f, dKap = 0.f, F = sAd[ar * LDK + i], f = 1.f;
             for (int s = ar - 1; s >= 0; --s) {
@@ -867,7 +853,7 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
             const float kf = f * aK[a][m];
             const bool last = ar == kChunk - 1;
             const float dKo = (last ? 0.f : kf) + dKap;  // without P's diagonal (and, on row L, without its G_L share)
-            dGn[a][m] = (float)((double)qv * dQo + (double)ev * dE - (double)kv * dKo);
+            sDG[ar * LDK + i] = (float)((double)qv * dQo + (double)ev * dE - (double)kv * dKo);  // T, dT unread
             lt[a][m] = last ? 0.f : kv * kf;
             if (ar < Lc) {
                 const size_t tok = tok0 + ar, idx = (tok * H + h) * DK + i;
@@ -881,23 +867,17 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
         }
     }
 #pragma unroll
-    for (int a = 0; a < 2; ++a) {  // the eight threads of a row are adjacent lanes, in a fixed order
-        kdb[a] += __shfl_xor_sync(0xffffffffu, kdb[a], 1);
-        kdb[a] += __shfl_xor_sync(0xffffffffu, kdb[a], 2);
-        kdb[a] += __shfl_xor_sync(0xffffffffu, kdb[a], 4);
-    }
-    __syncthreads();  // every thread is done reading T, dT and Q
+    for (int a = 0; a < QA; ++a)  // a row's channels are the 32 lanes of one warp, summed in a fixed order
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+        for (int o = 1; o < 32; o <<= 1) kdb[a] += __shfl_xor_sync(0xffffffffu, kdb[a], o);
+    __syncthreads();  // every thread is done reading Q
 #pragma unroll
-        for (int m = 0; m < CH; ++m) {
-            sDG[(qr + 32 * a) * LDK + qc + 8 * m] = dGn[a][m];
-            sLr[(qr + 32 * a) * LDK + qc + 8 * m] = lt[a][m];
-        }
-    if (p.kda && qc == 0) {
-        sdB[qr] += kdb[0];
-        sdB[qr + 32] += kdb[1];
-    }
+    for (int a = 0; a < QA; ++a)
+#pragma unroll
+        for (int m = 0; m < CM; ++m) sLr[(qw + 8 * a) * LDK + lane + 32 * m] = lt[a][m];
+    if (p.kda && lane == 0)
+#pragma unroll
+        for (int a = 0; a < QA; ++a) sdB[qw + 8 * a] += kdb[a];
     __syncthreads();
     // dg: reverse cumulative sum of dGn along the rows, with the terms of G_L on row 63
     for (int i = tid; i < DK; i += NT) {
