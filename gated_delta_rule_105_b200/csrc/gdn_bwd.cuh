@@ -489,10 +489,11 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
         sdP[e] = 0.f;
     }
     if (tid == 0) sdGam[0] = 0.f;
-    // Thread roles over a 64 x 16 value tile: row tr = tid / 4, columns tc .. tc + 3 (the row products and the
-    // per-row sums); rows qr, qr + 32 and channels qc + 8 m (the key-side register sums); rows 4 (tid / 16) ..
-    // + 3 and columns tid % 16 + 16 v (the dT, dP blocks).
-    const int tr = tid >> 2, tc = 4 * (tid & 3);
+    // Thread roles over a 64 x 16 value tile: row tr, columns tc .. tc + 3 (the row products and the per-row sums;
+    // K h, Q h and K dh' run as 4 x 4 blocks, rows pb .. pb + 3, the sum over the key channels split over the
+    // block's four threads, channels kq + 4 t, each thread keeping row tr = pb + kq); rows qr, qr + 32 and channels
+    // qc + 8 m (the key-side register sums); rows 4 (tid / 16) .. + 3 and columns tid % 16 + 16 v (dT, dP blocks).
+    const int kq = tid & 3, tc = 4 * ((tid >> 2) & 3), pb = 4 * (tid >> 4), tr = pb + kq;
     const int qr = tid >> 3, qc = tid & 7;
     const int pr = 4 * (tid >> 4), pc = tid & 15;
     constexpr int HV = DK * DVT / 4 / NT;  // float4 of each state slice per thread
@@ -534,14 +535,37 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
         }
         __syncthreads();
         // K h, Q h, K dh' of row tr ; X = beta V - beta F (K h)
-        float kh[4] = {}, qh[4] = {}, kd[4] = {};
-#pragma unroll 4
-        for (int i = 0; i < DK; ++i) {
-            const float kv = c.K[tr * LDK + i], qv = c.Q[tr * LDK + i];
-            const float4 hv = lds4(sH + i * LDV + tc), dhv = lds4(sDH + i * LDV + tc);
-            fma4(kh, kv, hv);
-            fma4(qh, qv, hv);
-            fma4(kd, kv, dhv);
+        float kh[4], qh[4], kd[4];
+        {
+            float bk[4][4] = {}, bq[4][4] = {}, bd[4][4] = {};
+#pragma unroll 2
+            for (int t = 0; t < DK / 4; ++t) {
+                const int i = kq + 4 * t;
+                const float4 hv = lds4(sH + i * LDV + tc), dhv = lds4(sDH + i * LDV + tc);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float kv = c.K[(pb + u) * LDK + i], qv = c.Q[(pb + u) * LDK + i];
+                    fma4(bk[u], kv, hv);
+                    fma4(bq[u], qv, hv);
+                    fma4(bd[u], kv, dhv);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int o = 1; o <= 2; o <<= 1) {
+                        bk[u][q] += __shfl_xor_sync(0xffffffffu, bk[u][q], o);
+                        bq[u][q] += __shfl_xor_sync(0xffffffffu, bq[u][q], o);
+                        bd[u][q] += __shfl_xor_sync(0xffffffffu, bd[u][q], o);
+                    }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                kh[q] = kq == 0 ? bk[0][q] : kq == 1 ? bk[1][q] : kq == 2 ? bk[2][q] : bk[3][q];
+                qh[q] = kq == 0 ? bq[0][q] : kq == 1 ? bq[1][q] : kq == 2 ? bq[2][q] : bq[3][q];
+                kd[q] = kq == 0 ? bd[0][q] : kq == 1 ? bd[1][q] : kq == 2 ? bd[2][q] : bd[3][q];
+            }
         }
         const float br = c.beta[tr], Fr = c.F[tr], fr = c.f[tr];
         const float vr[4] = {vv.x, vv.y, vv.z, vv.w}, dor[4] = {dov.x, dov.y, dov.z, dov.w};
@@ -640,14 +664,14 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
             }
         }
     }
-    // the per-row sums over the four threads of a row; dgamma over the CTA
-    rdb += __shfl_xor_sync(0xffffffffu, rdb, 1);
-    rdb += __shfl_xor_sync(0xffffffffu, rdb, 2);
-    rdF += __shfl_xor_sync(0xffffffffu, rdF, 1);
-    rdF += __shfl_xor_sync(0xffffffffu, rdF, 2);
-    rdf += __shfl_xor_sync(0xffffffffu, rdf, 1);
-    rdf += __shfl_xor_sync(0xffffffffu, rdf, 2);
-    if ((tid & 3) == 0) {
+    // the per-row sums over the four threads of a row (lanes 4 and 8 apart); dgamma over the CTA
+    rdb += __shfl_xor_sync(0xffffffffu, rdb, 4);
+    rdb += __shfl_xor_sync(0xffffffffu, rdb, 8);
+    rdF += __shfl_xor_sync(0xffffffffu, rdF, 4);
+    rdF += __shfl_xor_sync(0xffffffffu, rdF, 8);
+    rdf += __shfl_xor_sync(0xffffffffu, rdf, 4);
+    rdf += __shfl_xor_sync(0xffffffffu, rdf, 8);
+    if (tc == 0) {
         sdBeta[tr] = rdb;
         sdF[tr] = rdF;
         sdf[tr] = rdf;
