@@ -608,10 +608,12 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
         bw2_scale_rows_smem<DK>(sG, nullptr, sEF, sKf, p.kda ? sBt : nullptr, sLam, LDK);
     }
 
-    // Thread roles over a 64 x 16 value tile: row tr = tid / 4, columns tc .. tc + 3 (the row products); rows
-    // qw + 8 a and channels lane + 32 m (the key-side register sums, and later the gate phase: a warp's lanes
-    // share their rows); rows 4 (tid / 16) .. + 3 and columns tid % 16 + 16 v (the dT, dP blocks).
-    const int tr = tid >> 2, tc = 4 * (tid & 3);
+    // Thread roles over a 64 x 16 value tile: row tr, columns tc .. tc + 3 (the row products; (E . F) h and
+    // (K . f) dh' run as 4 x 4 blocks, rows pb .. pb + 3, the sum over the key channels split over the block's four
+    // threads, channels kq + 4 t, each thread keeping row tr = pb + kq); rows qw + 8 a and channels lane + 32 m (the
+    // key-side register sums, and later the gate phase: a warp's lanes share their rows); rows 4 (tid / 16) .. + 3
+    // and columns tid % 16 + 16 v (the dT, dP blocks).
+    const int kq = tid & 3, tc = 4 * ((tid >> 2) & 3), pb = 4 * (tid >> 4), tr = pb + kq;
     const int qw = tid >> 5, lane = tid & 31;
     const int pr = 4 * (tid >> 4), pc = tid & 15;
     constexpr int HV = DK * DVT / 4 / NT;  // float4 of each state slice per thread (channels tid / 4 + 64 m)
@@ -661,12 +663,33 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
         }
         __syncthreads();
         // X = w . V - (E . F) h ; (K . f) dh' of row tr
-        float eh[4] = {}, kd[4] = {};
-#pragma unroll 4
-        for (int i = 0; i < DK; ++i) {
-            const float ev = sEF[tr * LDK + i], kv = sKf[tr * LDK + i];
-            fma4(eh, ev, lds4(sH + i * LDV + tc));
-            fma4(kd, kv, lds4(sDH + i * LDV + tc));
+        float eh[4], kd[4];
+        {
+            float be[4][4] = {}, bd[4][4] = {};
+#pragma unroll 2
+            for (int t = 0; t < DK / 4; ++t) {
+                const int i = kq + 4 * t;
+                const float4 hv = lds4(sH + i * LDV + tc), dhv = lds4(sDH + i * LDV + tc);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    fma4(be[u], sEF[(pb + u) * LDK + i], hv);
+                    fma4(bd[u], sKf[(pb + u) * LDK + i], dhv);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int o = 1; o <= 2; o <<= 1) {
+                        be[u][q] += __shfl_xor_sync(0xffffffffu, be[u][q], o);
+                        bd[u][q] += __shfl_xor_sync(0xffffffffu, bd[u][q], o);
+                    }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                eh[q] = kq == 0 ? be[0][q] : kq == 1 ? be[1][q] : kq == 2 ? be[2][q] : be[3][q];
+                kd[q] = kq == 0 ? bd[0][q] : kq == 1 ? bd[1][q] : kq == 2 ? bd[2][q] : bd[3][q];
+            }
         }
         const float vr[4] = {vv.x, vv.y, vv.z, vv.w}, wr4[4] = {wv.x, wv.y, wv.z, wv.w};
         sts4(sX + tr * LDV + tc, wr4[0] * vr[0] - eh[0], wr4[1] * vr[1] - eh[1], wr4[2] * vr[2] - eh[2],
@@ -756,16 +779,16 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
             }
         }
     }
-    // the sums over the four threads that share a channel (dLambda) or a row (KDA dbeta)
+    // the sums over the four threads that share a channel (dLambda, adjacent lanes) or a row (KDA dbeta)
 #pragma unroll
     for (int m = 0; m < HV; ++m) {
         dlam[m] += __shfl_xor_sync(0xffffffffu, dlam[m], 1);
         dlam[m] += __shfl_xor_sync(0xffffffffu, dlam[m], 2);
         if ((tid & 3) == 0) sdLam[(tid + m * NT) / (DVT / 4)] = dlam[m];
     }
-    rdb += __shfl_xor_sync(0xffffffffu, rdb, 1);
-    rdb += __shfl_xor_sync(0xffffffffu, rdb, 2);
-    if (p.kda && (tid & 3) == 0) sdB[tr] = rdb;
+    rdb += __shfl_xor_sync(0xffffffffu, rdb, 4);  // the four threads of row tr: lanes 4 and 8 apart
+    rdb += __shfl_xor_sync(0xffffffffu, rdb, 8);
+    if (p.kda && tc == 0) sdB[tr] = rdb;
     __syncthreads();
     // dA = -T^T dT T^T on the strictly lower part (dT's diagonal and upper part do not reach A)
     float* sM = bsm + L::rM;
