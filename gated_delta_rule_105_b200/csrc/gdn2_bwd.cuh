@@ -159,24 +159,56 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_prep_kernel(const Bwd2Pa
     const size_t tok0 = (size_t)info[0];
     const TIn* q = static_cast<const TIn*>(p.q);
     const TIn* k = static_cast<const TIn*>(p.k);
-    for (int e = tid; e < kChunk * DK; e += NT) {
-        const int r = e / DK, i = e % DK;
-        float kv = 0.f, qv = 0.f, bv = 0.f;
-        if (r < Lc) {
-            const size_t idx = ((tok0 + r) * H + h) * DK + i;
-            kv = to_f32(k[idx]);
-            qv = to_f32(q[idx]);
-            bv = bw2_b(p, tok0 + r, h, i);
+    {  // eight elements of each tensor in flight per thread
+        constexpr int PER = kChunk * DK / NT, BATCH = 8;
+        for (int m0 = 0; m0 < PER; m0 += BATCH) {
+            float kv[BATCH], qv[BATCH], bv[BATCH];
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                const int e = tid + (m0 + u) * NT, r = e / DK, i = e % DK;
+                kv[u] = qv[u] = bv[u] = 0.f;
+                if (r < Lc) {
+                    const size_t idx = ((tok0 + r) * H + h) * DK + i;
+                    kv[u] = to_f32(k[idx]);
+                    qv[u] = to_f32(q[idx]);
+                    bv[u] = bw2_b(p, tok0 + r, h, i);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                const int e = tid + (m0 + u) * NT, r = e / DK, i = e % DK;
+                sK[r * LDK + i] = kv[u];
+                sQ[r * LDK + i] = qv[u];
+                sE[r * LDK + i] = bv[u] * kv[u];
+            }
         }
-        sK[r * LDK + i] = kv;
-        sQ[r * LDK + i] = qv;
-        sE[r * LDK + i] = bv * kv;
     }
-    for (int i = tid; i < DK; i += NT) {
+    {  // G of every row and channel: the fp64 running sum from row 0 (rows past Lc add nothing), two threads per
+       // channel, the first half's total handed to the second half through shared memory
+        constexpr int RH = kChunk / 2;
+        __shared__ double carry[DK];
+        const int i = tid % DK, half = tid / DK, r0 = half * RH;
+        const bool act = half < 2;
+        float gv[RH];
+#pragma unroll
+        for (int m = 0; m < RH; ++m) gv[m] = act && r0 + m < Lc ? p.g[((tok0 + r0 + m) * H + h) * DK + i] : 0.f;
         double acc = 0.0;
-        for (int r = 0; r < kChunk; ++r) {
-            if (r < Lc) acc += (double)p.g[((tok0 + r) * H + h) * DK + i];
-            sGd[i * kChunk + r] = acc * kLog2eD;
+        if (half == 0) {
+#pragma unroll
+            for (int m = 0; m < RH; ++m) {
+                acc += (double)gv[m];
+                sGd[i * kChunk + m] = acc * kLog2eD;
+            }
+            carry[i] = acc;
+        }
+        __syncthreads();
+        if (half == 1) {
+            acc = carry[i];
+#pragma unroll
+            for (int m = 0; m < RH; ++m) {
+                acc += (double)gv[m];
+                sGd[i * kChunk + r0 + m] = acc * kLog2eD;
+            }
         }
     }
     __syncthreads();

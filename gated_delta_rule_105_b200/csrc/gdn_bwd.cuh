@@ -67,6 +67,34 @@ struct BwChunk {
     float* gamma;  // [1]
 };
 
+// K and Q rows of a chunk into shared memory ([64][ldk], rows past Lc zero), eight elements of each in flight per
+// thread.
+template <typename TIn, int DK>
+__device__ __forceinline__ void bw_load_kq(float* K, float* Q, int ldk, const TIn* k, const TIn* q, size_t tok0,
+                                           int H, int h, int Lc) {
+    constexpr int PER = kChunk * DK / kBwThreads, BATCH = 8;
+    static_assert(PER % BATCH == 0, "batches");
+    for (int m0 = 0; m0 < PER; m0 += BATCH) {
+        float kv[BATCH], qv[BATCH];
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int e = threadIdx.x + (m0 + u) * kBwThreads, r = e / DK, i = e % DK;
+            kv[u] = qv[u] = 0.f;
+            if (r < Lc) {
+                const size_t idx = ((tok0 + r) * H + h) * DK + i;
+                kv[u] = to_f32(k[idx]);
+                qv[u] = to_f32(q[idx]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int e = threadIdx.x + (m0 + u) * kBwThreads, r = e / DK, i = e % DK;
+            K[r * ldk + i] = kv[u];
+            Q[r * ldk + i] = qv[u];
+        }
+    }
+}
+
 // Loads one chunk (rows past Lc zero: k = q = beta = g = 0) and forms G, F, f, gamma, Gamma, P and T.
 template <typename TIn, int DK>
 __device__ void bw_chunk_prep(const BwChunk<DK>& c, const BwdParams& p, size_t tok0, int h, int Lc) {
@@ -75,17 +103,7 @@ __device__ void bw_chunk_prep(const BwChunk<DK>& c, const BwdParams& p, size_t t
     const TIn* q = static_cast<const TIn*>(p.q);
     const TIn* k = static_cast<const TIn*>(p.k);
     __syncthreads();  // the previous user of these buffers is done
-    for (int e = tid; e < kChunk * DK; e += NT) {
-        const int r = e / DK, i = e % DK;
-        float kv = 0.f, qv = 0.f;
-        if (r < Lc) {
-            const size_t idx = ((tok0 + r) * H + h) * DK + i;
-            kv = to_f32(k[idx]);
-            qv = to_f32(q[idx]);
-        }
-        c.K[r * LDK + i] = kv;
-        c.Q[r * LDK + i] = qv;
-    }
+    bw_load_kq<TIn, DK>(c.K, c.Q, LDK, k, q, tok0, H, h, Lc);
     if (tid < kChunk) {
         const bool ok = tid < Lc;
         c.beta[tid] = ok ? p.beta[(tok0 + tid) * H + h] : 0.f;
@@ -149,18 +167,10 @@ __device__ void bw_chunk_load(const BwChunk<DK>& c, const BwdParams& p, size_t t
     const TIn* q = static_cast<const TIn*>(p.q);
     const TIn* k = static_cast<const TIn*>(p.k);
     __syncthreads();  // the previous user of these buffers is done
-    for (int e = tid; e < kChunk * DK; e += NT) {
-        const int r = e / DK, i = e % DK;
-        float kv = 0.f, qv = 0.f;
-        if (r < Lc) {
-            const size_t idx = ((tok0 + r) * H + h) * DK + i;
-            kv = to_f32(k[idx]);
-            qv = to_f32(q[idx]);
-        }
-        c.K[r * LDK + i] = kv;
-        c.Q[r * LDK + i] = qv;
-    }
-    for (int e = tid; e < kChunk * kChunk; e += NT) {
+    bw_load_kq<TIn, DK>(c.K, c.Q, LDK, k, q, tok0, H, h, Lc);
+#pragma unroll 8
+    for (int m = 0; m < kChunk * kChunk / NT; ++m) {
+        const int e = tid + m * NT;
         c.T[(e / kChunk) * LDT + e % kChunk] = tp[e];
         c.P[(e / kChunk) * LDT + e % kChunk] = tp[kChunk * kChunk + e];
     }
