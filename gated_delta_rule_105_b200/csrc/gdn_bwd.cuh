@@ -710,29 +710,52 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
         sdA[r * LDT + s] = -a;
     }
     __syncthreads();
-    // through A and P to K, Q, beta and Gamma: dKK = dA beta_r Gamma, dQK = dP Gamma; W = dGamma . Gamma
+    // through A and P to K, Q, beta and Gamma: dKK = dA beta_r Gamma, dQK = dP Gamma; W = dGamma . Gamma.  K K^T
+    // and Q K^T are formed again as 4 x 4 blocks (rows pr .. pr + 3, columns pc + 16 v).
     float* sW = sM;
-    for (int e = tid; e < kChunk * kChunk; e += NT) {
-        const int r = e / kChunk, s = e % kChunk;
-        float dkk = 0.f, dqk = 0.f, w = 0.f;
-        if (s <= r) {
-            float kk = 0.f, qk = 0.f;
-            for (int i = 0; i < DK; ++i) {
-                const float ks = c.K[s * LDK + i];
-                kk = fmaf(c.K[r * LDK + i], ks, kk);
-                qk = fmaf(c.Q[r * LDK + i], ks, qk);
+    {
+        float kk[4][4] = {}, qk[4][4] = {};
+#pragma unroll 2
+        for (int i = 0; i < DK; ++i) {
+            float ks[4], kr[4], qv[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) ks[v] = c.K[(pc + 16 * v) * LDK + i];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                kr[u] = c.K[(pr + u) * LDK + i];
+                qv[u] = c.Q[(pr + u) * LDK + i];
             }
-            const float gm = c.Gm[r * LDT + s], da = sdA[r * LDT + s], dp = sdP[r * LDT + s];
-            if (s < r) {
-                dkk = da * c.beta[r] * gm;
-                atomicAdd(&sdBeta[r], da * gm * kk);
-            }
-            dqk = dp * gm;
-            w = (da * c.beta[r] * kk + dp * qk) * gm;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    kk[u][v] = fmaf(kr[u], ks[v], kk[u][v]);
+                    qk[u][v] = fmaf(qv[u], ks[v], qk[u][v]);
+                }
         }
-        sdT[r * LDT + s] = dkk;  // dT holds dKK from here on
-        sdP[r * LDT + s] = dqk;  // dP holds dQK
-        sW[r * LDT + s] = w;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = pr + u;
+            float dbs = 0.f;  // this thread's share of dbeta_r
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int s2 = pc + 16 * v;
+                float dkk = 0.f, dqk = 0.f, w = 0.f;
+                if (s2 <= r) {
+                    const float gm = c.Gm[r * LDT + s2], da = sdA[r * LDT + s2], dp = sdP[r * LDT + s2];
+                    if (s2 < r) {
+                        dkk = da * c.beta[r] * gm;
+                        dbs = fmaf(da * gm, kk[u][v], dbs);
+                    }
+                    dqk = dp * gm;
+                    w = (da * c.beta[r] * kk[u][v] + dp * qk[u][v]) * gm;
+                }
+                sdT[r * LDT + s2] = dkk;  // dT holds dKK from here on
+                sdP[r * LDT + s2] = dqk;  // dP holds dQK
+                sW[r * LDT + s2] = w;
+            }
+            atomicAdd(&sdBeta[r], dbs);
+        }
     }
     __syncthreads();
     // gradient of the natural-log cumulative gate Gn (Gamma_rs = exp(Gn_r - Gn_s), F = exp(Gn), f = exp(Gn_L - Gn),
