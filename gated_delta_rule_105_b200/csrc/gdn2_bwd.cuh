@@ -884,36 +884,60 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
     float lt[QA][CM];
     float kdb[QA];  // KDA: this thread's share of sum_i k_ri dE_ri of its rows
 #pragma unroll
-    for (int a = 0; a < QA; ++a) {
-        const int ar = qw + 8 * a;
-        kdb[a] = 0.f;
+    for (int a = 0; a < QA; ++a) kdb[a] = 0.f;
 #pragma unroll
-        for (int m = 0; m < CM; ++m) {
-            const int i = lane + 32 * m;
+    for (int m = 0; m < CM; ++m) {
+        const int i = lane + 32 * m;
+        // one sweep down and one up channel i's column for all the thread's rows ar = qw + 8 a, sharing the loads
+        // of K, E, Q and a; each row's running product multiplies in the same order as a walk from its own row
+        float Fa[QA], dEa[QA], dQp[QA], fa[QA], dKap[QA];
+#pragma unroll
+        for (int a = 0; a < QA; ++a) {
+            Fa[a] = fa[a] = 1.f;
+            dEa[a] = dQp[a] = dKap[a] = 0.f;
+        }
+        for (int s = kChunk - 2; s >= 0; --s) {  // Fa = a_(s+1) ... a_ar for the rows below s
+            const float an = sAd[(s + 1) * LDK + i], k0 = sK[s * LDK + i];
+#pragma unroll
+            for (int a = 0; a < QA; ++a) {
+                const int ar = qw + 8 * a;
+                if (s < ar) {
+                    Fa[a] *= an;
+                    const float ks = k0 * Fa[a];
+                    dEa[a] = fmaf(sdA[ar * LDT + s], ks, dEa[a]);
+                    dQp[a] = fmaf(sdP[ar * LDT + s], ks, dQp[a]);
+                }
+            }
+        }
+        for (int r = 1; r < kChunk; ++r) {  // fa = a_(ar+1) ... a_r for the rows above r
+            const float ad = sAd[r * LDK + i], er = sE[r * LDK + i], qr = sQ[r * LDK + i];
+#pragma unroll
+            for (int a = 0; a < QA; ++a) {
+                const int ar = qw + 8 * a;
+                if (r > ar) {
+                    fa[a] *= ad;
+                    dKap[a] = fmaf(fmaf(sdA[r * LDT + ar], er, sdP[r * LDT + ar] * qr), fa[a], dKap[a]);
+                }
+            }
+        }
+        const float a0 = sAd[i];  // a_0: F = a_ar ... a_1 a_0
+#pragma unroll
+        for (int a = 0; a < QA; ++a) {
+            const int ar = qw + 8 * a;
             const float kv = sK[ar * LDK + i], qv = sQ[ar * LDK + i], ev = sE[ar * LDK + i];
-            float dEa = 0.f, dQp = 0.f, dKap = 0.f, F = sAd[ar * LDK + i], f = 1.f;
-            for (int s = ar - 1; s >= 0; --s) {
-                const float ks = sK[s * LDK + i] * F;
-                dEa = fmaf(sdA[ar * LDT + s], ks, dEa);
-                dQp = fmaf(sdP[ar * LDT + s], ks, dQp);
-                F *= sAd[s * LDK + i];
-            }
-            for (int r = ar + 1; r < kChunk; ++r) {
-                f *= sAd[r * LDK + i];
-                dKap = fmaf(fmaf(sdA[r * LDT + ar], sE[r * LDK + i], sdP[r * LDT + ar] * sQ[r * LDK + i]), f, dKap);
-            }
+            const float F = Fa[a] * a0, f = fa[a];
             const float pd = sdP[ar * LDT + ar];
-            const float dQo = fmaf(p.scale * F, aQ[a][m], dQp);  // without P's diagonal
-            const float dE = fmaf(-F, aE[a][m], dEa);
+            const float dQo = fmaf(p.scale * F, aQ[a][m], dQp[a]);  // without P's diagonal
+            const float dE = fmaf(-F, aE[a][m], dEa[a]);
             const float kf = f * aK[a][m];
             const bool last = ar == kChunk - 1;
-            const float dKo = (last ? 0.f : kf) + dKap;  // without P's diagonal (and, on row L, without its G_L share)
+            const float dKo = (last ? 0.f : kf) + dKap[a];  // without P's diagonal (and, on row L, its G_L share)
             sDG[ar * LDK + i] = (float)((double)qv * dQo + (double)ev * dE - (double)kv * dKo);  // T, dT unread
             lt[a][m] = last ? 0.f : kv * kf;
             if (ar < Lc) {
                 const size_t tok = tok0 + ar, idx = (tok * H + h) * DK + i;
                 const float bv = bw2_b(p, tok, h, i);
-                const float dK = kf + dKap + pd * qv;
+                const float dK = kf + dKap[a] + pd * qv;
                 p.dq[idx] = fmaf(pd, kv, dQo);
                 p.dk[idx] = fmaf(bv, dE, dK);
                 if (p.kda) kdb[a] = fmaf(kv, dE, kdb[a]);
