@@ -729,9 +729,9 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
         __syncthreads();
         // U = T X ; dU = scale P^T dO + (K . f) dh'
         {
-            float ur[4] = {}, du[4] = {};
-            for (int s2 = 0; s2 <= tr; ++s2) fma4(ur, sT[tr * LDT + s2], lds4(sX + s2 * LDV + tc));
-            for (int t = tr; t < kChunk; ++t) fma4(du, sP[t * LDT + tr], lds4(sDO + t * LDV + tc));
+            float ur[4], du[4];
+            blk_tri_TX<LDT, LDV>(sT, sX, pb, kq, tc, ur);
+            blk_tri_TtX<LDT, LDV>(sP, sDO, pb, kq, tc, du);
             sts4(sU + tr * LDV + tc, ur[0], ur[1], ur[2], ur[3]);
             sts4(sDU + tr * LDV + tc, fmaf(p.scale, du[0], kd[0]), fmaf(p.scale, du[1], kd[1]),
                  fmaf(p.scale, du[2], kd[2]), fmaf(p.scale, du[3], kd[3]));
@@ -739,8 +739,8 @@ __global__ void __launch_bounds__(kBw2Threads, 1) gdn2_bwd_chunk_kernel(const Bw
         __syncthreads();
         // dX = T^T dU ; dv = w . dX ; dw = V . dX (KDA: summed into dbeta)
         {
-            float dx[4] = {};
-            for (int t = tr; t < kChunk; ++t) fma4(dx, sT[t * LDT + tr], lds4(sDU + t * LDV + tc));
+            float dx[4];
+            blk_tri_TtX<LDT, LDV>(sT, sDU, pb, kq, tc, dx);
             sts4(sDX + tr * LDV + tc, dx[0], dx[1], dx[2], dx[3]);
             if (tr < Lc) {
                 const size_t idx = ((tok0 + tr) * H + h) * dv + j0 + tc;

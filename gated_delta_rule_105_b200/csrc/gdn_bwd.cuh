@@ -585,9 +585,9 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
         sts4(sX + tr * LDV + tc, xr[0], xr[1], xr[2], xr[3]);
         __syncthreads();
         // U = T X ; dU = scale P^T dO + diag(f) K dh'
-        float ur[4] = {}, du[4] = {};
-        for (int s2 = 0; s2 <= tr; ++s2) fma4(ur, c.T[tr * LDT + s2], lds4(sX + s2 * LDV + tc));
-        for (int t = tr; t < kChunk; ++t) fma4(du, c.P[t * LDT + tr], lds4(sDO + t * LDV + tc));
+        float ur[4], du[4];
+        blk_tri_TX<LDT, LDV>(c.T, sX, pb, kq, tc, ur);
+        blk_tri_TtX<LDT, LDV>(c.P, sDO, pb, kq, tc, du);
 #pragma unroll
         for (int q = 0; q < 4; ++q) du[q] = p.scale * du[q] + fr * kd[q];
         sts4(sU + tr * LDV + tc, ur[0], ur[1], ur[2], ur[3]);
@@ -595,8 +595,8 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_chunk_kernel(const BwdPara
         __syncthreads();
         // dX = T^T dU ; dv = beta dX ; the per-row sums of dbeta, dF, df
         {
-            float dx[4] = {};
-            for (int t = tr; t < kChunk; ++t) fma4(dx, c.T[t * LDT + tr], lds4(sDU + t * LDV + tc));
+            float dx[4];
+            blk_tri_TtX<LDT, LDV>(c.T, sDU, pb, kq, tc, dx);
             sts4(sDX + tr * LDV + tc, dx[0], dx[1], dx[2], dx[3]);
             if (tr < Lc)
                 *reinterpret_cast<float4*>(p.dv + ((tok0 + tr) * H + h) * dv + j0 + tc) =

@@ -168,6 +168,47 @@ __device__ __forceinline__ void tile_load_values(float* s, const TIn* src, size_
 
 namespace gdn {
 
+// Split-sum 4 x 4 blocks of the gradient kernels' [64][16] value tiles (row stride LDV): a block covers rows
+// pb .. pb + 3 and columns tc .. tc + 3, its four adjacent lanes (kq = lane % 4) each sum a quarter of the
+// inner index, shuffles combine the quarters and every lane keeps row pb + kq of the block.  All 32 lanes of
+// the warp must call them together.
+__device__ __forceinline__ void blk_keep_row(float (&b)[4][4], int kq, float (&out)[4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            b[u][q] += __shfl_xor_sync(0xffffffffu, b[u][q], 1);
+            b[u][q] += __shfl_xor_sync(0xffffffffu, b[u][q], 2);
+        }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) out[q] = kq == 0 ? b[0][q] : kq == 1 ? b[1][q] : kq == 2 ? b[2][q] : b[3][q];
+}
+
+// out = sum_{s <= r} T[r][s] X[s][tc ..]  for r = pb + kq (T lower triangular, zero above its diagonal)
+template <int LDT, int LDV>
+__device__ __forceinline__ void blk_tri_TX(const float* T, const float* X, int pb, int kq, int tc, float (&out)[4]) {
+    float b[4][4] = {};
+    for (int s2 = kq; s2 < pb + 4; s2 += 4) {
+        const float4 x = lds4(X + s2 * LDV + tc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) fma4(b[u], T[(pb + u) * LDT + s2], x);
+    }
+    blk_keep_row(b, kq, out);
+}
+
+// out = sum_{t >= r} T[t][r] X[t][tc ..]  for r = pb + kq (T^T X; T zero above its diagonal)
+template <int LDT, int LDV>
+__device__ __forceinline__ void blk_tri_TtX(const float* T, const float* X, int pb, int kq, int tc,
+                                            float (&out)[4]) {
+    float b[4][4] = {};
+    for (int t = pb + kq; t < kChunk; t += 4) {
+        const float4 x = lds4(X + t * LDV + tc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) fma4(b[u], T[t * LDT + pb + u], x);
+    }
+    blk_keep_row(b, kq, out);
+}
+
 // A [64][W] block of rows of a bf16 or fp32 tensor (row r at src + r * row_stride elements), held as raw 16-byte
 // vectors in the loading thread's registers: loaded while the previous chunk computes, stored (as fp32) into
 // shared memory once its buffers are free.  Rows at or past Lc are zero.
