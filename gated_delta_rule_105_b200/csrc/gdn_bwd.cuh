@@ -95,9 +95,10 @@ __device__ __forceinline__ void bw_load_kq(float* K, float* Q, int ldk, const TI
     }
 }
 
-// Loads one chunk (rows past Lc zero: k = q = beta = g = 0) and forms G, F, f, gamma, Gamma, P and T.
+// Loads one chunk (rows past Lc zero: k = q = beta = g = 0), forms G, F, f, gamma and T = (I + A)^-1 in shared
+// memory (A in c.A while inverting; c.Gm and c.P unused) and writes P, row stride 64, to Pg.
 template <typename TIn, int DK>
-__device__ void bw_chunk_prep(const BwChunk<DK>& c, const BwdParams& p, size_t tok0, int h, int Lc) {
+__device__ void bw_chunk_prep(const BwChunk<DK>& c, const BwdParams& p, size_t tok0, int h, int Lc, float* Pg) {
     constexpr int LDK = BwChunk<DK>::LDK, LDT = BwChunk<DK>::LDT, NT = kBwThreads;
     const int tid = threadIdx.x, H = p.H;
     const TIn* q = static_cast<const TIn*>(p.q);
@@ -123,23 +124,42 @@ __device__ void bw_chunk_prep(const BwChunk<DK>& c, const BwdParams& p, size_t t
         c.f[tid] = exp2f((float)(c.G[kChunk - 1] - c.G[tid]));
         if (tid == 0) c.gamma[0] = exp2f((float)c.G[kChunk - 1]);
     }
-    for (int e = tid; e < kChunk * kChunk; e += NT) {
-        const int r = e / kChunk, s = e % kChunk;
-        float gm = 0.f, a = 0.f, pp = 0.f;
-        if (s <= r) {
-            float kk = 0.f, qk = 0.f;
-            for (int i = 0; i < DK; ++i) {
-                const float ks = c.K[s * LDK + i];
-                kk = fmaf(c.K[r * LDK + i], ks, kk);
-                qk = fmaf(c.Q[r * LDK + i], ks, qk);
+    {  // K K^T and Q K^T as 4 x 4 blocks: rows pr .. pr + 3, columns pc + 16 v
+        static_assert(NT == 256, "16 x 16 blocks of 4 x 4 entries");
+        const int pr = 4 * (tid >> 4), pc = tid & 15;
+        float kk[4][4] = {}, qk[4][4] = {};
+#pragma unroll 2
+        for (int i = 0; i < DK; ++i) {
+            float ks[4], kr[4], qv[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) ks[v] = c.K[(pc + 16 * v) * LDK + i];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                kr[u] = c.K[(pr + u) * LDK + i];
+                qv[u] = c.Q[(pr + u) * LDK + i];
             }
-            gm = exp2f((float)(c.G[r] - c.G[s]));
-            a = s < r ? c.beta[r] * gm * kk : 0.f;
-            pp = gm * qk;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    kk[u][v] = fmaf(kr[u], ks[v], kk[u][v]);
+                    qk[u][v] = fmaf(qv[u], ks[v], qk[u][v]);
+                }
         }
-        c.Gm[r * LDT + s] = gm;
-        c.A[r * LDT + s] = a;
-        c.P[r * LDT + s] = pp;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int r = pr + u, s = pc + 16 * v;
+                float gm = 0.f, a = 0.f, pp = 0.f;
+                if (s <= r) {
+                    gm = exp2f((float)(c.G[r] - c.G[s]));
+                    a = s < r ? c.beta[r] * gm * kk[u][v] : 0.f;
+                    pp = gm * qk[u][v];
+                }
+                c.A[r * LDT + s] = a;
+                Pg[r * kChunk + s] = pp;
+            }
     }
     __syncthreads();
     // T = (I + A)^-1 row by row, four threads per column (adjacent lanes) splitting each row's sum
@@ -403,10 +423,9 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams 
 // that the state-cotangent kernel (every value slice of every chunk) and the gradient kernel read them instead
 // of forming them again.
 template <int DK>
-struct BwPrepSmem {  // 4-byte words: the bw_chunk_prep operands
+struct BwPrepSmem {  // 4-byte words: the bw_chunk_prep operands (~100 KB for dk = 128: two CTAs per SM)
     static constexpr int LDK = DK + 1, LDT = kChunk + 1;
-    static constexpr int oK = 0, oQ = oK + kChunk * LDK, oGm = oQ + kChunk * LDK, oT = oGm + kChunk * LDT;
-    static constexpr int oP = oT + kChunk * LDT, oA = oP + kChunk * LDT;
+    static constexpr int oK = 0, oQ = oK + kChunk * LDK, oT = oQ + kChunk * LDK, oA = oT + kChunk * LDT;
     static constexpr int oG = oA + kChunk * LDT;  // double [64]
     static constexpr int oBeta = oG + 2 * kChunk, oF = oBeta + kChunk, of = oF + kChunk, oGam = of + kChunk;
     static constexpr int total = oGam + 4;
@@ -417,7 +436,7 @@ template <typename TIn, int DK>
 __global__ void __launch_bounds__(kBwThreads) gdn_bwd_prep_kernel(const BwdParams p, unsigned* err) {
     using L = BwPrepSmem<DK>;
     extern __shared__ __align__(16) float bsm[];
-    const BwChunk<DK> c{bsm + L::oK, bsm + L::oQ, bsm + L::oGm, bsm + L::oT, bsm + L::oP, bsm + L::oA,
+    const BwChunk<DK> c{bsm + L::oK, bsm + L::oQ, nullptr, bsm + L::oT, nullptr, bsm + L::oA,
                         reinterpret_cast<double*>(bsm + L::oG), bsm + L::oBeta, bsm + L::oF, bsm + L::of,
                         bsm + L::oGam};
     __shared__ int info[2];
@@ -428,13 +447,10 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_prep_kernel(const BwdParam
     __syncthreads();
     const int Lc = info[1];
     if (Lc == 0) return;
-    bw_chunk_prep<TIn, DK>(c, p, (size_t)info[0], h, Lc);
+    float* out = p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk;  // T, then P
+    bw_chunk_prep<TIn, DK>(c, p, (size_t)info[0], h, Lc, out + kChunk * kChunk);
     __syncthreads();
-    float* out = p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk;
-    for (int e = tid; e < kChunk * kChunk; e += kBwThreads) {
-        out[e] = c.T[(e / kChunk) * L::LDT + e % kChunk];
-        out[kChunk * kChunk + e] = c.P[(e / kChunk) * L::LDT + e % kChunk];
-    }
+    for (int e = tid; e < kChunk * kChunk; e += kBwThreads) out[e] = c.T[(e / kChunk) * L::LDT + e % kChunk];
 }
 
 template <int DK>
