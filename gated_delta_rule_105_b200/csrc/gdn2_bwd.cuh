@@ -134,7 +134,8 @@ struct Bw2PrepSmem {  // 4-byte words; the cumulative gate is fp64, transposed [
     static constexpr int oGd = 0;  // double [DK][64]
     static constexpr int oK = oGd + 2 * DK * kChunk, oQ = oK + kChunk * LDK, oE = oQ + kChunk * LDK;
     static constexpr int oA = oE + kChunk * LDK, oT = oA + kChunk * LDT;
-    static constexpr int total = oT + kChunk * LDT;
+    static constexpr int oAd = oT + kChunk * LDT;  // per-token decays of 64 channels [row][channel], LDT apart
+    static constexpr int total = oAd + kChunk * LDT;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
 
@@ -212,21 +213,48 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_prep_kernel(const Bwd2Pa
         }
     }
     __syncthreads();
-    // A and P: thread column s = tid % 64, rows r = tid / 64 + 4 m.  The decay 2^(G_r - G_s) comes from the fp64
-    // difference: an fp32 G of a strongly decaying channel (hundreds in magnitude) would cost ~1e-5 of it.
+    // A and P: thread column s = tid % 64, rows 16 rb .. 16 rb + 15 (rb = tid / 64).  Per channel the decay
+    // 2^(G_r - G_s) starts at the block's first row r0 at or below s (1 when r0 = s, else exp2 of the fp64
+    // difference: an fp32 G of a strongly decaying channel, hundreds in magnitude, would cost ~1e-5 of it) and is
+    // carried down the block by the per-token decays a_r = 2^(G_r - G_(r-1)), shared by the warp through shared
+    // memory, 64 channels at a time (at most 15 roundings more than one exp2 per entry: ~1e-6).
     float* P = p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk + kChunk * kChunk;
-    const int s = tid & (kChunk - 1);
-    for (int r = tid >> 6; r < kChunk; r += NT / kChunk) {
-        float a = 0.f, pp = 0.f;
-        if (s <= r) {
-            for (int i = 0; i < DK; ++i) {
-                const float d = exp2f((float)(sGd[i * kChunk + r] - sGd[i * kChunk + s])), ks = sK[s * LDK + i] * d;
-                a = fmaf(sE[r * LDK + i], ks, a);
-                pp = fmaf(sQ[r * LDK + i], ks, pp);
-            }
+    float* sAd = bsm + L::oAd;
+    const int s = tid & (kChunk - 1), rb = tid >> 6, r0 = max(16 * rb, s);
+    const bool act = r0 < 16 * rb + 16;
+    float accA[16], accP[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) accA[u] = accP[u] = 0.f;
+    for (int i0 = 0; i0 < DK; i0 += 64) {
+        __syncthreads();  // the previous channels' decays are no longer read
+        for (int e = tid; e < 64 * kChunk; e += NT) {
+            const int ii = e / kChunk, r = e % kChunk;
+            const double* gd = sGd + (i0 + ii) * kChunk;
+            sAd[r * LDT + ii] = r == 0 ? 1.f : exp2f((float)(gd[r] - gd[r - 1]));
         }
-        sA[r * LDT + s] = s < r ? a : 0.f;
-        P[r * kChunk + s] = pp;
+        __syncthreads();
+        if (act)
+            for (int ii = 0; ii < 64; ++ii) {
+                const int i = i0 + ii;
+                const float ks = sK[s * LDK + i];
+                float D = r0 == s ? 1.f : exp2f((float)(sGd[i * kChunk + r0] - sGd[i * kChunk + s]));
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int r = 16 * rb + u;
+                    if (r > r0) D *= sAd[r * LDT + ii];
+                    if (r >= r0) {
+                        const float kd = ks * D;
+                        accA[u] = fmaf(sE[r * LDK + i], kd, accA[u]);
+                        accP[u] = fmaf(sQ[r * LDK + i], kd, accP[u]);
+                    }
+                }
+            }
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const int r = 16 * rb + u;
+        sA[r * LDT + s] = s < r ? accA[u] : 0.f;
+        P[r * kChunk + s] = accP[u];
     }
     __syncthreads();
     bw2_invert_lower(sA, sT, LDT);
