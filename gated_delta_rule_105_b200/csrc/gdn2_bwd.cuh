@@ -160,44 +160,39 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_prep_kernel(const Bwd2Pa
     const size_t tok0 = (size_t)info[0];
     const TIn* q = static_cast<const TIn*>(p.q);
     const TIn* k = static_cast<const TIn*>(p.k);
-    {  // eight elements of each tensor in flight per thread
-        constexpr int PER = kChunk * DK / NT, BATCH = 8;
-        for (int m0 = 0; m0 < PER; m0 += BATCH) {
-            float kv[BATCH], qv[BATCH], bv[BATCH];
-#pragma unroll
-            for (int u = 0; u < BATCH; ++u) {
-                const int e = tid + (m0 + u) * NT, r = e / DK, i = e % DK;
-                kv[u] = qv[u] = bv[u] = 0.f;
-                if (r < Lc) {
-                    const size_t idx = ((tok0 + r) * H + h) * DK + i;
-                    kv[u] = to_f32(k[idx]);
-                    qv[u] = to_f32(q[idx]);
-                    bv[u] = bw2_b(p, tok0 + r, h, i);
-                }
+    // Every load of the chunk in one round trip, as 16-byte vectors: k, q into their buffers, the erase gate into
+    // E (multiplied by k below), the raw gate rows into A, T and the decay buffer (free until the A and P sweep).
+    float* sGr = sA;
+    static_assert(L::oA + kChunk * LDK <= L::total, "the raw gate rows fit over A, T and the decays");
+    {
+        RowBlock<TIn, DK> rk, rq;
+        RowBlock<float, DK> rg, rb;
+        const size_t base = (tok0 * H + h) * DK, rs = (size_t)H * DK;
+        rk.load(k + base, rs, Lc);
+        rq.load(q + base, rs, Lc);
+        rg.load(p.g + base, rs, Lc);
+        if (!p.kda) rb.load(p.b + base, rs, Lc);
+        rk.store_scalar(sK, LDK);
+        rq.store_scalar(sQ, LDK);
+        rg.store_scalar(sGr, LDK);
+        if (!p.kda) rb.store_scalar(sE, LDK);
+        else
+            for (int e = tid; e < kChunk * DK; e += NT) {  // KDA: beta of the row
+                const int r = e / DK;
+                sE[r * LDK + e % DK] = r < Lc ? p.b[(tok0 + r) * H + h] : 0.f;
             }
-#pragma unroll
-            for (int u = 0; u < BATCH; ++u) {
-                const int e = tid + (m0 + u) * NT, r = e / DK, i = e % DK;
-                sK[r * LDK + i] = kv[u];
-                sQ[r * LDK + i] = qv[u];
-                sE[r * LDK + i] = bv[u] * kv[u];
-            }
-        }
     }
+    __syncthreads();
     {  // G of every row and channel: the fp64 running sum from row 0 (rows past Lc add nothing), two threads per
-       // channel, the first half's total handed to the second half through shared memory
+       // channel, the first half's total handed to the second half through shared memory; E = b . k on the way
         constexpr int RH = kChunk / 2;
         __shared__ double carry[DK];
         const int i = tid % DK, half = tid / DK, r0 = half * RH;
-        const bool act = half < 2;
-        float gv[RH];
-#pragma unroll
-        for (int m = 0; m < RH; ++m) gv[m] = act && r0 + m < Lc ? p.g[((tok0 + r0 + m) * H + h) * DK + i] : 0.f;
         double acc = 0.0;
         if (half == 0) {
-#pragma unroll
+#pragma unroll 8
             for (int m = 0; m < RH; ++m) {
-                acc += (double)gv[m];
+                acc += (double)sGr[m * LDK + i];
                 sGd[i * kChunk + m] = acc * kLog2eD;
             }
             carry[i] = acc;
@@ -205,12 +200,14 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_prep_kernel(const Bwd2Pa
         __syncthreads();
         if (half == 1) {
             acc = carry[i];
-#pragma unroll
+#pragma unroll 8
             for (int m = 0; m < RH; ++m) {
-                acc += (double)gv[m];
+                acc += (double)sGr[(r0 + m) * LDK + i];
                 sGd[i * kChunk + r0 + m] = acc * kLog2eD;
             }
         }
+        if (half < 2)
+            for (int m = 0; m < RH; ++m) sE[(r0 + m) * LDK + i] *= sK[(r0 + m) * LDK + i];
     }
     __syncthreads();
     // A and P: thread column s = tid % 64, rows 16 rb .. 16 rb + 15 (rb = tid / 64).  Per channel the decay

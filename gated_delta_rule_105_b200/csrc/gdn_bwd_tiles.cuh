@@ -227,6 +227,24 @@ struct RowBlock {
                           : make_uint4(0u, 0u, 0u, 0u);
         }
     }
+    // One element at a time, for a row stride that is not a multiple of 4 (v[m] holds EPV consecutive elements).
+    __device__ __forceinline__ void store_scalar(float* dst, int ld) const {
+#pragma unroll
+        for (int m = 0; m < N; ++m) {
+            const int e = threadIdx.x + m * kTileThreads, r = e / VPR, c = e % VPR;
+            float* d = dst + r * ld + c * EPV;
+            const unsigned w[4] = {v[m].x, v[m].y, v[m].z, v[m].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if constexpr (sizeof(TIn) == 2) {
+                    d[2 * q] = __uint_as_float(w[q] << 16);
+                    d[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+                } else {
+                    d[q] = __uint_as_float(w[q]);
+                }
+            }
+        }
+    }
     __device__ __forceinline__ void store(float* dst, int ld) const {
 #pragma unroll
         for (int m = 0; m < N; ++m) {
