@@ -113,20 +113,6 @@ __device__ __forceinline__ float bw2_w(const Bwd2Params& p, size_t tok, int h, i
     return p.kda ? p.b[tok * p.H + h] : p.w[(tok * p.H + h) * p.vdim + j];
 }
 
-// T = (I + A)^-1 of a strictly lower A (row-major, leading dimension ldt), row by row, four adjacent threads per
-// column splitting each row's sum.  Needs 4 * 64 = 256 threads.
-__device__ __forceinline__ void bw2_invert_lower(const float* A, float* T, int ldt) {
-    const int col = threadIdx.x >> 2, part = threadIdx.x & 3;
-    for (int r = 0; r < kChunk; ++r) {
-        float acc = 0.f;
-        for (int s = col + part; s < r; s += 4) acc = fmaf(A[r * ldt + s], T[s * ldt + col], acc);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if (part == 0) T[r * ldt + col] = r < col ? 0.f : (r == col ? 1.f : -acc);
-        __syncthreads();
-    }
-}
-
 // (0) One CTA per (chunk slot, head): T and P of the chunk into the workspace.
 template <int DK>
 struct Bw2PrepSmem {  // 4-byte words; the cumulative gate is fp64, transposed [channel][row]
@@ -254,7 +240,7 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_prep_kernel(const Bwd2Pa
         P[r * kChunk + s] = accP[u];
     }
     __syncthreads();
-    bw2_invert_lower(sA, sT, LDT);
+    inv_unit_lower64(sA, sT, LDT, sK);  // K is no longer read: it holds the inverse's scratch
     float* Tg = p.tp + ((size_t)slot * H + h) * 2 * kChunk * kChunk;
     for (int e = tid; e < kChunk * kChunk; e += NT) Tg[e] = sT[(e / kChunk) * LDT + e % kChunk];
 }

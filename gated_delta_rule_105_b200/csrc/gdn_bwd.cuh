@@ -162,18 +162,7 @@ __device__ void bw_chunk_prep(const BwChunk<DK>& c, const BwdParams& p, size_t t
             }
     }
     __syncthreads();
-    // T = (I + A)^-1 row by row, four threads per column (adjacent lanes) splitting each row's sum
-    {
-        const int col = tid >> 2, part = tid & 3;
-        for (int r = 0; r < kChunk; ++r) {
-            float acc = 0.f;
-            for (int s = col + part; s < r; s += 4) acc = fmaf(c.A[r * LDT + s], c.T[s * LDT + col], acc);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (part == 0) c.T[r * LDT + col] = r < col ? 0.f : (r == col ? 1.f : -acc);
-            __syncthreads();
-        }
-    }
+    inv_unit_lower64(c.A, c.T, LDT, c.K);  // K is no longer read: it holds the inverse's scratch
 }
 
 // Loads one chunk as bw_chunk_prep does, but takes T and P from the prep kernel's output (`tp`: T then P,

@@ -209,6 +209,49 @@ __device__ __forceinline__ void blk_tri_TtX(const float* T, const float* X, int 
     blk_keep_row(b, kq, out);
 }
 
+// T = (I + A)^-1 for a strictly lower-triangular 64 x 64 A (row stride ldt), 256 threads, W a [64][ldt] scratch.
+// The four diagonal 16 x 16 blocks by forward substitution, one warp each (16 columns x 2 lanes splitting each
+// row's sum); then the blocks below the diagonal, one block-diagonal at a time (distance d = i - j = 1, 2, 3):
+// W_ij = sum_{k=j}^{i-1} A_ik T_kj, then T_ij = -T_ii W_ij.  Seven block-wide barriers instead of one per row.
+// Every entry of T is written (zero above the diagonal).  Called by every thread of the block.
+__device__ __forceinline__ void inv_unit_lower64(const float* A, float* T, int ldt, float* W) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (warp < 4) {  // diagonal block `warp`
+        const int R = 16 * warp, c = lane & 15, part = lane >> 4;
+        for (int r = 0; r < 16; ++r) {
+            float acc = 0.f;
+            for (int s2 = c + part; s2 < r; s2 += 2) acc = fmaf(A[(R + r) * ldt + R + s2], T[(R + s2) * ldt + R + c], acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+            if (part == 0) T[(R + r) * ldt + R + c] = r < c ? 0.f : (r == c ? 1.f : -acc);
+            __syncwarp();
+        }
+    } else {  // the six blocks above the diagonal are zero
+        for (int e = tid - 128; e < 6 * 256; e += 128) {
+            const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            const int bi = b < 3 ? 0 : (b < 5 ? 1 : 2), bj = b < 3 ? b + 1 : (b < 5 ? b - 1 : 3);
+            T[(16 * bi + r) * ldt + 16 * bj + c] = 0.f;
+        }
+    }
+    __syncthreads();
+    const int r = tid >> 4, c = tid & 15;
+    for (int d = 1; d < 4; ++d) {
+        for (int j = 0; j + d < 4; ++j) {  // W_ij = sum_k A_ik T_kj over the blocks k = j .. i - 1
+            const int i = j + d;
+            float acc = 0.f;
+            for (int kk = 16 * j; kk < 16 * i; ++kk) acc = fmaf(A[(16 * i + r) * ldt + kk], T[kk * ldt + 16 * j + c], acc);
+            W[(16 * i + r) * ldt + 16 * j + c] = acc;
+        }
+        __syncthreads();
+        for (int j = 0; j + d < 4; ++j) {  // T_ij = -T_ii W_ij (T_ii unit lower triangular)
+            const int i = j + d;
+            float acc = 0.f;
+            for (int t = 0; t <= r; ++t) acc = fmaf(T[(16 * i + r) * ldt + 16 * i + t], W[(16 * i + t) * ldt + 16 * j + c], acc);
+            T[(16 * i + r) * ldt + 16 * j + c] = -acc;
+        }
+        __syncthreads();
+    }
+}
+
 // A [64][W] block of rows of a bf16 or fp32 tensor (row r at src + r * row_stride elements), held as raw 16-byte
 // vectors in the loading thread's registers: loaded while the previous chunk computes, stored (as fp32) into
 // shared memory once its buffers are free.  Rows at or past Lc are zero.
