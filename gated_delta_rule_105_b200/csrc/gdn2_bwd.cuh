@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_states_kernel(const Bwd2
         __syncthreads();
         {  // X = w . V - (E . F) h (KDA: w = beta of the row); sX holds w until the thread's own tile is read
             float a[2][4] = {};
-            tile_acc_AD<LDK>(sEF, sH, DK, a);
+            tile_acc_AD_split<DK, LDK>(sEF, sH, a);
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int s = s0 + u;
@@ -508,7 +508,7 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_dh_kernel(const Bwd2Para
             for (int u = 0; u < 2; ++u)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) a[u][c] *= p.scale;
-            tile_acc_AD<LDK>(sKf, sDh, DK, a);
+            tile_acc_AD_split<DK, LDK>(sKf, sDh, a);
 #pragma unroll
             for (int u = 0; u < 2; ++u) sts4(sDu + (s0 + u) * LDV + tj, a[u][0], a[u][1], a[u][2], a[u][3]);
         }

@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams 
         {  // dU = scale P^T dO + diag(f) K dh'
             float a[2][4] = {}, b[2][4] = {};
             tile_acc_AtX<LDT>(sP, sDo, wr, a);
-            tile_acc_AD<LDK>(sK, sDh, DK, b);
+            tile_acc_AD_split<DK, LDK>(sK, sDh, b);
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const float fs = sf[s0 + u];

@@ -69,6 +69,39 @@ __device__ __forceinline__ void tile_acc_AD(const float* A, const float* D, int 
     }
 }
 
+// The same product over the full key width DK, as 4 x 4 blocks (rows 4 (tid / 16) .. + 3, the thread's columns) whose
+// sum over i is split between the two lanes 8 apart (each sums half of DK); a shuffle combines the halves and
+// each lane adds its own two rows s0, s0 + 1 to acc.  One 16-byte load feeds 16 FMAs instead of 8.  Called by
+// every thread of the warp.
+template <int DK, int LDA>
+__device__ __forceinline__ void tile_acc_AD_split(const float* A, const float* D, float (&acc)[2][4]) {
+    const int j0 = tile_j0(), pb = 4 * (threadIdx.x >> 4), kq = (threadIdx.x >> 3) & 1;
+    float b[4][4] = {};
+#pragma unroll 2
+    for (int i = kq * (DK / 2); i < (kq + 1) * (DK / 2); i += 4) {
+        float4 d[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) d[q] = lds4(D + (i + q) * kTileLdv + j0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float4 a = lds4(A + (pb + u) * LDA + i);
+            fma4(b[u], a.x, d[0]);
+            fma4(b[u], a.y, d[1]);
+            fma4(b[u], a.z, d[2]);
+            fma4(b[u], a.w, d[3]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) b[u][q] += __shfl_xor_sync(0xffffffffu, b[u][q], 8);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        acc[0][q] += kq == 0 ? b[0][q] : b[2][q];
+        acc[1][q] += kq == 0 ? b[1][q] : b[3][q];
+    }
+}
+
 // The thread's tile of a [DK][32] result: rows i0 .. i0 + DK/32 - 1, columns j0 .. j0 + 3.
 template <int DK>
 __device__ __forceinline__ int tile_i0() { return (DK / 32) * (threadIdx.x >> 3); }
