@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_states_kernel(const Bwd2
                 a[u][2] = lam * d.z;
                 a[u][3] = lam * d.w;
             }
-            tile_acc_KtX<DK, LDK>(sKf, sU, a);
+            tile_acc_KtX_split<DK, LDK>(sKf, sU, nullptr, nullptr, a);
 #pragma unroll
             for (int u = 0; u < IP; ++u) sts4(sH + (i0 + u) * LDV + tj, a[u][0], a[u][1], a[u][2], a[u][3]);
         }
@@ -536,8 +536,7 @@ __global__ void __launch_bounds__(kBw2Threads) gdn2_bwd_dh_kernel(const Bwd2Para
                 a[u][2] = lam * d.z;
                 a[u][3] = lam * d.w;
             }
-            tile_acc_KtX<DK, LDK>(sQF, sDo, a);
-            tile_acc_KtX<DK, LDK>(sEF, sDx, a);
+            tile_acc_KtX_split<DK, LDK>(sQF, sDo, sEF, sDx, a);
 #pragma unroll
             for (int u = 0; u < IP; ++u) sts4(sDh + (i0 + u) * LDV + tj, a[u][0], a[u][1], a[u][2], a[u][3]);
         }

@@ -398,8 +398,7 @@ __global__ void __launch_bounds__(kBwThreads) gdn_bwd_dh_kernel(const BwdParams 
                 a[u][2] = gam * d.z;
                 a[u][3] = gam * d.w;
             }
-            tile_acc_KtX<DK, LDK>(sQ, sDo, a);
-            tile_acc_KtX<DK, LDK>(sK, sDx, a);
+            tile_acc_KtX_split<DK, LDK>(sQ, sDo, sK, sDx, a);
 #pragma unroll
             for (int u = 0; u < IP; ++u) sts4(sDh + (i0 + u) * LDV + tj, a[u][0], a[u][1], a[u][2], a[u][3]);
         }

@@ -128,6 +128,47 @@ __device__ __forceinline__ void tile_acc_KtX(const float* A, const float* X, flo
     }
 }
 
+// acc += A1^T X1 (+ A2^T X2 when A2 is given) on the thread's [DK][32] tile, for DK = 128 as 8 x 4 blocks (channels
+// 8 (tid / 16) .. + 7, the thread's columns) whose sum over the 64 rows is split between the two lanes 8 apart; one
+// shuffle combines the halves of both products and each lane adds its own four channels.  12 wavefronts feed 32
+// FMAs per lane instead of 8 feeding 16.  Other widths use tile_acc_KtX.  Called by every thread of the warp.
+template <int DK, int LDA>
+__device__ __forceinline__ void tile_acc_KtX_split(const float* A1, const float* X1, const float* A2, const float* X2,
+                                                   float (&acc)[DK / 32][4]) {
+    if constexpr (DK != 128) {
+        tile_acc_KtX<DK, LDA>(A1, X1, acc);
+        if (A2) tile_acc_KtX<DK, LDA>(A2, X2, acc);
+    } else {
+        const int j0 = tile_j0(), cb = 8 * (threadIdx.x >> 4), kq = (threadIdx.x >> 3) & 1;
+        float b[8][4] = {};
+        for (int pass = 0; pass < (A2 ? 2 : 1); ++pass) {
+            const float* A = pass ? A2 : A1;
+            const float* X = pass ? X2 : X1;
+#pragma unroll 4
+            for (int r = 32 * kq; r < 32 * kq + 32; ++r) {
+                const float4 x = lds4(X + r * kTileLdv + j0);
+                const float4 a0 = lds4(A + r * LDA + cb), a1 = lds4(A + r * LDA + cb + 4);
+                fma4(b[0], a0.x, x);
+                fma4(b[1], a0.y, x);
+                fma4(b[2], a0.z, x);
+                fma4(b[3], a0.w, x);
+                fma4(b[4], a1.x, x);
+                fma4(b[5], a1.y, x);
+                fma4(b[6], a1.z, x);
+                fma4(b[7], a1.w, x);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) b[u][q] += __shfl_xor_sync(0xffffffffu, b[u][q], 8);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[u][q] += kq == 0 ? b[u][q] : b[u + 4][q];
+    }
+}
+
 // Eight consecutive inputs (bf16 or fp32, 16-byte aligned) as floats.
 __device__ __forceinline__ void ldg8(const float* src, float (&o)[8]) {
     const float4 a = __ldg(reinterpret_cast<const float4*>(src)), b = __ldg(reinterpret_cast<const float4*>(src) + 1);
